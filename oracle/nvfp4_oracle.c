@@ -1,0 +1,332 @@
+/*
+ * nvfp4_oracle.c -- plain, slow, obviously-correct CPU statement of the NVFP4
+ * W4A4 quantized linear layer.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check and the CPU
+ * baseline leg of the benchmark may load this library.  It shares no code,
+ * header, table or constant generator with the CUDA path, and the CUDA path
+ * never calls it.
+ *
+ * Sources (the web pages on "Why Gated DeltaNet Survives 4-Bit Quantization:
+ * NVFP4 W4A4 for the Recurrent Half of a Hybrid 27B LLM"):
+ *   - evolve.pub review, "Report preview / Scope & Claims": NVFP4 W4A4 means
+ *     E2M1 values with one E4M3 scale per 16-element block, applied to both
+ *     weights and activations of every linear layer.
+ *   - thevalue.engineering news page, second section: the same format
+ *     (4-bit E2M1 values, an E4M3 scale per 16-element block) for native
+ *     execution.
+ *   - chatpaper.ai abstract: per-module-calibrated checkpoints served by
+ *     kernels that fuse several modules into one GEMM suffer a global-scale
+ *     mismatch, which the paper repairs.
+ * The pages print no formula.  Where they are silent the oracle takes the
+ * plainest reading consistent with the public NVFP4 definition:
+ *   g   = fl32(amax / (6 * 448))                   (per-tensor FP32 scale)
+ *   s8  = E4M3_RNE_satfinite(fl32(fl32(blockmax / 6) / g))
+ *   d   = fl32(E4M3(s8) * g)
+ *   q   = E2M1_RNE_satfinite(fl32(x / d))          (all 0 if d == 0)
+ *   Y   = bf16_RNE( gA * gW[seg(n)] * sum_k qa*sa * qw*sw )  (sum in FP64)
+ *
+ * Every floating-point step of the quantizer is one IEEE binary32 operation
+ * written out separately; the file is compiled with -ffp-contract=off so no
+ * step is fused or reassociated.  The E2M1 and E4M3 encoders are exhaustive
+ * nearest-value searches over the format's value tables (ties to the even
+ * code), not bit tricks.  The GEMM is a plain FP64 dot product in k order.
+ *
+ * No parity claim rests on an unpinned function: each one is pinned by the
+ * CPU tests against closed forms, brute force, torch's float8_e4m3fn cast or
+ * invariants of the format.
+ */
+#include <stdint.h>
+#include <string.h>
+#include <math.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* ---------------------------------------------------------------------- */
+/* Formats                                                                 */
+/* ---------------------------------------------------------------------- */
+
+/* E2M1 magnitudes for codes 0..7 (1 sign bit, 2 exponent bits, 1 mantissa
+ * bit, exponent bias 1; code 1 is the single subnormal).  Bit 3 is the sign.
+ * Source: the E2M1 element format named on the evolve.pub review (Scope &
+ * Claims) and the thevalue.engineering page. */
+static const double E2M1_MAG[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+
+double oracle_e2m1_value(int code)
+{
+    double m = E2M1_MAG[code & 7];
+    return (code & 8) ? -m : m;
+}
+
+/* Unsigned E4M3 ("E4M3FN" without the sign): exponent bias 7, subnormals
+ * k * 2^-9, largest finite 448 (code 0x7E); 0x7F is NaN and is never
+ * produced by the encoder.  Bit 7 (the sign) is always 0 for block scales. */
+double oracle_e4m3_value(int code)
+{
+    int e = (code >> 3) & 15;
+    int m = code & 7;
+    double v;
+    if ((code & 0x7F) == 0x7F) return NAN;
+    if (e == 0) v = ldexp((double)m, -9);
+    else        v = ldexp(1.0 + m / 8.0, e - 7);
+    return (code & 0x80) ? -v : v;
+}
+
+/* E2M1 round-to-nearest-even with saturation: the code whose value is nearest
+ * to t; on a tie the even code (mantissa bit 0) wins.  Magnitudes beyond 6
+ * (infinity included) saturate to 6.  The sign bit is taken from t
+ * itself, so a negative t that rounds to magnitude 0 gives code 0x8. */
+int oracle_e2m1_encode(float t)
+{
+    double a = fabs((double)t);
+    if (a > 6.0) a = 6.0;      /* satfinite: beyond the largest value (incl. inf) */
+    int best = 0;
+    double best_d = fabs(a - E2M1_MAG[0]);
+    for (int c = 1; c < 8; ++c) {
+        double dist = fabs(a - E2M1_MAG[c]);
+        if (dist < best_d || (dist == best_d && (c & 1) == 0 && (best & 1) == 1)) {
+            best = c;
+            best_d = dist;
+        }
+    }
+    return signbit(t) ? (best | 8) : best;
+}
+
+/* Unsigned E4M3 round-to-nearest-even with saturation to 448: nearest over the
+ * 127 finite non-negative codes 0x00..0x7E, tie to the even code.  s must be
+ * >= 0 (block scales are magnitudes). */
+int oracle_e4m3_encode(float s)
+{
+    double a = (double)s;
+    if (a > 448.0) a = 448.0;  /* satfinite: beyond the largest value (incl. inf) */
+    int best = 0;
+    double best_d = fabs(a - oracle_e4m3_value(0));
+    for (int c = 1; c <= 0x7E; ++c) {
+        double dist = fabs(a - oracle_e4m3_value(c));
+        if (dist < best_d || (dist == best_d && (c & 1) == 0 && (best & 1) == 1)) {
+            best = c;
+            best_d = dist;
+        }
+    }
+    return best;
+}
+
+/* BF16 bit pattern -> float (exact: BF16 is the top half of binary32). */
+static float bf16_to_float(uint16_t b)
+{
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, 4);
+    return f;
+}
+
+/* double -> BF16 with ONE round-to-nearest-even step (no detour through
+ * binary32, which would round twice).  BF16: 8 significant bits, exponent
+ * range of binary32, subnormal spacing 2^-133.  Overflow gives +-inf. */
+uint16_t oracle_bf16_from_double(double x)
+{
+    uint16_t sign = signbit(x) ? 0x8000 : 0;
+    double a = fabs(x);
+    if (isnan(x)) return 0x7FC0;
+    if (a == 0.0) return sign;
+    int e;
+    frexp(a, &e);              /* a = f * 2^e, f in [0.5, 1) -> 2^(e-1) <= a */
+    int ulp_exp = (e - 1) - 7; /* spacing of an 8-bit significand */
+    if (ulp_exp < -133) ulp_exp = -133;
+    double q = nearbyint(ldexp(a, -ulp_exp)); /* default mode: nearest-even */
+    double r = ldexp(q, ulp_exp);
+    if (r > 3.3895313892515355e38) return sign | 0x7F80; /* beyond bf16 max */
+    /* r is exactly a BF16 value; read its top 16 bits through binary32 */
+    float f = (float)r;
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    return sign | (uint16_t)((u >> 16) & 0x7FFF);
+}
+
+/* ---------------------------------------------------------------------- */
+/* Step 1: per-tensor global scale                                         */
+/* ---------------------------------------------------------------------- */
+
+/* amax = max |x| over the whole tensor; g = fl32(amax / 2688), 2688 = 6*448
+ * being the largest magnitude an E2M1 value times an E4M3 scale can hold.
+ * An all-zero tensor gets g = 1 so that later divisions stay finite.
+ * Source: the per-module global scale implied by the chatpaper.ai abstract
+ * ("per-module-calibrated NVFP4 checkpoints", "global-scale mismatch") and
+ * the evolve.pub review (Key claims, fourth bullet); the absmax reading is
+ * the plainest one for a dynamic activation scale. */
+float oracle_global_scale(const uint16_t* x, int64_t rows, int64_t cols,
+                          int64_t ld, float* amax_out)
+{
+    float amax = 0.0f;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t c = 0; c < cols; ++c) {
+            float v = fabsf(bf16_to_float(x[r * ld + c]));
+            if (v > amax) amax = v;
+        }
+    if (amax_out) *amax_out = amax;
+    if (amax == 0.0f) return 1.0f;
+    float g = amax / 2688.0f;
+    return g;
+}
+
+/* ---------------------------------------------------------------------- */
+/* Steps 2-3: 16-element block scales and E2M1 codes                       */
+/* ---------------------------------------------------------------------- */
+
+/* Quantize a BF16 [rows, cols] tensor (row stride ld elements) under global
+ * scale g.  For each row and each block of 16 consecutive elements:
+ *   ab  = max |x| over the block
+ *   sf  = fl32(fl32(ab / 6) / g);   s8 = E4M3_RNE_sat(sf)
+ *   d   = fl32(E4M3(s8) * g)
+ *   code_i = 0 if d == 0, else E2M1_RNE_sat(fl32(x_i / d))
+ * Codes are packed two per byte, element 2j in the low nibble of byte j:
+ * codes[r * (cols/2) + j].  Scales go to sf_linear[r * (cols/16) + b].
+ * cols must be a multiple of 16.
+ * Source: evolve.pub review (Scope & Claims: E2M1 values, E4M3 scale per
+ * 16-element block); thevalue.engineering page (same format). */
+void oracle_quantize(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld,
+                     float g, uint8_t* codes, uint8_t* sf_linear)
+{
+    int64_t nblk = cols / 16;
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t b = 0; b < nblk; ++b) {
+            const uint16_t* blk = x + r * ld + b * 16;
+            float ab = 0.0f;
+            for (int i = 0; i < 16; ++i) {
+                float v = fabsf(bf16_to_float(blk[i]));
+                if (v > ab) ab = v;
+            }
+            float sf = ab / 6.0f;
+            sf = sf / g;
+            int s8 = oracle_e4m3_encode(sf);
+            sf_linear[r * nblk + b] = (uint8_t)s8;
+            float d = (float)oracle_e4m3_value(s8) * g;
+            for (int i = 0; i < 16; i += 2) {
+                int c0 = 0, c1 = 0;
+                if (d != 0.0f) {
+                    float t0 = bf16_to_float(blk[i]) / d;
+                    float t1 = bf16_to_float(blk[i + 1]) / d;
+                    c0 = oracle_e2m1_encode(t0);
+                    c1 = oracle_e2m1_encode(t1);
+                }
+                codes[r * (cols / 2) + b * 8 + i / 2] = (uint8_t)(c0 | (c1 << 4));
+            }
+        }
+    }
+}
+
+/* ---------------------------------------------------------------------- */
+/* Scale-factor layout used by the block-scaled tensor-core MMA            */
+/* ---------------------------------------------------------------------- */
+
+/* Byte offset of scale (r, c) -- row r, 16-block column c -- in the
+ * tensor-core scale-factor layout: rows are grouped in 128-row blocks and
+ * scale columns in groups of 4; each (128 x 4) group is a 512-byte atom,
+ * atoms ordered with the scale-column group fastest, and inside an atom
+ * row r sits at (r % 32) * 16 + ((r / 32) % 4) * 4 and column c at c % 4.
+ * sfcols_padded = (cols/16) rounded up to a multiple of 4.
+ * This is the public block-scale layout of the PTX ISA block-scaling
+ * section; the pages do not describe a memory layout. */
+int64_t oracle_sf_offset_tcgen05(int64_t r, int64_t c, int64_t sfcols_padded)
+{
+    int64_t atom = (r / 128) * (sfcols_padded / 4) + (c / 4);
+    int64_t inner = (r % 32) * 16 + ((r / 32) % 4) * 4 + (c % 4);
+    return atom * 512 + inner;
+}
+
+/* Re-lay a linear [rows, sfcols] scale matrix into the tensor-core layout.
+ * out must hold (rows rounded up to 128) * (sfcols rounded up to 4) bytes;
+ * padding bytes are written as 0. */
+void oracle_sf_to_tcgen05(const uint8_t* sf_linear, int64_t rows, int64_t sfcols,
+                          uint8_t* out)
+{
+    int64_t rows_p = (rows + 127) / 128 * 128;
+    int64_t cols_p = (sfcols + 3) / 4 * 4;
+    memset(out, 0, (size_t)(rows_p * cols_p));
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t c = 0; c < sfcols; ++c)
+            out[oracle_sf_offset_tcgen05(r, c, cols_p)] = sf_linear[r * sfcols + c];
+}
+
+/* ---------------------------------------------------------------------- */
+/* Step 4: dequantization and the block-scaled GEMM                        */
+/* ---------------------------------------------------------------------- */
+
+/* xq[r, k] = E2M1(code) * E4M3(s8 of the block), WITHOUT the global scale,
+ * in FP64 (exact: a 2-bit by 4-bit significand product). */
+void oracle_dequantize_noglobal(const uint8_t* codes, const uint8_t* sf_linear,
+                                int64_t rows, int64_t cols, double* out)
+{
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t k = 0; k < cols; ++k) {
+            uint8_t byte = codes[r * (cols / 2) + k / 2];
+            int code = (k % 2 == 0) ? (byte & 15) : (byte >> 4);
+            double s = oracle_e4m3_value(sf_linear[r * (cols / 16) + k / 16]);
+            out[r * cols + k] = oracle_e2m1_value(code) * s;
+        }
+}
+
+/* Y[m, n] = alpha[n] * sum_k A[m, k] * W[n, k] in FP64, k in increasing
+ * order; A and W are dequantized operands without global scales and
+ * alpha[n] = gA * gW[seg(n)] (an FP64 product of the two FP32 scales).
+ * Only the rows listed in row_ids (n_rows of them) are computed; out is
+ * [n_rows, N].  Source: W4A4 GEMM of the chatpaper.ai abstract and the
+ * evolve.pub FAQ ("running natively on NVFP4-capable hardware"); the
+ * per-column alpha is the per-module global scale of the fused-GEMM repair
+ * (chatpaper.ai abstract; evolve.pub Key claims, fourth bullet). */
+void oracle_gemm_f64(const double* A, const double* W, const double* alpha,
+                     int64_t N, int64_t K, const int64_t* row_ids, int64_t n_rows,
+                     double* out)
+{
+    #pragma omp parallel for schedule(dynamic)
+    for (int64_t i = 0; i < n_rows; ++i) {
+        const double* a = A + row_ids[i] * K;
+        for (int64_t n = 0; n < N; ++n) {
+            const double* w = W + n * K;
+            double acc = 0.0;
+            for (int64_t k = 0; k < K; ++k) acc += a[k] * w[k];
+            out[i * N + n] = alpha[n] * acc;
+        }
+    }
+}
+
+/* Round an FP64 matrix to BF16 bit patterns (one RNE step per element). */
+void oracle_bf16_round(const double* y, int64_t n, uint16_t* out)
+{
+    for (int64_t i = 0; i < n; ++i) out[i] = oracle_bf16_from_double(y[i]);
+}
+
+/* ---------------------------------------------------------------------- */
+/* Array helpers for the Python wrapper (plain loops over the above)       */
+/* ---------------------------------------------------------------------- */
+
+void oracle_e2m1_encode_array(const float* t, int64_t n, uint8_t* out)
+{
+    for (int64_t i = 0; i < n; ++i) out[i] = (uint8_t)oracle_e2m1_encode(t[i]);
+}
+
+void oracle_e4m3_encode_array(const float* s, int64_t n, uint8_t* out)
+{
+    for (int64_t i = 0; i < n; ++i) out[i] = (uint8_t)oracle_e4m3_encode(s[i]);
+}
+
+void oracle_bf16_from_double_array(const double* x, int64_t n, uint16_t* out)
+{
+    for (int64_t i = 0; i < n; ++i) out[i] = oracle_bf16_from_double(x[i]);
+}
+
+int oracle_num_threads(void)
+{
+#ifdef _OPENMP
+    int n = 1;
+    #pragma omp parallel
+    {
+        #pragma omp single
+        n = omp_get_num_threads();
+    }
+    return n;
+#else
+    return 1;
+#endif
+}

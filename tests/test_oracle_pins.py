@@ -1,0 +1,421 @@
+"""Pins of the CPU oracle against what the format and the mathematics fix.
+
+None of these re-types the oracle's own algorithm: each pin uses another route
+-- the format's bit-field definition, torch's float8_e4m3fn cast (a library
+round-to-nearest-even), exact rational arithmetic, hand-derived worked
+examples under tests/golden/, invariants (monotonicity, nearest-value, error
+bounds) and closed forms (one-hot GEMMs, segment scaling) -- so that a dropped
+term, a wrong sign or index, or a transposed operand in the oracle fails here.
+"""
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from conftest import read_golden
+
+pytestmark = pytest.mark.filterwarnings("ignore::DeprecationWarning")
+
+
+def f32(x):
+    return np.float32(x)
+
+
+def all_bf16_nonneg_finite():
+    bits = np.arange(0, 0x7F80, dtype=np.uint32)  # +0 .. largest finite
+    return (bits << 16).view(np.float32)
+
+
+# ---------------------------------------------------------------------------
+# E2M1 element format
+# ---------------------------------------------------------------------------
+
+def e2m1_from_fields(code):
+    """E2M1 value from its bit fields: sign | 2-bit exponent | 1-bit mantissa."""
+    s = -1.0 if code & 8 else 1.0
+    e = (code >> 1) & 3
+    m = code & 1
+    if e == 0:
+        return s * (m / 2.0) * 2.0 ** (1 - 1)
+    return s * (1.0 + m / 2.0) * 2.0 ** (e - 1)
+
+
+def test_e2m1_values_golden(golden_dir):
+    for line in read_golden(os.path.join(golden_dir, "e2m1_values.txt")):
+        code, val = line.split()
+        got = oracle.e2m1_value(int(code))
+        assert got == float(val) and math.copysign(1, got) == math.copysign(1, float(val))
+        assert got == e2m1_from_fields(int(code))
+
+
+def test_e2m1_rne_golden(golden_dir):
+    for line in read_golden(os.path.join(golden_dir, "e2m1_rne_points.txt")):
+        t, code = line.split()
+        assert int(oracle.e2m1_encode(np.array([float(t)], np.float32))[0]) == int(code), t
+
+
+def test_e2m1_roundtrip_representable():
+    vals = np.array([e2m1_from_fields(c) for c in range(16) if c != 8], np.float32)
+    codes = oracle.e2m1_encode(vals)
+    back = np.array([oracle.e2m1_value(int(c)) for c in codes])
+    assert np.array_equal(back, vals.astype(np.float64))
+
+
+def _nearest_dist(t):
+    grid = np.array([0, .5, 1, 1.5, 2, 3, 4, 6])
+    return np.min(np.abs(np.minimum(np.abs(t.astype(np.float64)), 6.0)[:, None] - grid[None, :]), axis=1)
+
+
+@pytest.mark.parametrize("d", [1.0, 0.5, 2.0 ** -7, 3.0, 1.0 / 3.0])
+def test_e2m1_exhaustive_bf16_nearest_and_monotone(d):
+    # every non-negative finite BF16 divided by d (an FP32 division, as in the
+    # quantizer); the chosen value must be a nearest one, ties to an even code,
+    # and the map must be monotone in t.
+    with np.errstate(over="ignore"):
+        t = (all_bf16_nonneg_finite() / np.float32(d)).astype(np.float32)
+    codes = oracle.e2m1_encode(t)
+    vals = np.array([oracle.e2m1_value(c) for c in range(8)])[codes & 7]
+    err = np.abs(np.minimum(t.astype(np.float64), 6.0) - vals)
+    best = _nearest_dist(t)
+    assert np.all(err == best)
+    tie = np.isclose(err, best) & (err > 0)
+    # at exact midpoints both neighbours are at distance err: the even code wins
+    grid = np.array([0, .5, 1, 1.5, 2, 3, 4, 6])
+    mids = (grid[1:] + grid[:-1]) / 2
+    at_mid = np.isin(t.astype(np.float64), mids)
+    assert np.all((codes[at_mid & tie] & 1) == 0)
+    order = np.argsort(t, kind="stable")
+    assert np.all(np.diff(vals[order]) >= 0)
+    # negative inputs mirror positive ones with the sign bit set
+    cn = oracle.e2m1_encode(-t)
+    assert np.array_equal(cn, codes | 8)
+
+
+def test_e2m1_saturates_and_keeps_sign_of_zero():
+    t = np.array([6.0, 6.0001, 1e38, np.inf, -np.inf, -0.0, 0.0, -1e-30], np.float32)
+    assert list(oracle.e2m1_encode(t)) == [7, 7, 7, 7, 15, 8, 0, 8]
+
+
+# ---------------------------------------------------------------------------
+# E4M3 scale format
+# ---------------------------------------------------------------------------
+
+def e4m3_from_fields(code):
+    e = (code >> 3) & 15
+    m = code & 7
+    if e == 0:
+        return m * 2.0 ** -9
+    return (1 + m / 8.0) * 2.0 ** (e - 7)
+
+
+def test_e4m3_values_fields_and_torch():
+    codes = np.arange(0, 0x7F, dtype=np.uint8)
+    lib = torch.from_numpy(codes.copy()).view(torch.float8_e4m3fn).float().numpy()
+    for c in codes:
+        v = oracle.e4m3_value(int(c))
+        assert v == e4m3_from_fields(int(c)) == float(lib[c])
+    assert oracle.e4m3_value(0x7E) == 448.0
+    assert math.isnan(oracle.e4m3_value(0x7F))
+
+
+def test_e4m3_rne_golden(golden_dir):
+    for line in read_golden(os.path.join(golden_dir, "e4m3_rne_points.txt")):
+        v, code = line.split()
+        assert int(oracle.e4m3_encode(np.array([float(v)], np.float32))[0]) == int(code, 16), v
+
+
+def test_e4m3_encode_matches_torch_cast_exhaustive_bf16():
+    s = all_bf16_nonneg_finite()
+    s = s[s < 464.0]                 # torch's cast has no saturation above this
+    ours = oracle.e4m3_encode(s)
+    ref = torch.from_numpy(s.copy()).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(ours, ref)
+
+
+def test_e4m3_encode_matches_torch_cast_random_fp32():
+    rng = np.random.default_rng(123)
+    s = np.concatenate([rng.uniform(0, 463.99, 400_000),
+                        np.exp(rng.uniform(np.log(1e-6), np.log(460), 400_000))]).astype(np.float32)
+    ours = oracle.e4m3_encode(s)
+    ref = torch.from_numpy(s.copy()).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(ours, ref)
+
+
+def test_e4m3_saturates_at_448():
+    s = np.array([448.0, 463.9, 464.0, 500.0, 3e38, np.inf], np.float32)
+    assert np.all(oracle.e4m3_encode(s) == 0x7E)
+
+
+# ---------------------------------------------------------------------------
+# FP64 -> BF16 single rounding
+# ---------------------------------------------------------------------------
+
+def test_bf16_round_matches_torch_on_fp32_inputs():
+    rng = np.random.default_rng(7)
+    x = (rng.standard_normal(200_000) * np.exp(rng.uniform(-30, 30, 200_000))).astype(np.float32)
+    ours = oracle.bf16_from_double(x.astype(np.float64))
+    ref = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(ours, ref)
+
+
+def test_bf16_round_single_step_ties_and_overflow():
+    one = 1.0
+    ulp = 2.0 ** -7
+    cases = [
+        (one + ulp / 2, 0x3F80),                 # tie -> even (1.0)
+        (one + 3 * ulp / 2, 0x3F82),             # tie -> even (1 + 2ulp)
+        (one + ulp / 2 + 2.0 ** -40, 0x3F81),    # just above the tie: up (a
+                                                 # detour through FP32 would tie)
+        (-(one + ulp / 2 + 2.0 ** -40), 0xBF81),
+        (3.4e38, 0x7F80),                        # rounds past the largest finite
+        (3.3895313892515355e38, 0x7F7F),
+        (0.0, 0x0000), (-0.0, 0x8000),
+        (2.0 ** -133, 0x0001),                   # smallest BF16 subnormal
+        (2.0 ** -134, 0x0000),                   # tie with zero -> even (zero)
+        (1.5 * 2.0 ** -133, 0x0002),             # tie between 1 and 2 -> 2
+    ]
+    for x, want in cases:
+        assert int(oracle.bf16_from_double(np.array([x]))[0]) == want, x
+
+
+# ---------------------------------------------------------------------------
+# Step 1: global scale
+# ---------------------------------------------------------------------------
+
+def bf16_bits_of(arr):
+    return torch.from_numpy(np.asarray(arr, np.float32)).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+def test_global_scale_zero_tensor():
+    g, amax = oracle.global_scale(np.zeros((3, 32), np.uint16))
+    assert g == 1.0 and amax == 0.0
+
+
+def test_global_scale_is_correctly_rounded_quotient():
+    rng = np.random.default_rng(5)
+    for trial in range(50):
+        x = rng.standard_normal((7, 48)).astype(np.float32) * np.float32(10 ** rng.uniform(-20, 20))
+        bits = bf16_bits_of(x)
+        g, amax = oracle.global_scale(bits)
+        vals = oracle.bf16_bits_to_f64(bits)
+        assert amax == np.max(np.abs(vals))           # exact maximum
+        q = Fraction(float(amax)) / 2688
+        lo = np.nextafter(g, np.float32(0), dtype=np.float32)
+        hi = np.nextafter(g, np.float32(np.inf), dtype=np.float32)
+        dg = abs(Fraction(float(g)) - q)
+        assert dg <= abs(Fraction(float(lo)) - q) and dg <= abs(Fraction(float(hi)) - q)
+
+
+def test_global_scale_closed_forms():
+    for amax, want in [(2688.0, 1.0), (1344.0, 0.5), (6.0 * 448.0 * 2 ** -20, 2 ** -20)]:
+        x = np.zeros((2, 32), np.float32)
+        x[1, 5] = -amax
+        g, a = oracle.global_scale(bf16_bits_of(x))
+        assert a == amax and g == np.float32(want)
+
+
+# ---------------------------------------------------------------------------
+# Steps 2-3: block scales and codes
+# ---------------------------------------------------------------------------
+
+def test_quantize_worked_blocks(golden_dir):
+    for line in read_golden(os.path.join(golden_dir, "quantize_worked_blocks.txt")):
+        name, g, vals, s8, codes = [p.strip() for p in line.split("|")]
+        x = np.array([float(v) for v in vals.split()], np.float32)[None, :]
+        bits = bf16_bits_of(x)
+        assert np.array_equal(oracle.bf16_bits_to_f64(bits)[0], x[0].astype(np.float64)), name
+        c, sf = oracle.quantize(bits, float(g))
+        assert int(sf[0, 0]) == int(s8, 16), name
+        assert [int(b) for b in c[0]] == [int(h, 16) for h in codes.split()], name
+
+
+def test_absmax_block_gets_largest_scale():
+    rng = np.random.default_rng(11)
+    for _ in range(20):
+        x = (rng.standard_t(3, (9, 64)) * 10 ** rng.uniform(-3, 3)).astype(np.float32)
+        bits = bf16_bits_of(x)
+        g, amax = oracle.global_scale(bits)
+        _, sf = oracle.quantize(bits, g)
+        vals = np.abs(oracle.bf16_bits_to_f64(bits))
+        r, c = np.unravel_index(np.argmax(vals), vals.shape)
+        assert sf[r, c // 16] == 0x7E
+
+
+def test_block_scale_tracks_absmax_over_6():
+    # dec(s8) * g is within the E4M3 half-spacing of (block absmax / 6)
+    rng = np.random.default_rng(3)
+    x = (rng.standard_t(3, (64, 256)) * np.exp(rng.uniform(-4, 4, (64, 1)))).astype(np.float32)
+    bits = bf16_bits_of(x)
+    g, _ = oracle.global_scale(bits)
+    _, sf = oracle.quantize(bits, g)
+    vals = np.abs(oracle.bf16_bits_to_f64(bits)).reshape(64, 16, 16)
+    ab = vals.max(axis=2)
+    target = ab / 6.0 / float(g)
+    dec = np.vectorize(oracle.e4m3_value)(sf)
+    normal = target >= 2.0 ** -6
+    assert np.all(np.abs(dec[normal] - target[normal]) <= target[normal] * 2.0 ** -4 * (1 + 1e-6))
+    assert np.all(np.abs(dec[~normal] - target[~normal]) <= 2.0 ** -10 * (1 + 1e-6))
+
+
+def test_dequantization_error_bound():
+    # |x - xhat| <= half the E2M1 spacing at |x/d| times d (plus the FP32
+    # rounding of x/d), or the clip error when |x/d| > 6.
+    rng = np.random.default_rng(9)
+    x = (rng.standard_t(3, (32, 512)) * 0.7).astype(np.float32)
+    x[:, 17] *= 200
+    bits = bf16_bits_of(x)
+    g, _ = oracle.global_scale(bits)
+    codes, sf = oracle.quantize(bits, g)
+    xh = oracle.dequantize_noglobal(codes, sf) * float(g)
+    xv = oracle.bf16_bits_to_f64(bits)
+    d = np.repeat(np.vectorize(oracle.e4m3_value)(sf), 16, axis=1) * float(g)
+    d32 = d.astype(np.float32).astype(np.float64)
+    t = np.abs(xv) / np.where(d32 > 0, d32, 1)
+    half = np.where(t < 2, 0.25, np.where(t < 4, 0.5, 1.0))
+    bound = np.where(t <= 6, half * d32, (t - 6) * d32) * (1 + 1e-6) + 1e-30
+    ok = (d32 == 0) | (np.abs(xv - xh) <= bound + np.abs(d - d32) * 6)
+    assert np.all(ok)
+
+
+def test_nibble_order_low_first():
+    x = np.zeros((1, 16), np.float32)
+    x[0, 0] = 6.0        # -> code 7 in the low nibble of byte 0
+    x[0, 3] = -1.0       # -> code 0xA in the high nibble of byte 1
+    codes, _ = oracle.quantize(bf16_bits_of(x), 1.0)
+    assert codes[0, 0] == 0x07 and codes[0, 1] == 0xA0
+
+
+# ---------------------------------------------------------------------------
+# Scale-factor layout for the tensor cores
+# ---------------------------------------------------------------------------
+
+def test_sf_layout_hand_offsets():
+    # atom = 128 rows x 4 scale columns = 512 B; inner (r%32)*16 + (r//32%4)*4 + c%4
+    cases = [((0, 0), 0), ((1, 0), 16), ((31, 3), 31 * 16 + 3), ((32, 0), 4),
+             ((33, 2), 16 + 4 + 2), ((127, 1), 31 * 16 + 12 + 1), ((0, 4), 512),
+             ((128, 0), 512 * 5)]   # 20 scale columns -> 5 atoms per row block
+    for (r, c), want in cases:
+        assert oracle.sf_offset_tcgen05(r, c, 20) == want
+
+
+def test_sf_layout_bijection_and_padding():
+    rng = np.random.default_rng(1)
+    rows, sfcols = 300, 10          # pads to 384 rows and 12 scale columns
+    sf = rng.integers(1, 255, (rows, sfcols)).astype(np.uint8)
+    out = oracle.sf_to_tcgen05(sf)
+    assert out.size == 384 * 12
+    offs = np.array([[oracle.sf_offset_tcgen05(r, c, 12) for c in range(12)] for r in range(384)])
+    assert np.array_equal(np.sort(offs.ravel()), np.arange(384 * 12))
+    assert np.array_equal(out[offs[:rows, :sfcols]], sf)
+    pad = np.ones(384 * 12, bool)
+    pad[offs[:rows, :sfcols].ravel()] = False
+    assert np.all(out[pad] == 0)
+
+
+# ---------------------------------------------------------------------------
+# Step 4: the GEMM
+# ---------------------------------------------------------------------------
+
+def test_gemm_brute_force_exact_fractions():
+    rng = np.random.default_rng(2)
+    M, N, K = 3, 5, 32
+    A = rng.integers(-6, 7, (M, K)) * 0.5
+    W = rng.integers(-6, 7, (N, K)) * 0.25
+    alpha = np.array([0.75, 1.0, 2.0 ** -9, 3.0, 1.5])
+    y = oracle.gemm_f64(A, W, alpha)
+    for m in range(M):
+        for n in range(N):
+            exact = Fraction(alpha[n]) * sum(Fraction(A[m, k]) * Fraction(W[n, k]) for k in range(K))
+            assert y[m, n] == float(exact)
+
+
+def test_gemm_matches_library_matmul_and_row_subset():
+    rng = np.random.default_rng(4)
+    A = rng.standard_normal((40, 96))
+    W = rng.standard_normal((70, 96))
+    alpha = rng.uniform(0.1, 2, 70)
+    y = oracle.gemm_f64(A, W, alpha)
+    assert np.allclose(y, (A @ W.T) * alpha[None, :], rtol=1e-12, atol=1e-12)
+    rows = np.array([39, 0, 17])
+    assert np.array_equal(oracle.gemm_f64(A, W, alpha, rows), y[rows])
+
+
+def _quant(x32, g=None):
+    bits = bf16_bits_of(x32)
+    if g is None:
+        g, _ = oracle.global_scale(bits)
+    codes, sf = oracle.quantize(bits, g)
+    return codes, sf, np.float32(g)
+
+
+def test_one_hot_gemm_closed_form():
+    # one nonzero per row: Y[m,n] = gA*gW*dec(sA)*dec(sW)*vA*vW
+    M, N, K = 4, 3, 64
+    xa = np.zeros((M, K), np.float32)
+    xw = np.zeros((N, K), np.float32)
+    ka = [0, 17, 33, 63]
+    for m in range(M):
+        xa[m, ka[m]] = [3.0, -1.5, 0.25, 40.0][m]
+    for n in range(N):
+        xw[n, ka] = [0.02, -0.5, 7.0][n]
+    ca, sa, ga = _quant(xa)
+    cw, sw, gw = _quant(xw)
+    y64, _ = oracle.linear(ca, sa, ga, cw, sw, [(0, N, gw)])
+    for m in range(M):
+        k = ka[m]
+        qa = ((ca[m, k // 2] >> (4 * (k % 2))) & 15)
+        for n in range(N):
+            qw = ((cw[n, k // 2] >> (4 * (k % 2))) & 15)
+            want = (float(ga) * float(gw) * oracle.e4m3_value(sa[m, k // 16]) *
+                    oracle.e4m3_value(sw[n, k // 16]) * oracle.e2m1_value(qa) * oracle.e2m1_value(qw))
+            # same factors, another FP64 multiplication order: within 2 ulp
+            assert abs(y64[m, n] - want) <= 4.5e-16 * abs(want)
+    # the one-hot values are recovered to within the E2M1/E4M3 resolution
+    assert abs(y64[0, 0] - 3.0 * 0.02) / (3.0 * 0.02) < 0.15
+
+
+def test_fused_segments_equal_per_module_and_negative_control():
+    rng = np.random.default_rng(8)
+    K = 128
+    x = rng.standard_t(3, (16, K)).astype(np.float32)
+    mods = [(48, 0.02), (16, 0.2), (32, 0.002)]
+    ws = [rng.standard_normal((n, K)).astype(np.float32) * s for n, s in mods]
+    ca, sa, ga = _quant(x)
+    qs = [_quant(w) for w in ws]
+    cw = np.concatenate([q[0] for q in qs])
+    sw = np.concatenate([q[1] for q in qs])
+    segs, off = [], 0
+    for (n, _), q in zip(mods, qs):
+        segs.append((off, n, q[2]))
+        off += n
+    y_fused, yb_fused = oracle.linear(ca, sa, ga, cw, sw, segs)
+    for (o, n, gw), q in zip(segs, qs):
+        y_mod, yb_mod = oracle.linear(ca, sa, ga, q[0], q[1], [(0, n, gw)])
+        assert np.array_equal(y_fused[:, o:o + n], y_mod)
+        assert np.array_equal(yb_fused[:, o:o + n], yb_mod)
+    # a single global scale for the fused GEMM mis-scales every other module by
+    # its scale ratio -- the global-scale mismatch the pages repair
+    y_one, _ = oracle.linear(ca, sa, ga, cw, sw, [(0, off, segs[0][2])])
+    for (o, n, gw) in segs:
+        ratio = float(segs[0][2]) / float(gw)
+        nz = y_fused[:, o:o + n] != 0
+        assert np.allclose(y_one[:, o:o + n][nz] / y_fused[:, o:o + n][nz], ratio, rtol=1e-12)
+    assert float(segs[0][2]) / float(segs[2][2]) > 5      # really different scales
+
+
+def test_quantized_gemm_close_to_bf16_gemm():
+    # NVFP4 keeps a W4A4 GEMM within a few percent of the BF16 one on Gaussian
+    # data (a property of 16-element block scaling, not a parity target)
+    rng = np.random.default_rng(6)
+    x = rng.standard_normal((32, 512)).astype(np.float32)
+    w = (rng.standard_normal((48, 512)) * 0.02).astype(np.float32)
+    ca, sa, ga = _quant(x)
+    cw, sw, gw = _quant(w)
+    y64, _ = oracle.linear(ca, sa, ga, cw, sw, [(0, 48, gw)])
+    ref = oracle.bf16_bits_to_f64(bf16_bits_of(x)) @ oracle.bf16_bits_to_f64(bf16_bits_of(w)).T
+    rel = np.linalg.norm(y64 - ref) / np.linalg.norm(ref)
+    assert 0.01 < rel < 0.2
