@@ -1,0 +1,391 @@
+#!/usr/bin/env python
+"""Benchmark of the NVFP4 W4A4 quantized-linear hot path on B200.
+
+One step = one pass of the whole path over one batch: per-tensor global scale
+of the BF16 activation, its 16-block NVFP4 quantization, and the fused
+multi-module block-scaled FP4 GEMM with per-module global scales in the BF16
+epilogue -- the Gated DeltaNet input projection q/k/v/z/b/a at prefill,
+X [8192, 5120] x W [24704, 5120] (weights quantized once, outside the timed
+region, as a serving stack would).  Metric: whole-job TFLOP/s of the step
+(2*M*N*K per step); the quantizer's GB/s on the [32768, 5120] activation is
+reported beside it.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun every rank runs its own batch (the path is data parallel over
+tokens with replicated weights: no data-path collective, weak scaling); the
+reported time is the max over ranks.  ``--impl reference`` times the plain CPU
+oracle on the host cores instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+M_TOK, K_HID = 8192, 5120
+METRIC = "W4A4 GEMM TFLOPS (% dense FP4 peak); quantize GB/s (% HBM peak)"
+WORKLOAD = "fused GDN input projection prefill: X bf16 [8192,5120] -> W q/k/v/z/b/a [24704,5120]"
+L2_FLUSH_BYTES = 256 << 20
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# clocks: NVML samples of our GPU during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    REASONS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+               "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80}
+
+    def __init__(self, device_index: int, period_s: float = 0.01):
+        self.samples, self.reasons = [], set()
+        self.max_mhz = None
+        self.period = period_s
+        self._stop = threading.Event()
+        self._h = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            props = torch.cuda.get_device_properties(device_index)
+            try:
+                self._h = pynvml.nvmlDeviceGetHandleByUUID("GPU-" + str(props.uuid))
+            except Exception:  # noqa: BLE001
+                bus = "%08x:%02x:%02x.0" % (props.pci_domain_id, props.pci_bus_id,
+                                            props.pci_device_id)
+                self._h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            self._nv = pynvml
+            self._reasons_fn = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # noqa: BLE001 - clocks are best effort
+            self.error = repr(e)
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                r = self._reasons_fn(self._h)
+                for name, bit in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:  # noqa: BLE001
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self._h is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._h is not None:
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": 0}
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+def build_workload(dev):
+    import nvfp4_w4a4_quantized_09_b200 as nv
+    from nvfp4_w4a4_quantized_09_b200 import synth
+    rank = int(os.environ.get("RANK", "0"))
+    x = synth.student_t_activations(M_TOK, K_HID, seed=3 + 1000 * rank, device=dev)
+    ws = [w for _, w in synth.gdn_weights(synth.GDN_MODULES, device=dev)]
+    fw = nv.FusedWeight.from_modules(ws)
+    del ws
+    return x, fw
+
+
+def act_stats(x):
+    xf = x.float()
+    rms = xf.pow(2).mean().sqrt()
+    mx = xf.abs().max()
+    m4 = xf.pow(4).mean()
+    return {"max_over_rms": float(mx / rms), "kurtosis": float(m4 / rms ** 4),
+            "pages_table2": {"max_over_rms": 63.5, "kurtosis": 1564}}
+
+
+def run_ours(args, dev, world, rank):
+    import nvfp4_w4a4_quantized_09_b200 as nv
+    from nvfp4_w4a4_quantized_09_b200 import synth
+    peaks, peak_src = load_peaks()
+    torch.cuda.set_device(dev)
+    x, fw = build_workload(dev)
+    N = fw.rows
+    M, K = x.shape
+    segs = fw.segments()
+    flops = 2.0 * M * N * K
+    stream = torch.cuda.current_stream()
+    g = torch.empty(1, dtype=torch.float32, device=dev)
+    amax = torch.empty(1, dtype=torch.float32, device=dev)
+    codes = torch.empty(M, K // 2, dtype=torch.uint8, device=dev)
+    sf = torch.empty(nv.sf_bytes(M, K), dtype=torch.uint8, device=dev)
+    y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    a = nv.QuantizedTensor(codes, sf, g, M, K)
+
+    def step():
+        nv.global_scale(x, g, amax)
+        nv.quantize(x, g, nv.SF_TCGEN05, codes, sf)
+        nv.fused_gemm(a, fw.codes, fw.sf, segs, y)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        for i in range(args.steps):
+            flush.zero_()                      # L2 flushed between timed steps
+            e0, e1, e2 = ev[i]
+            e0.record(stream)
+            nv.global_scale(x, g, amax)
+            nv.quantize(x, g, nv.SF_TCGEN05, codes, sf)
+            e1.record(stream)
+            nv.fused_gemm(a, fw.codes, fw.sf, segs, y)
+            e2.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    step_ms = [e0.elapsed_time(e2) for e0, _, e2 in ev]
+    gemm_ms = [e1.elapsed_time(e2) for _, e1, e2 in ev]
+    quant_ms = [e0.elapsed_time(e1) for e0, e1, _ in ev]
+    total_ms = float(sum(step_ms))
+    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    value = world * flops * args.steps / (total_ms * 1e-3) / 1e12
+
+    gemm_avg_ms = float(np.mean(gemm_ms))
+    achieved = flops / (gemm_avg_ms * 1e-3) / 1e12
+    fp4_peak = peaks["bf16_tflops"] * 4.0
+    roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(fp4_peak, 1),
+                "unit": "TFLOP/s", "frac": round(achieved / fp4_peak, 4),
+                "traffic": None, "kernel": "nvf4_gemm_kernel (fused, 8192x24704x5120)",
+                "peak_source": f"{peak_src} bf16 burst x 4 (nominal dense FP4/BF16 ratio 9/2.25)"}
+
+    # quantizer alone on the [32768, 5120] activation: global scale + quantize
+    xq = synth.student_t_activations(32768, K_HID, seed=1, device=dev)
+    cq = torch.empty(32768, K_HID // 2, dtype=torch.uint8, device=dev)
+    sq = torch.empty(nv.sf_bytes(32768, K_HID), dtype=torch.uint8, device=dev)
+    qt = []
+    for i in range(args.warmup + 20):
+        flush.zero_()
+        e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        e0.record(stream)
+        nv.global_scale(xq, g, amax)
+        e1.record(stream)
+        nv.quantize(xq, g, nv.SF_TCGEN05, cq, sq)
+        e2.record(stream)
+        qt.append((e0, e1, e2))
+    torch.cuda.synchronize()
+    qt = qt[args.warmup:]
+    n_el = xq.numel()
+    gs_ms = float(np.mean([a.elapsed_time(b) for a, b, _ in qt]))
+    qz_ms = float(np.mean([b.elapsed_time(c) for _, b, c in qt]))
+    hbm = peaks["hbm_gbs"]
+    q_bytes = n_el * 2 + n_el // 2 + n_el // 16
+    quantizer = {
+        "workload": "activation [32768,5120] bf16",
+        "quantize_GBps": round(q_bytes / (qz_ms * 1e-3) / 1e9, 1),
+        "quantize_frac_hbm": round(q_bytes / (qz_ms * 1e-3) / 1e9 / hbm, 4),
+        "global_scale_GBps": round(n_el * 2 / (gs_ms * 1e-3) / 1e9, 1),
+        "global_scale_frac_hbm": round(n_el * 2 / (gs_ms * 1e-3) / 1e9 / hbm, 4),
+        "both_GBps": round((q_bytes + n_el * 2) / ((qz_ms + gs_ms) * 1e-3) / 1e9, 1),
+        "quantize_us": round(qz_ms * 1e3, 2), "global_scale_us": round(gs_ms * 1e3, 2),
+        "hbm_peak_GBps": hbm, "peak_source": peak_src}
+    del xq, cq, sq
+
+    # end to end through the public API with host buffers: pinned X in, Y out
+    x_host = x.cpu().pin_memory()
+    y_host = torch.empty(M, N, dtype=torch.bfloat16).pin_memory()
+    x_dev = torch.empty_like(x)
+    e2e_steps = max(3, min(args.steps, 20))
+    for i in range(2 + e2e_steps):
+        if i == 2:
+            torch.cuda.synchronize()
+            s0 = torch.cuda.Event(enable_timing=True)
+            s0.record(stream)
+        x_dev.copy_(x_host, non_blocking=True)
+        nv.linear(x_dev, fw, y)
+        y_host.copy_(y, non_blocking=True)
+    s1 = torch.cuda.Event(enable_timing=True)
+    s1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = s0.elapsed_time(s1) / e2e_steps
+    e2e = {"value": round(world * flops / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+           "h2d_bytes_per_step": int(x.numel() * 2), "d2h_bytes_per_step": int(y.numel() * 2),
+           "ms_per_step": round(e2e_ms, 3)}
+
+    # sanity (reported, not a target): quantized vs BF16 GEMM on sampled rows
+    rows = torch.arange(0, M, M // 16, device=dev)
+    w_bf16 = torch.cat([w for _, w in synth.gdn_weights(synth.GDN_MODULES, device=dev)])
+    ref = x[rows].float() @ w_bf16.float().t()
+    nv.linear(x, fw, y)
+    torch.cuda.synchronize()
+    sanity = float((y[rows].float() - ref).norm() / ref.norm())
+    del w_bf16
+
+    out = {
+        "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4-e2m1/ue4m3, fp32 accumulate, bf16 out",
+        "data": "synthetic (seeded Student-t nu=3 activations with 8 outlier channels x200; N(0,sigma) weights per module)",
+        "config": {"workload": WORKLOAD, "M": M, "N": N, "K": K, "segments": [s[1] for s in segs],
+                   "global_batch_tokens": M * world, "parallelism": f"data-parallel replicas x{world}",
+                   "l2": "flushed between timed steps (256 MB write)"},
+        "components_us": {"global_scale+quantize": round(float(np.mean(quant_ms)) * 1e3, 2),
+                          "fused_gemm": round(gemm_avg_ms * 1e3, 2)},
+        "roofline": roofline, "quantizer": quantizer, "e2e": e2e,
+        "gpu_launches": 3 * args.steps,
+        "clocks": clk.summary(),
+        "activation_stats": act_stats(x),
+        "sanity_rel_err_vs_bf16_gemm": {"value": round(sanity, 4), "pages_gate_proj": 0.11},
+    }
+    return out
+
+
+def cpu_baseline_ours(budget_rows=512):
+    """The oracle as it stands, on a bounded sample of the same step: global
+    scale over the whole activation, quantization of `budget_rows` rows and
+    their FP64 GEMM against the whole fused weight."""
+    import oracle
+    from nvfp4_w4a4_quantized_09_b200 import synth
+    x = synth.bf16_bits(synth.student_t_activations(M_TOK, K_HID, seed=3))
+    cw, sw, segs, off = [], [], [], 0
+    for _, w in synth.gdn_weights(synth.GDN_MODULES):
+        b = synth.bf16_bits(w)
+        gw, _ = oracle.global_scale(b)
+        c, s = oracle.quantize(b, gw)
+        cw.append(c), sw.append(s), segs.append((off, w.shape[0], gw))
+        off += w.shape[0]
+    W = oracle.dequantize_noglobal(np.concatenate(cw), np.concatenate(sw))
+    N = W.shape[0]
+    t0 = time.perf_counter()
+    g, _ = oracle.global_scale(x)
+    ca, sa = oracle.quantize(x[:budget_rows], g)
+    A = oracle.dequantize_noglobal(ca, sa)
+    y64 = oracle.gemm_f64(A, W, oracle.segment_alpha(g, segs))
+    oracle.bf16_from_double(y64)
+    dt = time.perf_counter() - t0
+    return {"value": round(2.0 * budget_rows * N * K_HID / dt / 1e12, 6), "unit": "TFLOP/s",
+            "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"global scale over X[8192,5120] + quantize and FP64 GEMM of {budget_rows} "
+                      f"rows x {N} x {K_HID} ({dt:.1f} s)"}
+
+
+# ---------------------------------------------------------------------------
+# reference arm: the oracle on the host cores
+# ---------------------------------------------------------------------------
+def run_reference(args):
+    import oracle
+    from nvfp4_w4a4_quantized_09_b200 import synth
+    rows_per_step = 8
+    x = synth.bf16_bits(synth.student_t_activations(M_TOK, K_HID, seed=3))
+    cw, sw, segs, off = [], [], [], 0
+    for _, w in synth.gdn_weights(synth.GDN_MODULES):
+        b = synth.bf16_bits(w)
+        gw, _ = oracle.global_scale(b)
+        c, s = oracle.quantize(b, gw)
+        cw.append(c), sw.append(s), segs.append((off, w.shape[0], gw))
+        off += w.shape[0]
+    W = oracle.dequantize_noglobal(np.concatenate(cw), np.concatenate(sw))
+    N = W.shape[0]
+
+    def step(i):
+        r0 = (i * rows_per_step) % M_TOK
+        g, _ = oracle.global_scale(x)
+        ca, sa = oracle.quantize(x[r0:r0 + rows_per_step], g)
+        A = oracle.dequantize_noglobal(ca, sa)
+        oracle.bf16_from_double(oracle.gemm_f64(A, W, oracle.segment_alpha(g, segs)))
+
+    for i in range(args.warmup):
+        step(i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        step(i)
+    dt = time.perf_counter() - t0
+    value = 2.0 * rows_per_step * N * K_HID * args.steps / dt / 1e12
+    cores = oracle.num_threads()
+    sample = (f"per step: global scale over X[8192,5120], quantize + FP64 GEMM of "
+              f"{rows_per_step} rows x {N} x {K_HID}")
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s",
+            "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(dt / args.steps * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle)", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "M": M_TOK, "N": N, "K": K_HID},
+            "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cores,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=dev)
+    out = run_ours(args, dev, world, rank)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline_ours()
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()

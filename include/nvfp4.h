@@ -1,0 +1,192 @@
+/*
+ * nvfp4.h -- C ABI of the NVFP4 W4A4 quantized linear layer for B200 (sm_100a).
+ *
+ * The layer follows the pages on "Why Gated DeltaNet Survives 4-Bit
+ * Quantization: NVFP4 W4A4 for the Recurrent Half of a Hybrid 27B LLM":
+ *   - every linear layer runs with 4-bit weights AND activations (chatpaper.ai
+ *     abstract: "NVFP4 W4A4 on all 496 linear layers");
+ *   - NVFP4 = E2M1 values with one E4M3 scale per 16-element block
+ *     (evolve.pub review, Scope & Claims; thevalue.engineering, second section);
+ *   - the GEMM runs natively on NVFP4-capable hardware (evolve.pub FAQ);
+ *   - modules fused into one GEMM keep their own global scales, which is the
+ *     global-scale mismatch the paper repairs (chatpaper.ai abstract;
+ *     evolve.pub Key claims, fourth bullet).
+ *
+ * Conventions shared by every entry point:
+ *   - Pointers marked (device) are CUDA device pointers on the current device;
+ *     (host) pointers are read during the call only.  The caller allocates and
+ *     owns every buffer; the library allocates no device memory.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Work is enqueued asynchronously; nothing synchronizes except
+ *     nvfp4_last_device_status().  Global scales stay in device memory, so a
+ *     whole layer runs without a host round trip.
+ *   - Argument checks happen on the host before anything is enqueued; a
+ *     failing check returns an error status and enqueues nothing.  A CUDA
+ *     launch error returns NVFP4_ERR_CUDA.  No C++ exception crosses the ABI.
+ *   - BF16 tensors are row-major with a row stride `ld` in elements.
+ *   - Packed codes: two E2M1 codes per byte, element 2j in the low nibble of
+ *     byte j (sign in bit 3 of each nibble); a [rows, cols] tensor occupies
+ *     rows * cols/2 contiguous bytes.
+ *   - Block scales: unsigned E4M3 bytes (largest 448 = 0x7E), one per 16
+ *     consecutive elements of a row.
+ */
+#ifndef NVFP4_H_
+#define NVFP4_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    NVFP4_OK = 0,
+    NVFP4_ERR_INVALID_ARG = 1,       /* null pointer, negative size, bad enum  */
+    NVFP4_ERR_ALIGNMENT = 2,         /* pointer or stride not 16-byte aligned  */
+    NVFP4_ERR_UNSUPPORTED_SHAPE = 3, /* shape outside what the kernels accept  */
+    NVFP4_ERR_CUDA = 4,              /* a CUDA runtime/driver call failed      */
+    NVFP4_ERR_TIMEOUT = 5,           /* a bounded device-side wait gave up     */
+    NVFP4_ERR_DEVICE = 6             /* current device is not sm_100           */
+} nvfp4_status;
+
+typedef enum {
+    /* [rows, cols/16] bytes, row-major, no padding. */
+    NVFP4_SF_LINEAR = 0,
+    /* The block-scaled tensor-core layout the GEMM consumes: rows padded to a
+     * multiple of 128, scale columns to a multiple of 4; each 128-row x
+     * 4-column group is a 512-byte atom, atoms ordered with the scale-column
+     * group fastest; inside an atom, scale (r, c) sits at byte
+     * (r % 32) * 16 + ((r / 32) % 4) * 4 + (c % 4).  Padding bytes are 0. */
+    NVFP4_SF_TCGEN05 = 1
+} nvfp4_sf_layout;
+
+/* One module of a fused weight: rows [n_offset, n_offset + n_size) of the
+ * concatenated weight (= output columns of the GEMM) use the FP32 global
+ * scale at w_gscale (device pointer). */
+typedef struct {
+    int64_t n_offset;
+    int64_t n_size;
+    const float* w_gscale;
+} nvfp4_segment;
+
+#define NVFP4_MAX_SEGMENTS 16
+/* Bytes of the zero-initialised workspace nvfp4_global_scale needs. */
+#define NVFP4_GLOBAL_SCALE_WORKSPACE_BYTES 256
+
+/* Per-tensor FP32 global scale from the absolute maximum.
+ *   amax = max |x| over x[rows, cols] (BF16, row stride ld, device);
+ *   g = fl32(amax / 2688) (2688 = 6 * 448, the largest E2M1 value times the
+ *   largest E4M3 scale); g = 1 when amax == 0.
+ * g_out (device, 1 float) receives g; amax_out (device, 1 float) receives
+ * amax, or may be NULL.  workspace (device, NVFP4_GLOBAL_SCALE_WORKSPACE_BYTES,
+ * 16-byte aligned) must be zero before the first call; every call leaves it
+ * zero again.  Calls that share a workspace must not overlap in time.
+ * Requirements: cols % 8 == 0, ld % 8 == 0, ld >= cols, x 16-byte aligned.
+ * rows == 0 or cols == 0 yields amax = 0, g = 1.
+ * Source: the per-module global scale behind the fused-GEMM repair
+ * (chatpaper.ai abstract); absmax is the dynamic reading of it. */
+nvfp4_status nvfp4_global_scale(const void* x, int64_t rows, int64_t cols, int64_t ld,
+                                float* g_out, float* amax_out, void* workspace,
+                                void* stream);
+
+/* Bytes of the scale buffer for a [rows, cols] tensor in `layout`:
+ * LINEAR rows * cols/16; TCGEN05 roundup(rows,128) * roundup(cols/16,4).
+ * cols must be a multiple of 16. */
+nvfp4_status nvfp4_sf_bytes(int64_t rows, int64_t cols, nvfp4_sf_layout layout,
+                            size_t* bytes);
+
+/* 16-element block quantization of x[rows, cols] (BF16, row stride ld, device)
+ * under the global scale *g (device).  Per row and 16-block:
+ *   s8 = E4M3_RNE_satfinite(fl32(fl32(blockmax / 6) / g)),
+ *   d = fl32(E4M3(s8) * g), code = E2M1_RNE_satfinite(fl32(x / d)),
+ *   all codes 0 when d == 0; a negative value that rounds to 0 keeps its
+ *   sign (code 8).
+ * codes (device, rows * cols/2 bytes) and sf (device, nvfp4_sf_bytes bytes in
+ * `layout`) are written completely, padding included.
+ * Requirements: cols % 32 == 0, ld % 8 == 0, ld >= cols; x, codes, sf 16-byte
+ * aligned.  rows == 0 enqueues nothing.
+ * Source: evolve.pub review, Scope & Claims (E2M1 values, E4M3 scale per
+ * 16-element block); thevalue.engineering, second section. */
+nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t ld,
+                            const float* g, uint8_t* codes, uint8_t* sf,
+                            nvfp4_sf_layout layout, void* stream);
+
+/* As nvfp4_quantize, for rows [row_offset, row_offset + rows) of a larger
+ * [total_rows, cols] quantized tensor -- one module of a fused weight, which
+ * keeps its own global scale *g.  codes and sf point to the start of the WHOLE
+ * tensor's buffers (total_rows * cols/2 code bytes; nvfp4_sf_bytes(total_rows,
+ * cols, layout) scale bytes); only this slice's rows are written, plus, when
+ * row_offset + rows == total_rows, the tensor-core layout's padding rows.
+ * Calls for different slices of one tensor may run in any order.
+ * Requirements as nvfp4_quantize; 0 <= row_offset, row_offset + rows <=
+ * total_rows.
+ * Source: per-module global scales of a fused GEMM (chatpaper.ai abstract;
+ * evolve.pub Key claims, fourth bullet). */
+nvfp4_status nvfp4_quantize_slice(const void* x, int64_t rows, int64_t cols, int64_t ld,
+                                  const float* g, uint8_t* codes, uint8_t* sf,
+                                  nvfp4_sf_layout layout, int64_t row_offset,
+                                  int64_t total_rows, void* stream);
+
+/* W4A4 GEMM: y[m, n] = BF16_RNE(fl32(acc[m, n] * fl32(*a_g * *w_g))) with
+ * acc[m, n] = sum_k E2M1(a[m,k]) E4M3(sa[m,k/16]) E2M1(w[n,k]) E4M3(sw[n,k/16])
+ * accumulated in FP32 on the tensor cores (block-scaled FP4 MMA).
+ *   a_codes [M, K/2], w_codes [N, K/2]  (device, packed as above, K-major)
+ *   a_sf, w_sf  (device) block scales in NVFP4_SF_TCGEN05 layout
+ *   a_g, w_g    (device) FP32 global scales
+ *   y [M, N] BF16 (device), row stride ldy elements
+ * Weights are [N, K] (the nn.Linear convention) and are quantized with
+ * nvfp4_quantize like activations.  No bias.
+ * Requirements: K % 32 == 0, K >= 32; ldy >= N, ldy % 8 == 0; all pointers
+ * 16-byte aligned.  M == 0 or N == 0 enqueues nothing.
+ * Source: chatpaper.ai abstract (W4A4 on every linear layer); evolve.pub FAQ
+ * (native NVFP4 execution). */
+nvfp4_status nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_g,
+                        const uint8_t* w_codes, const uint8_t* w_sf, const float* w_g,
+                        void* y, int64_t ldy, int64_t M, int64_t N, int64_t K,
+                        void* stream);
+
+/* Fused multi-module W4A4 GEMM: as nvfp4_gemm, but output column n uses the
+ * global scale of the segment containing n:  alpha_n = fl32(*a_g *
+ * *segs[i].w_gscale) for n in [segs[i].n_offset, +n_size).  The fused
+ * result equals, bit for bit, nvfp4_gemm run per module with that module's
+ * scale (the kernel configuration depends on M and K only, and every output
+ * element is accumulated in the same K order), which is the repair of the
+ * global-scale mismatch.
+ *   segs (host, nseg entries, copied during the call): in order, contiguous,
+ *   starting at 0, n_size > 0; N = sum of n_size.  1 <= nseg <=
+ *   NVFP4_MAX_SEGMENTS.  w_codes/w_sf hold the concatenated [N, K] weight,
+ *   each module quantized with its own global scale.
+ * Requirements as nvfp4_gemm.
+ * Source: chatpaper.ai abstract ("kernels that fuse those modules into one
+ * GEMM"); evolve.pub Key claims, fourth bullet. */
+nvfp4_status nvfp4_fused_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_g,
+                              const uint8_t* w_codes, const uint8_t* w_sf,
+                              const nvfp4_segment* segs, int nseg,
+                              void* y, int64_t ldy, int64_t M, int64_t K,
+                              void* stream);
+
+/* Synchronizes `stream`, then reads and clears the library's device status
+ * word on the current device: NVFP4_ERR_TIMEOUT if a bounded wait inside a
+ * kernel gave up since the last call (that kernel's output is then invalid),
+ * NVFP4_ERR_CUDA if the stream reports an error, else NVFP4_OK. */
+nvfp4_status nvfp4_last_device_status(void* stream);
+
+/* Diagnostic: launches one CTA whose thread waits on a barrier nothing ever
+ * arrives on, bounded by limit_ns (1 .. 10^9).  The wait gives up, sets the
+ * device status word and returns, so the next nvfp4_last_device_status()
+ * reports NVFP4_ERR_TIMEOUT while the context stays usable.  Exercises the
+ * timeout path every kernel's waits share, without faulting the GPU. */
+nvfp4_status nvfp4_debug_wait_timeout(int64_t limit_ns, void* stream);
+
+/* Static English description of a status code. */
+const char* nvfp4_status_string(nvfp4_status s);
+
+/* ABI version (major * 10000 + minor * 100 + patch). */
+int nvfp4_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NVFP4_H_ */

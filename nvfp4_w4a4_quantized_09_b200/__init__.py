@@ -1,0 +1,228 @@
+"""NVFP4 W4A4 quantized linear layer for B200 (sm_100a).
+
+Thin torch-facing wrappers over the C ABI in ``include/nvfp4.h``: PyTorch only
+provides device memory and streams; every step of the path (global scale,
+16-block quantization, block-scaled FP4 GEMM, scaled BF16 epilogue, fused
+multi-module GEMM with per-module global scales) runs in the library's CUDA
+kernels.  There is no CPU or PyTorch fallback: if ``libnvfp4.so`` is missing,
+the first call raises.
+
+Method: the pages on "Why Gated DeltaNet Survives 4-Bit Quantization: NVFP4
+W4A4 for the Recurrent Half of a Hybrid 27B LLM" -- NVFP4 (E2M1 values, E4M3
+scale per 16-element block) on weights and activations of every linear layer
+(evolve.pub review, Scope & Claims), served by fused multi-module GEMMs whose
+per-module global scales must be honoured (chatpaper.ai abstract).
+"""
+from __future__ import annotations
+
+import ctypes
+from dataclasses import dataclass
+from typing import List, Optional, Sequence
+
+import torch
+
+from . import _lib
+from ._lib import SF_LINEAR, SF_TCGEN05, MAX_SEGMENTS, Nvfp4Error
+
+__all__ = [
+    "SF_LINEAR", "SF_TCGEN05", "MAX_SEGMENTS", "Nvfp4Error", "QuantizedTensor",
+    "global_scale", "sf_bytes", "quantize", "quantize_into", "quantize_tensor",
+    "gemm", "fused_gemm", "FusedWeight", "linear", "last_device_status",
+    "debug_wait_timeout", "library_path",
+]
+
+
+def library_path() -> str:
+    return _lib.LIB_PATH
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return ctypes.c_void_p(0 if t is None else t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+_workspaces = {}
+
+
+def _workspace(device: torch.device) -> torch.Tensor:
+    """Zero-initialised global-scale workspace, one per device (left zeroed by
+    every call).  Callers on several streams pass their own."""
+    idx = device.index if device.index is not None else torch.cuda.current_device()
+    ws = _workspaces.get(idx)
+    if ws is None:
+        ws = torch.zeros(_lib.GLOBAL_SCALE_WORKSPACE_BYTES, dtype=torch.uint8, device=device)
+        _workspaces[idx] = ws
+    return ws
+
+
+def _check_bf16_matrix(x: torch.Tensor, name: str):
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or not x.is_cuda:
+        raise ValueError(f"{name} must be a 2-D bfloat16 CUDA tensor")
+    if x.stride(1) != 1:
+        raise ValueError(f"{name} must have unit stride along its last dimension")
+
+
+def sf_bytes(rows: int, cols: int, layout: int = SF_TCGEN05) -> int:
+    n = ctypes.c_size_t(0)
+    _lib.check("nvfp4_sf_bytes", _lib.lib().nvfp4_sf_bytes(rows, cols, layout, ctypes.byref(n)))
+    return int(n.value)
+
+
+def global_scale(x: torch.Tensor, g_out: Optional[torch.Tensor] = None,
+                 amax_out: Optional[torch.Tensor] = None,
+                 workspace: Optional[torch.Tensor] = None, stream=None):
+    """(g, amax) as 1-element FP32 device tensors: g = amax / (6 * 448)."""
+    _check_bf16_matrix(x, "x")
+    dev = x.device
+    g_out = torch.empty(1, dtype=torch.float32, device=dev) if g_out is None else g_out
+    amax_out = torch.empty(1, dtype=torch.float32, device=dev) if amax_out is None else amax_out
+    ws = _workspace(dev) if workspace is None else workspace
+    rows, cols = x.shape
+    _lib.check("nvfp4_global_scale", _lib.lib().nvfp4_global_scale(
+        _ptr(x), rows, cols, x.stride(0), _ptr(g_out), _ptr(amax_out), _ptr(ws), _stream(stream)))
+    return g_out, amax_out
+
+
+@dataclass
+class QuantizedTensor:
+    """Packed NVFP4 tensor: codes [rows, cols/2] uint8, block scales (flat,
+    in ``layout``), and its FP32 global scale(s) in device memory."""
+    codes: torch.Tensor
+    sf: torch.Tensor
+    g: torch.Tensor
+    rows: int
+    cols: int
+    layout: int = SF_TCGEN05
+
+
+def quantize(x: torch.Tensor, g: torch.Tensor, layout: int = SF_TCGEN05,
+             codes: Optional[torch.Tensor] = None, sf: Optional[torch.Tensor] = None,
+             stream=None):
+    """Codes and block scales of x under the global scale g (device tensor)."""
+    _check_bf16_matrix(x, "x")
+    rows, cols = x.shape
+    dev = x.device
+    if codes is None:
+        codes = torch.empty(rows, cols // 2, dtype=torch.uint8, device=dev)
+    if sf is None:
+        sf = torch.empty(sf_bytes(rows, cols, layout), dtype=torch.uint8, device=dev)
+    _lib.check("nvfp4_quantize", _lib.lib().nvfp4_quantize(
+        _ptr(x), rows, cols, x.stride(0), _ptr(g), _ptr(codes), _ptr(sf), layout, _stream(stream)))
+    return codes, sf
+
+
+def quantize_into(x: torch.Tensor, g: torch.Tensor, codes: torch.Tensor, sf: torch.Tensor,
+                  row_offset: int, total_rows: int, layout: int = SF_TCGEN05, stream=None):
+    """Quantize x as rows [row_offset, row_offset + rows) of a larger tensor."""
+    _check_bf16_matrix(x, "x")
+    rows, cols = x.shape
+    _lib.check("nvfp4_quantize_slice", _lib.lib().nvfp4_quantize_slice(
+        _ptr(x), rows, cols, x.stride(0), _ptr(g), _ptr(codes), _ptr(sf), layout,
+        row_offset, total_rows, _stream(stream)))
+
+
+def quantize_tensor(x: torch.Tensor, layout: int = SF_TCGEN05, stream=None) -> QuantizedTensor:
+    """Global scale from the absmax, then 16-block quantization."""
+    g, _ = global_scale(x, stream=stream)
+    codes, sf = quantize(x, g, layout, stream=stream)
+    return QuantizedTensor(codes, sf, g, x.shape[0], x.shape[1], layout)
+
+
+def gemm(a: QuantizedTensor, w: QuantizedTensor, y: Optional[torch.Tensor] = None,
+         stream=None) -> torch.Tensor:
+    """y = a @ w.T in BF16 from NVFP4 operands (both in the tensor-core layout)."""
+    if a.layout != SF_TCGEN05 or w.layout != SF_TCGEN05:
+        raise ValueError("the GEMM reads block scales in the tensor-core layout")
+    if a.cols != w.cols:
+        raise ValueError("inner dimensions differ")
+    M, K, N = a.rows, a.cols, w.rows
+    if y is None:
+        y = torch.empty(M, N, dtype=torch.bfloat16, device=a.codes.device)
+    _lib.check("nvfp4_gemm", _lib.lib().nvfp4_gemm(
+        _ptr(a.codes), _ptr(a.sf), _ptr(a.g), _ptr(w.codes), _ptr(w.sf), _ptr(w.g),
+        _ptr(y), y.stride(0), M, N, K, _stream(stream)))
+    return y
+
+
+class FusedWeight:
+    """Several modules' weights concatenated along N, each quantized with its
+    own global scale -- the layout a fused multi-module GEMM serves."""
+
+    def __init__(self, codes, sf, g_list, sizes, cols):
+        self.codes = codes
+        self.sf = sf
+        self.g_list = list(g_list)
+        self.sizes = list(sizes)
+        self.cols = cols
+        self.rows = sum(self.sizes)
+
+    @classmethod
+    def from_modules(cls, weights: Sequence[torch.Tensor], stream=None) -> "FusedWeight":
+        if not 1 <= len(weights) <= MAX_SEGMENTS:
+            raise ValueError(f"1..{MAX_SEGMENTS} modules")
+        cols = weights[0].shape[1]
+        total = sum(w.shape[0] for w in weights)
+        dev = weights[0].device
+        codes = torch.empty(total, cols // 2, dtype=torch.uint8, device=dev)
+        sf = torch.empty(sf_bytes(total, cols, SF_TCGEN05), dtype=torch.uint8, device=dev)
+        gs, off = [], 0
+        for w in weights:
+            if w.shape[1] != cols:
+                raise ValueError("modules must share K")
+            g, _ = global_scale(w, stream=stream)
+            quantize_into(w, g, codes, sf, off, total, SF_TCGEN05, stream=stream)
+            gs.append(g)
+            off += w.shape[0]
+        return cls(codes, sf, gs, [w.shape[0] for w in weights], cols)
+
+    def segments(self):
+        out, off = [], 0
+        for n, g in zip(self.sizes, self.g_list):
+            out.append((off, n, g))
+            off += n
+        return out
+
+
+def fused_gemm(a: QuantizedTensor, w_codes: torch.Tensor, w_sf: torch.Tensor,
+               segments: List, y: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Fused multi-module GEMM; segments = [(n_offset, n_size, g_tensor)]."""
+    if a.layout != SF_TCGEN05:
+        raise ValueError("the GEMM reads block scales in the tensor-core layout")
+    nseg = len(segments)
+    arr = (_lib.Segment * max(nseg, 1))()
+    for i, (off, n, g) in enumerate(segments):
+        arr[i].n_offset = int(off)
+        arr[i].n_size = int(n)
+        arr[i].w_gscale = g.data_ptr()
+    N = sum(int(s[1]) for s in segments)
+    M, K = a.rows, a.cols
+    if y is None:
+        y = torch.empty(M, N, dtype=torch.bfloat16, device=a.codes.device)
+    _lib.check("nvfp4_fused_gemm", _lib.lib().nvfp4_fused_gemm(
+        _ptr(a.codes), _ptr(a.sf), _ptr(a.g), _ptr(w_codes), _ptr(w_sf), arr, nseg,
+        _ptr(y), y.stride(0), M, K, _stream(stream)))
+    return y
+
+
+def linear(x: torch.Tensor, w, y: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """W4A4 linear layer: quantize the BF16 activation x at run time, then the
+    (fused) NVFP4 GEMM against a pre-quantized weight (QuantizedTensor or
+    FusedWeight)."""
+    a = quantize_tensor(x, stream=stream)
+    if isinstance(w, FusedWeight):
+        return fused_gemm(a, w.codes, w.sf, w.segments(), y, stream)
+    return gemm(a, w, y, stream)
+
+
+def last_device_status(stream=None) -> int:
+    """Synchronize and return (and clear) the device status: 0 ok, 5 timeout."""
+    return int(_lib.lib().nvfp4_last_device_status(_stream(stream)))
+
+
+def debug_wait_timeout(limit_ns: int, stream=None) -> None:
+    _lib.check("nvfp4_debug_wait_timeout",
+               _lib.lib().nvfp4_debug_wait_timeout(int(limit_ns), _stream(stream)))

@@ -1,0 +1,559 @@
+// gemm.cu -- block-scaled FP4 x FP4 GEMM with FP32 accumulation in tensor
+// memory and a BF16 epilogue that applies the global scales per N-segment.
+//
+// Y[m, n] = bf16( fl32( acc[m, n] * fl32(gA * gW[seg(n)]) ) ),
+// acc[m, n] = sum_k e2m1(a[m,k]) e4m3(sa[m,k/16]) e2m1(w[n,k]) e4m3(sw[n,k/16]).
+//
+// Sources (pages on "Why Gated DeltaNet Survives 4-Bit Quantization"):
+// W4A4 on every linear layer and the fused-module global-scale repair
+// (chatpaper.ai abstract); native NVFP4 execution (evolve.pub FAQ).
+//
+// Design (sm_100a, one CTA per SM, persistent):
+//   warp 0      TMA producer: A/B code tiles by tiled TMA (128-byte swizzle),
+//               their scale atoms by 1-D bulk copies (the scales are stored
+//               in the tensor-core layout, so one k-step of a 128-row block
+//               is 2 KB of contiguous bytes).
+//   warp 1      TMEM allocator and MMA issuer (one thread): per k-step it
+//               copies the scale atoms shared->TMEM and issues
+//               tcgen05.mma.kind::mxf4nvf4.block_scale (M=128, N=BN, K=64).
+//   warps 2..5  epilogue: TMEM -> registers, alpha per column, BF16 stores.
+// Every wait is bounded; a timeout sets the device status word and all roles
+// leave their loops, drain in-flight copies and free TMEM.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "host_common.h"
+#include "nvfp4.h"
+#include "ptx.cuh"
+
+namespace nvfp4 {
+
+__device__ int g_device_status;
+
+namespace {
+
+constexpr int kBM = 128;             // MMA M (rows of A per tile)
+constexpr int kBKBytes = 128;        // one k-step: 256 FP4 values = 128 bytes per row
+constexpr int kAtom = 512;           // one scale atom: 128 rows x 4 scales
+constexpr int kAtomsPerStep = 4;     // 256 values = 16 scales = 4 atoms per row block
+constexpr int kThreads = 192;        // producer, MMA, 4 epilogue warps
+constexpr int kEpiThreads = 128;
+constexpr uint64_t kTimeoutNs = 1000000000ull;  // 1 s per wait
+
+struct GemmArgs {
+    const uint8_t* a_sf;
+    const uint8_t* w_sf;
+    const float* a_g;
+    uint16_t* y;
+    int64_t ldy;
+    int M, N, K;
+    int m_tiles, n_tiles, k_steps;
+    int atoms_per_rb;     // ceil(K/64): scale atoms per 128-row block
+    int w_rowblocks;      // ceil(N/128)
+    int group_m;          // raster: tiles visit group_m m-tiles per n sweep
+    int nseg;
+    int seg_end[NVFP4_MAX_SEGMENTS];
+    const float* seg_g[NVFP4_MAX_SEGMENTS];
+    uint64_t timeout_ns;
+    int* status;
+};
+
+template <int BN>
+__host__ __device__ constexpr uint32_t make_idesc() {
+    // kind::mxf4nvf4 block-scaled descriptor: A and B E2M1 (format 1), both
+    // K-major, UE4M3 scales (bit 23 = 0), dense, N >> 3 at bit 17, M >> 4 at
+    // bit 24, scale-factor ids 0.
+    return (1u << 7) | (1u << 10) | (static_cast<uint32_t>(BN >> 3) << 17) |
+           (static_cast<uint32_t>(kBM >> 4) << 24);
+}
+
+template <int BN, int STAGES, int ACC>
+struct Cfg {
+    static constexpr int A_BYTES = kBM * kBKBytes;
+    static constexpr int B_BYTES = BN * kBKBytes;
+    static constexpr int SFA_BYTES = kAtomsPerStep * kAtom;
+    static constexpr int SFB_BYTES = (BN / 128) * kAtomsPerStep * kAtom;
+    static constexpr int OFF_A = 0;
+    static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
+    static constexpr int OFF_SFA = OFF_B + STAGES * B_BYTES;
+    static constexpr int OFF_SFB = OFF_SFA + STAGES * SFA_BYTES;
+    static constexpr int OFF_BAR = OFF_SFB + STAGES * SFB_BYTES;
+    static constexpr int NBAR = 2 * STAGES + 2 * ACC + 1;
+    static constexpr int OFF_SEGA = OFF_BAR + NBAR * 8;
+    static constexpr int OFF_SEGE = OFF_SEGA + NVFP4_MAX_SEGMENTS * 4;
+    static constexpr int OFF_MISC = OFF_SEGE + NVFP4_MAX_SEGMENTS * 4;
+    static constexpr int SMEM = OFF_MISC + 16 + 1024;  // + slack for 1024-byte alignment
+    static constexpr int SFA_COL = ACC * BN;
+    static constexpr int SFB_COL = SFA_COL + kAtomsPerStep * 4;
+    static constexpr int COLS_USED = SFB_COL + kAtomsPerStep * (BN / 32);
+    static constexpr int TMEM_COLS = COLS_USED <= 32 ? 32 : COLS_USED <= 64 ? 64
+                                   : COLS_USED <= 128 ? 128 : COLS_USED <= 256 ? 256 : 512;
+    static_assert(COLS_USED <= 512, "tensor memory overflow");
+    static_assert(SMEM <= 232448, "shared memory overflow");
+    static_assert(BN % 128 == 0 && BN <= 256, "BN must be 128 or 256");
+};
+
+__device__ __forceinline__ void tile_coords(int t, const GemmArgs& a, int& mt, int& nt) {
+    const int per_group = a.group_m * a.n_tiles;
+    const int grp = t / per_group;
+    const int first_m = grp * a.group_m;
+    const int gsize = min(a.group_m, a.m_tiles - first_m);
+    const int local = t - grp * per_group;
+    mt = first_m + local % gsize;
+    nt = local / gsize;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    const uint32_t l = __bfloat16_as_ushort(__float2bfloat16_rn(lo));
+    const uint32_t h = __bfloat16_as_ushort(__float2bfloat16_rn(hi));
+    return l | (h << 16);
+}
+
+template <int BN, int STAGES, int ACC>
+__global__ void __launch_bounds__(kThreads, 1)
+nvf4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
+                 const __grid_constant__ CUtensorMap tmap_b, const GemmArgs args) {
+    using C = Cfg<BN, STAGES, ACC>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+    uint64_t* full = bars;
+    uint64_t* empty = bars + STAGES;
+    uint64_t* tmem_full = bars + 2 * STAGES;
+    uint64_t* tmem_empty = bars + 2 * STAGES + ACC;
+    uint64_t* drain = bars + 2 * STAGES + 2 * ACC;
+    float* s_seg_alpha = reinterpret_cast<float*>(smem + C::OFF_SEGA);
+    int* s_seg_end = reinterpret_cast<int*>(smem + C::OFF_SEGE);
+    uint32_t* s_tmem_base = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+    volatile int* s_abort = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int total_tiles = args.m_tiles * args.n_tiles;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < STAGES; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], 1);
+        }
+        for (int i = 0; i < ACC; ++i) {
+            mbar_init(&tmem_full[i], 1);
+            mbar_init(&tmem_empty[i], kEpiThreads / 32);
+        }
+        mbar_init(drain, 1);
+        *s_abort = 0;
+        fence_mbar_init();
+        prefetch_tmap(&tmap_a);
+        prefetch_tmap(&tmap_b);
+    }
+    if (warp == 1) {
+        tmem_alloc(s_tmem_base, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    if (threadIdx.x >= 64 && threadIdx.x < 64 + NVFP4_MAX_SEGMENTS) {
+        const int s = threadIdx.x - 64;
+        s_seg_alpha[s] = (s < args.nseg) ? __fmul_rn(*args.a_g, *args.seg_g[s]) : 0.0f;
+        s_seg_end[s] = (s < args.nseg) ? args.seg_end[s] : 0x7FFFFFFF;
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *s_tmem_base;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ---------------- TMA producer ----------------
+            const uint64_t pol = l2_policy_evict_normal();
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t issued = 0, issued_parity = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+                int mt, nt;
+                tile_coords(t, args, mt, nt);
+                for (int kb = 0; kb < args.k_steps; ++kb) {
+                    if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, args.timeout_ns, s_abort,
+                                           args.status)) {
+                        ok = false;
+                        break;
+                    }
+                    const int natoms = min(kAtomsPerStep, args.atoms_per_rb - kb * kAtomsPerStep);
+                    int w_rbs = 0;
+                    for (int r = 0; r < BN / 128; ++r)
+                        if (nt * (BN / 128) + r < args.w_rowblocks) ++w_rbs;
+                    const uint32_t bytes = C::A_BYTES + C::B_BYTES + natoms * kAtom * (1 + w_rbs);
+                    mbar_arrive_expect_tx(&full[stage], bytes);
+                    tma_load_2d(smem + C::OFF_A + stage * C::A_BYTES, &tmap_a, &full[stage],
+                                kb * kBKBytes, mt * kBM, pol);
+                    tma_load_2d(smem + C::OFF_B + stage * C::B_BYTES, &tmap_b, &full[stage],
+                                kb * kBKBytes, nt * BN, pol);
+                    const size_t a_off =
+                        (static_cast<size_t>(mt) * args.atoms_per_rb + kb * kAtomsPerStep) * kAtom;
+                    bulk_load(smem + C::OFF_SFA + stage * C::SFA_BYTES, args.a_sf + a_off,
+                              natoms * kAtom, &full[stage], pol);
+                    for (int r = 0; r < w_rbs; ++r) {
+                        const size_t w_off = (static_cast<size_t>(nt * (BN / 128) + r) *
+                                                  args.atoms_per_rb + kb * kAtomsPerStep) * kAtom;
+                        bulk_load(smem + C::OFF_SFB + stage * C::SFB_BYTES + r * kAtomsPerStep * kAtom,
+                                  args.w_sf + w_off, natoms * kAtom, &full[stage], pol);
+                    }
+                    issued |= 1u << stage;
+                    issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (!ok) {
+                // leave no copy in flight: wait (bounded) for every stage issued
+                int local_abort = 0;
+                for (int s = 0; s < STAGES; ++s)
+                    if (issued & (1u << s))
+                        mbar_wait_bounded(&full[s], (issued_parity >> s) & 1u, args.timeout_ns,
+                                          &local_abort, args.status);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ---------------- MMA issuer ----------------
+            constexpr uint32_t idesc = make_idesc<BN>();
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            int i = 0;
+            for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x, ++i) {
+                const int acc = i % ACC;
+                const uint32_t acc_phase = (i / ACC) & 1;
+                if (!mbar_wait_bounded(&tmem_empty[acc], acc_phase ^ 1u, args.timeout_ns, s_abort,
+                                       args.status)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + acc * BN;
+                for (int kb = 0; kb < args.k_steps; ++kb) {
+                    if (!mbar_wait_bounded(&full[stage], phase, args.timeout_ns, s_abort,
+                                           args.status)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const int natoms = min(kAtomsPerStep, args.atoms_per_rb - kb * kAtomsPerStep);
+                    const uint32_t sa = smem_u32(smem + C::OFF_A + stage * C::A_BYTES);
+                    const uint32_t sb = smem_u32(smem + C::OFF_B + stage * C::B_BYTES);
+                    const uint32_t ssfa = smem_u32(smem + C::OFF_SFA + stage * C::SFA_BYTES);
+                    const uint32_t ssfb = smem_u32(smem + C::OFF_SFB + stage * C::SFB_BYTES);
+                    for (int j = 0; j < natoms; ++j) {
+                        tc_copy_scales(tmem_base + C::SFA_COL + j * 4, sdesc_scales(ssfa + j * kAtom));
+#pragma unroll
+                        for (int r = 0; r < BN / 128; ++r)
+                            tc_copy_scales(tmem_base + C::SFB_COL + j * (BN / 32) + r * 4,
+                                           sdesc_scales(ssfb + r * kAtomsPerStep * kAtom + j * kAtom));
+                    }
+                    for (int j = 0; j < natoms; ++j) {
+                        tc_mma_nvf4(d_tmem, sdesc_kmajor_sw128(sa + j * 32),
+                                    sdesc_kmajor_sw128(sb + j * 32), idesc,
+                                    tmem_base + C::SFA_COL + j * 4,
+                                    tmem_base + C::SFB_COL + j * (BN / 32), (kb | j) != 0);
+                    }
+                    tc_commit(&empty[stage]);
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (ok) tc_commit(&tmem_full[acc]);
+            }
+            // every tcgen05 operation issued above has finished before TMEM is freed
+            tc_commit(drain);
+            int local_abort = 0;
+            mbar_wait_bounded(drain, 0, args.timeout_ns, &local_abort, args.status);
+        }
+    } else {
+        // ---------------- epilogue (warps 2..5) ----------------
+        // Lane 0 of each warp waits for the accumulator and the result is
+        // broadcast, so the warp stays converged for tcgen05.ld and leaves
+        // together on an abort.  alpha per column comes from the segment table;
+        // a 32-column chunk almost always lies inside one segment.
+        const int q = warp & 3;                  // TMEM lane quarter of this warp
+        const int row = q * 32 + lane;
+        int i = 0;
+        for (int t = blockIdx.x; t < total_tiles; t += gridDim.x, ++i) {
+            int mt, nt;
+            tile_coords(t, args, mt, nt);
+            const int acc = i % ACC;
+            const uint32_t acc_phase = (i / ACC) & 1;
+            int ok = 1;
+            if (lane == 0)
+                ok = mbar_wait_bounded(&tmem_full[acc], acc_phase, args.timeout_ns, s_abort,
+                                       args.status);
+            ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+            if (!ok) break;
+            tc_fence_after();
+            const int m = mt * kBM + row;
+            uint16_t* yrow = args.y + static_cast<int64_t>(m) * args.ldy;
+#pragma unroll 1
+            for (int ch = 0; ch < BN / 32; ++ch) {
+                uint32_t r[32];
+                tmem_ld_32cols(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN + ch * 32, r);
+                tmem_ld_wait();
+                const int n0 = nt * BN + ch * 32;
+                int s0 = 0;
+                while (s0 < args.nseg - 1 && n0 >= s_seg_end[s0]) ++s0;
+                const bool one_seg = (s0 == args.nseg - 1) || (n0 + 31 < s_seg_end[s0]);
+                if (m < args.M && n0 < args.N) {
+                    float v[32];
+                    if (one_seg) {
+                        const float al = s_seg_alpha[s0];
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) v[j] = __fmul_rn(__uint_as_float(r[j]), al);
+                    } else {
+                        int s = s0;
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) {
+                            while (s < args.nseg - 1 && n0 + j >= s_seg_end[s]) ++s;
+                            v[j] = __fmul_rn(__uint_as_float(r[j]), s_seg_alpha[s]);
+                        }
+                    }
+                    uint32_t o[16];
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) o[j] = pack_bf16x2(v[2 * j], v[2 * j + 1]);
+                    if (n0 + 32 <= args.N) {
+                        uint4* dst = reinterpret_cast<uint4*>(yrow + n0);
+#pragma unroll
+                        for (int u = 0; u < 4; ++u)
+                            dst[u] = make_uint4(o[4 * u], o[4 * u + 1], o[4 * u + 2], o[4 * u + 3]);
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j)
+                            if (n0 + j < args.N)
+                                yrow[n0 + j] = static_cast<uint16_t>((o[j >> 1] >> (16 * (j & 1))) & 0xFFFFu);
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tmem_empty[acc]);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) {
+        __syncwarp();
+        tmem_dealloc(tmem_base, C::TMEM_COLS);
+    }
+}
+
+}  // namespace
+
+
+// ---------------------------------------------------------------------------
+// Bounded-wait self-test: one thread waits on a barrier nothing arrives on.
+// The wait must give up after limit_ns and set the device status word; the
+// context stays usable.  Lets the timeout path be tested without a fault.
+// ---------------------------------------------------------------------------
+__global__ void wait_timeout_selftest_kernel(uint64_t limit_ns, int* status) {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        abort_flag = 0;
+        fence_mbar_init();
+        mbar_wait_bounded(&bar, 0, limit_ns, &abort_flag, status);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+// [rows, row_bytes] byte matrix read in boxes of 128 bytes x box_rows rows,
+// 128-byte swizzle, zero fill out of bounds.
+bool make_code_map(CUtensorMap* m, const uint8_t* base, int64_t rows, int64_t row_bytes,
+                   int box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(row_bytes), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_bytes)};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(kBKBytes), static_cast<cuuint32_t>(box_rows)};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(base), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+int* device_status_ptr() {
+    static int* cache[64] = {nullptr};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    if (!cache[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return nullptr;
+        cache[dev] = static_cast<int*>(p);
+    }
+    return cache[dev];
+}
+
+template <int BN, int STAGES, int ACC>
+nvfp4_status launch_gemm(const uint8_t* a_codes, const uint8_t* w_codes, GemmArgs& args,
+                         const DeviceInfo& dev, cudaStream_t stream) {
+    using Cf = Cfg<BN, STAGES, ACC>;
+    auto kern = nvf4_gemm_kernel<BN, STAGES, ACC>;
+    static bool attr_set[64] = {false};
+    int devid = 0;
+    if (cudaGetDevice(&devid) != cudaSuccess || devid < 0 || devid >= 64) return NVFP4_ERR_CUDA;
+    if (!attr_set[devid]) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::SMEM) !=
+            cudaSuccess)
+            return NVFP4_ERR_CUDA;
+        attr_set[devid] = true;
+    }
+    CUtensorMap ta, tb;
+    if (!make_code_map(&ta, a_codes, args.M, args.K / 2, kBM)) return NVFP4_ERR_CUDA;
+    if (!make_code_map(&tb, w_codes, args.N, args.K / 2, BN)) return NVFP4_ERR_CUDA;
+    args.m_tiles = (args.M + kBM - 1) / kBM;
+    args.n_tiles = (args.N + BN - 1) / BN;
+    const int tiles = args.m_tiles * args.n_tiles;
+    const int grid = tiles < dev.sms ? tiles : dev.sms;
+    kern<<<grid, kThreads, Cf::SMEM, stream>>>(ta, tb, args);
+    return cuda_status(cudaGetLastError());
+}
+
+nvfp4_status gemm_impl(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_g,
+                       const uint8_t* w_codes, const uint8_t* w_sf, const nvfp4_segment* segs,
+                       int nseg, void* y, int64_t ldy, int64_t M, int64_t K, void* stream) {
+    if (!segs || nseg < 1 || nseg > NVFP4_MAX_SEGMENTS) return NVFP4_ERR_INVALID_ARG;
+    if (M < 0 || K < 0 || !a_g) return NVFP4_ERR_INVALID_ARG;
+    int64_t N = 0;
+    for (int s = 0; s < nseg; ++s) {
+        if (segs[s].n_offset != N || segs[s].n_size <= 0 || !segs[s].w_gscale)
+            return NVFP4_ERR_INVALID_ARG;
+        N += segs[s].n_size;
+    }
+    if (K % 32 != 0 || K < 32) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31) || K >= (int64_t(1) << 31))
+        return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (ldy < N || ldy % 8 != 0) return NVFP4_ERR_ALIGNMENT;
+    if (M == 0) return NVFP4_OK;
+    if (!a_codes || !a_sf || !w_codes || !w_sf || !y) return NVFP4_ERR_INVALID_ARG;
+    if (!aligned16(a_codes) || !aligned16(a_sf) || !aligned16(w_codes) || !aligned16(w_sf) ||
+        !aligned16(y))
+        return NVFP4_ERR_ALIGNMENT;
+    DeviceInfo dev;
+    nvfp4_status st = require_sm100(&dev);
+    if (st != NVFP4_OK) return st;
+    int* status = device_status_ptr();
+    if (!status) return NVFP4_ERR_CUDA;
+
+    GemmArgs args = {};
+    args.a_sf = a_sf;
+    args.w_sf = w_sf;
+    args.a_g = a_g;
+    args.y = static_cast<uint16_t*>(y);
+    args.ldy = ldy;
+    args.M = static_cast<int>(M);
+    args.N = static_cast<int>(N);
+    args.K = static_cast<int>(K);
+    args.k_steps = static_cast<int>((K + 255) / 256);
+    args.atoms_per_rb = static_cast<int>((K + 63) / 64);
+    args.w_rowblocks = static_cast<int>((N + 127) / 128);
+    args.group_m = 16;
+    args.nseg = nseg;
+    for (int s = 0; s < nseg; ++s) {
+        args.seg_end[s] = static_cast<int>(segs[s].n_offset + segs[s].n_size);
+        args.seg_g[s] = segs[s].w_gscale;
+    }
+    args.timeout_ns = kTimeoutNs;
+    args.status = status;
+    cudaStream_t cs = as_stream(stream);
+    // The configuration depends on M only, so a fused GEMM and its per-module
+    // GEMMs accumulate every output element identically.
+    if (M > 256) return launch_gemm<256, 4, 1>(a_codes, w_codes, args, dev, cs);
+    return launch_gemm<128, 6, 2>(a_codes, w_codes, args, dev, cs);
+}
+
+}  // namespace
+}  // namespace nvfp4
+
+using namespace nvfp4;
+
+extern "C" nvfp4_status nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_g,
+                                   const uint8_t* w_codes, const uint8_t* w_sf, const float* w_g,
+                                   void* y, int64_t ldy, int64_t M, int64_t N, int64_t K,
+                                   void* stream) {
+    if (N < 0 || !w_g) return NVFP4_ERR_INVALID_ARG;
+    if (N == 0) return (M >= 0 && K >= 0) ? NVFP4_OK : NVFP4_ERR_INVALID_ARG;
+    nvfp4_segment seg = {0, N, w_g};
+    return gemm_impl(a_codes, a_sf, a_g, w_codes, w_sf, &seg, 1, y, ldy, M, K, stream);
+}
+
+extern "C" nvfp4_status nvfp4_fused_gemm(const uint8_t* a_codes, const uint8_t* a_sf,
+                                         const float* a_g, const uint8_t* w_codes,
+                                         const uint8_t* w_sf, const nvfp4_segment* segs, int nseg,
+                                         void* y, int64_t ldy, int64_t M, int64_t K,
+                                         void* stream) {
+    return gemm_impl(a_codes, a_sf, a_g, w_codes, w_sf, segs, nseg, y, ldy, M, K, stream);
+}
+
+extern "C" nvfp4_status nvfp4_last_device_status(void* stream) {
+    if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return NVFP4_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_device_status, sizeof(int)) != cudaSuccess) return NVFP4_ERR_CUDA;
+    if (v != 0) {
+        const int zero = 0;
+        if (cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int)) != cudaSuccess)
+            return NVFP4_ERR_CUDA;
+        return NVFP4_ERR_TIMEOUT;
+    }
+    return NVFP4_OK;
+}
+
+extern "C" nvfp4_status nvfp4_debug_wait_timeout(int64_t limit_ns, void* stream) {
+    if (limit_ns <= 0 || limit_ns > 1000000000) return NVFP4_ERR_INVALID_ARG;
+    int* status = device_status_ptr();
+    if (!status) return NVFP4_ERR_CUDA;
+    wait_timeout_selftest_kernel<<<1, 32, 0, as_stream(stream)>>>(static_cast<uint64_t>(limit_ns),
+                                                                 status);
+    return cuda_status(cudaGetLastError());
+}
+
+extern "C" const char* nvfp4_status_string(nvfp4_status s) {
+    switch (s) {
+        case NVFP4_OK: return "ok";
+        case NVFP4_ERR_INVALID_ARG: return "invalid argument";
+        case NVFP4_ERR_ALIGNMENT: return "pointer or stride not aligned";
+        case NVFP4_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+        case NVFP4_ERR_CUDA: return "CUDA error";
+        case NVFP4_ERR_TIMEOUT: return "device-side wait timed out";
+        case NVFP4_ERR_DEVICE: return "device is not sm_100";
+    }
+    return "unknown status";
+}
+
+extern "C" int nvfp4_version(void) { return 100; }

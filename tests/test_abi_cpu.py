@@ -1,0 +1,137 @@
+"""The C-ABI library without a GPU: it loads, exports every entry point that
+include/nvfp4.h declares, and rejects bad arguments on the host before any
+CUDA call (no compute runs here)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from nvfp4_w4a4_quantized_09_b200 import _lib, build as _build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "nvfp4.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    _build.build()
+    return _lib.lib()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(nvfp4_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_declares_the_path():
+    names = declared_functions()
+    for required in ["nvfp4_global_scale", "nvfp4_quantize", "nvfp4_gemm", "nvfp4_fused_gemm",
+                     "nvfp4_sf_bytes", "nvfp4_quantize_slice"]:
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared_functions():
+        assert hasattr(L, name), name
+        assert name in _lib.SIGNATURES, f"binding lacks {name}"
+
+
+def test_status_strings_and_version(L):
+    for s in range(7):
+        assert len(L.nvfp4_status_string(s)) > 0
+    assert L.nvfp4_version() >= 100
+
+
+def test_sf_bytes(L):
+    n = ctypes.c_size_t()
+    assert L.nvfp4_sf_bytes(300, 160, _lib.SF_TCGEN05, ctypes.byref(n)) == 0
+    assert n.value == 384 * 12
+    assert L.nvfp4_sf_bytes(300, 160, _lib.SF_LINEAR, ctypes.byref(n)) == 0
+    assert n.value == 300 * 10
+    assert L.nvfp4_sf_bytes(32768, 5120, _lib.SF_TCGEN05, ctypes.byref(n)) == 0
+    assert n.value == 32768 * 320
+    assert L.nvfp4_sf_bytes(10, 24, _lib.SF_LINEAR, ctypes.byref(n)) == _lib.NVFP4_ERR_UNSUPPORTED_SHAPE
+    assert L.nvfp4_sf_bytes(-1, 32, _lib.SF_LINEAR, ctypes.byref(n)) == _lib.NVFP4_ERR_INVALID_ARG
+    assert L.nvfp4_sf_bytes(1, 32, 7, ctypes.byref(n)) == _lib.NVFP4_ERR_INVALID_ARG
+
+
+FAKE = ctypes.c_void_p(0x10000)      # 16-byte aligned, never dereferenced
+ODD = ctypes.c_void_p(0x10008)       # 8-byte aligned only
+NUL = ctypes.c_void_p(0)
+
+
+def test_quantize_rejects_bad_arguments(L):
+    q = L.nvfp4_quantize
+    assert q(FAKE, 4, 48, 48, FAKE, FAKE, FAKE, 1, NUL) == _lib.NVFP4_ERR_ALIGNMENT   # cols % 32
+    assert q(FAKE, 4, 64, 60, FAKE, FAKE, FAKE, 1, NUL) == _lib.NVFP4_ERR_ALIGNMENT   # ld % 8
+    assert q(FAKE, 4, 64, 64, NUL, FAKE, FAKE, 1, NUL) == _lib.NVFP4_ERR_INVALID_ARG  # g null
+    assert q(FAKE, 4, 64, 64, FAKE, FAKE, FAKE, 9, NUL) == _lib.NVFP4_ERR_INVALID_ARG  # layout
+    assert q(FAKE, -1, 64, 64, FAKE, FAKE, FAKE, 1, NUL) == _lib.NVFP4_ERR_INVALID_ARG
+    assert q(FAKE, 4, 64, 32, FAKE, FAKE, FAKE, 1, NUL) == _lib.NVFP4_ERR_INVALID_ARG  # ld < cols
+    assert q(ODD, 4, 64, 64, FAKE, FAKE, FAKE, 1, NUL) == _lib.NVFP4_ERR_ALIGNMENT
+    assert q(FAKE, 4, 64, 64, FAKE, NUL, FAKE, 1, NUL) == _lib.NVFP4_ERR_INVALID_ARG
+    assert q(FAKE, 0, 64, 64, FAKE, NUL, NUL, 0, NUL) == _lib.NVFP4_OK                # empty
+
+
+def test_quantize_slice_rejects_bad_ranges(L):
+    q = L.nvfp4_quantize_slice
+    assert q(FAKE, 4, 64, 64, FAKE, FAKE, FAKE, 1, 10, 12, NUL) == _lib.NVFP4_ERR_INVALID_ARG
+    assert q(FAKE, 4, 64, 64, FAKE, FAKE, FAKE, 1, -1, 12, NUL) == _lib.NVFP4_ERR_INVALID_ARG
+
+
+def test_global_scale_rejects_bad_arguments(L):
+    gs = L.nvfp4_global_scale
+    assert gs(FAKE, 4, 64, 64, NUL, NUL, FAKE, NUL) == _lib.NVFP4_ERR_INVALID_ARG     # g_out
+    assert gs(FAKE, 4, 64, 64, FAKE, NUL, NUL, NUL) == _lib.NVFP4_ERR_INVALID_ARG     # workspace
+    assert gs(FAKE, 4, 60, 64, FAKE, NUL, FAKE, NUL) == _lib.NVFP4_ERR_ALIGNMENT
+    assert gs(ODD, 4, 64, 64, FAKE, NUL, FAKE, NUL) == _lib.NVFP4_ERR_ALIGNMENT
+    assert gs(FAKE, 4, 64, 64, FAKE, NUL, ODD, NUL) == _lib.NVFP4_ERR_ALIGNMENT
+
+
+def test_gemm_rejects_bad_arguments(L):
+    g = L.nvfp4_gemm
+    ok = (FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE)
+    assert g(*ok, 128, 64, 128, 48, NUL) == _lib.NVFP4_ERR_UNSUPPORTED_SHAPE          # K % 32
+    assert g(*ok, 128, 64, 128, 0, NUL) == _lib.NVFP4_ERR_UNSUPPORTED_SHAPE           # K = 0
+    assert g(*ok, 100, 64, 128, 64, NUL) == _lib.NVFP4_ERR_ALIGNMENT                  # ldy < N
+    assert g(*ok, 132, 64, 130, 64, NUL) == _lib.NVFP4_ERR_ALIGNMENT                  # ldy % 8
+    assert g(FAKE, FAKE, FAKE, FAKE, FAKE, NUL, FAKE, 128, 64, 128, 64, NUL) == _lib.NVFP4_ERR_INVALID_ARG
+    assert g(ODD, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 128, 64, 128, 64, NUL) == _lib.NVFP4_ERR_ALIGNMENT
+    assert g(*ok, 128, 0, 128, 64, NUL) == _lib.NVFP4_OK                              # M = 0
+
+
+def seg_array(entries):
+    arr = (_lib.Segment * len(entries))()
+    for i, (o, n, p) in enumerate(entries):
+        arr[i].n_offset, arr[i].n_size, arr[i].w_gscale = o, n, p
+    return arr
+
+
+def test_fused_gemm_validates_segment_table(L):
+    f = L.nvfp4_fused_gemm
+    args = (FAKE, FAKE, FAKE, FAKE, FAKE)
+    good = seg_array([(0, 64, 0x10000), (64, 64, 0x10010)])
+    assert f(*args, good, 0, FAKE, 128, 4, 64, NUL) == _lib.NVFP4_ERR_INVALID_ARG      # nseg 0
+    assert f(*args, good, 17, FAKE, 128, 4, 64, NUL) == _lib.NVFP4_ERR_INVALID_ARG     # > max
+    gap = seg_array([(0, 64, 0x10000), (72, 64, 0x10010)])
+    assert f(*args, gap, 2, FAKE, 136, 4, 64, NUL) == _lib.NVFP4_ERR_INVALID_ARG       # not contiguous
+    empty = seg_array([(0, 64, 0x10000), (64, 0, 0x10010)])
+    assert f(*args, empty, 2, FAKE, 128, 4, 64, NUL) == _lib.NVFP4_ERR_INVALID_ARG     # n_size 0
+    noscale = seg_array([(0, 64, 0x10000), (64, 64, 0)])
+    assert f(*args, noscale, 2, FAKE, 128, 4, 64, NUL) == _lib.NVFP4_ERR_INVALID_ARG
+    assert f(*args, good, 2, FAKE, 120, 4, 64, NUL) == _lib.NVFP4_ERR_ALIGNMENT        # ldy < N
+    assert f(*args, good, 2, FAKE, 128, 0, 64, NUL) == _lib.NVFP4_OK                   # M = 0
+
+
+def test_debug_wait_rejects_bad_limits(L):
+    assert L.nvfp4_debug_wait_timeout(0, NUL) == _lib.NVFP4_ERR_INVALID_ARG
+    assert L.nvfp4_debug_wait_timeout(2_000_000_000, NUL) == _lib.NVFP4_ERR_INVALID_ARG
+
+
+def test_python_api_refuses_cpu_tensors():
+    import torch
+    import nvfp4_w4a4_quantized_09_b200 as nv
+    with pytest.raises(ValueError):
+        nv.quantize_tensor(torch.zeros(4, 64, dtype=torch.bfloat16))
