@@ -78,30 +78,43 @@ def test_fused_gdn_prefill_full_size():
         assert torch.equal(y[:, off:off + n].view(torch.int16), ym.view(torch.int16))
 
 
-@pytest.mark.parametrize("M", [1, 8, 32, 128])
+_decode_cache = {}
+
+
+def decode_weights(which):
+    """GPU weights and the oracle's quantization of them, built once per
+    weight set for the whole sweep."""
+    if which not in _decode_cache:
+        if which == "gdn24640":
+            ws = [w for _, w in synth.gdn_weights(synth.GDN_MODULES_DECODE, device=DEV)]
+        else:
+            N = 5120 if which == "dense5120" else 34816
+            ws = [synth.gaussian_weights(N, 5120, 0.015, seed=20, device=DEV)]
+        cw, sw, segs = quantize_modules_oracle(ws)
+        _decode_cache[which] = (ws, cw, dequant(cw, sw), segs)
+    return _decode_cache[which]
+
+
 @pytest.mark.parametrize("which", ["dense5120", "gdn24640", "gateup34816"])
-def test_decode_sweep(M, which):
+@pytest.mark.parametrize("M", [1, 8, 32, 128])
+def test_decode_sweep(which, M):
     K = 5120
+    ws, cw, W, segs = decode_weights(which)
     x = synth.student_t_activations(M, K, seed=100 + M, device=DEV)
     a = nv.quantize_tensor(x)
     if which == "gdn24640":
-        ws = [w for _, w in synth.gdn_weights(synth.GDN_MODULES_DECODE, device=DEV)]
         fw = nv.FusedWeight.from_modules(ws)
+        assert np.array_equal(np_u8(fw.codes), cw)
         y = nv.fused_gemm(a, fw.codes, fw.sf, fw.segments())
-        cw, sw, segs = quantize_modules_oracle(ws)
     else:
-        N = 5120 if which == "dense5120" else 34816
-        w = synth.gaussian_weights(N, K, 0.015, seed=20, device=DEV)
-        wq = nv.quantize_tensor(w)
+        wq = nv.quantize_tensor(ws[0])
         y = nv.gemm(a, wq)
-        cw, sw, segs = quantize_modules_oracle([w])
     torch.cuda.synchronize()
     xb = host_bits(x)
     ga, _ = oracle.global_scale(xb)
     rows = sample_rows(M, 6, M)
     ca, sa = oracle.quantize(xb[rows], ga)
     A = dequant(ca, sa)
-    W = dequant(cw, sw)
     alpha = oracle.segment_alpha(ga, segs)
     assert_gemm_matches(host_bits(y[torch.from_numpy(rows).to(DEV)]), A, W, alpha,
                         label=f"decode M={M} {which}")
