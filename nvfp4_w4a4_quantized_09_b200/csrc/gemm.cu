@@ -16,7 +16,10 @@
 //   warp 1      TMEM allocator and MMA issuer (one thread): per k-step it
 //               copies the scale atoms shared->TMEM and issues
 //               tcgen05.mma.kind::mxf4nvf4.block_scale (M=128, N=BN, K=64).
-//   warps 2..5  epilogue: TMEM -> registers, alpha per column, BF16 stores.
+//   warps 2..9  epilogue: two warps per TMEM lane quarter, each draining half
+//               of the tile's columns into registers; the accumulator is
+//               released as soon as all of it sits in registers, so the next
+//               tile's MMAs overlap the alpha scaling and the BF16 stores.
 // Every wait is bounded; a timeout sets the device status word and all roles
 // leave their loops, drain in-flight copies and free TMEM.
 #include <cuda.h>
@@ -38,8 +41,8 @@ constexpr int kBM = 128;             // MMA M (rows of A per tile)
 constexpr int kBKBytes = 128;        // one k-step: 256 FP4 values = 128 bytes per row
 constexpr int kAtom = 512;           // one scale atom: 128 rows x 4 scales
 constexpr int kAtomsPerStep = 4;     // 256 values = 16 scales = 4 atoms per row block
-constexpr int kThreads = 192;        // producer, MMA, 4 epilogue warps
-constexpr int kEpiThreads = 128;
+constexpr int kEpiWarps = 8;         // two per TMEM lane quarter, each half the columns
+constexpr int kThreads = 64 + 32 * kEpiWarps;  // producer, MMA, epilogue warps
 constexpr uint64_t kTimeoutNs = 1000000000ull;  // 1 s per wait
 
 struct GemmArgs {
@@ -141,7 +144,7 @@ nvf4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
         }
         for (int i = 0; i < ACC; ++i) {
             mbar_init(&tmem_full[i], 1);
-            mbar_init(&tmem_empty[i], kEpiThreads / 32);
+            mbar_init(&tmem_empty[i], kEpiWarps);
         }
         mbar_init(drain, 1);
         *s_abort = 0;
@@ -166,7 +169,7 @@ nvf4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
     if (warp == 0) {
         if (lane == 0) {
             // ---------------- TMA producer ----------------
-            const uint64_t pol = l2_policy_evict_normal();
+            const uint64_t pol = l2_policy_evict_last();   // operands are re-read by many tiles
             int stage = 0;
             uint32_t phase = 0;
             uint32_t issued = 0, issued_parity = 0;
@@ -274,13 +277,17 @@ nvf4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
             mbar_wait_bounded(drain, 0, args.timeout_ns, &local_abort, args.status);
         }
     } else {
-        // ---------------- epilogue (warps 2..5) ----------------
+        // ---------------- epilogue (warps 2..9) ----------------
         // Lane 0 of each warp waits for the accumulator and the result is
         // broadcast, so the warp stays converged for tcgen05.ld and leaves
         // together on an abort.  alpha per column comes from the segment table;
         // a 32-column chunk almost always lies inside one segment.
+        constexpr int kHalf = BN / 2;            // columns per epilogue warp
+        constexpr int kChunks = kHalf / 32;
         const int q = warp & 3;                  // TMEM lane quarter of this warp
+        const int half = (warp - 2) >> 2;        // which half of the columns
         const int row = q * 32 + lane;
+        const uint64_t pol_y = l2_policy_evict_first();
         int i = 0;
         for (int t = blockIdx.x; t < total_tiles; t += gridDim.x, ++i) {
             int mt, nt;
@@ -294,14 +301,19 @@ nvf4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
             ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
             if (!ok) break;
             tc_fence_after();
+            uint32_t r[kChunks][32];
+            const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN + half * kHalf;
+#pragma unroll
+            for (int ch = 0; ch < kChunks; ++ch) tmem_ld_32cols(taddr + ch * 32, r[ch]);
+            tmem_ld_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tmem_empty[acc]);   // accumulator free for the next tile
             const int m = mt * kBM + row;
             uint16_t* yrow = args.y + static_cast<int64_t>(m) * args.ldy;
-#pragma unroll 1
-            for (int ch = 0; ch < BN / 32; ++ch) {
-                uint32_t r[32];
-                tmem_ld_32cols(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN + ch * 32, r);
-                tmem_ld_wait();
-                const int n0 = nt * BN + ch * 32;
+#pragma unroll
+            for (int ch = 0; ch < kChunks; ++ch) {
+                const int n0 = nt * BN + half * kHalf + ch * 32;
                 int s0 = 0;
                 while (s0 < args.nseg - 1 && n0 >= s_seg_end[s0]) ++s0;
                 const bool one_seg = (s0 == args.nseg - 1) || (n0 + 31 < s_seg_end[s0]);
@@ -310,23 +322,23 @@ nvf4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                     if (one_seg) {
                         const float al = s_seg_alpha[s0];
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) v[j] = __fmul_rn(__uint_as_float(r[j]), al);
+                        for (int j = 0; j < 32; ++j) v[j] = __fmul_rn(__uint_as_float(r[ch][j]), al);
                     } else {
                         int s = s0;
 #pragma unroll
                         for (int j = 0; j < 32; ++j) {
                             while (s < args.nseg - 1 && n0 + j >= s_seg_end[s]) ++s;
-                            v[j] = __fmul_rn(__uint_as_float(r[j]), s_seg_alpha[s]);
+                            v[j] = __fmul_rn(__uint_as_float(r[ch][j]), s_seg_alpha[s]);
                         }
                     }
                     uint32_t o[16];
 #pragma unroll
                     for (int j = 0; j < 16; ++j) o[j] = pack_bf16x2(v[2 * j], v[2 * j + 1]);
                     if (n0 + 32 <= args.N) {
-                        uint4* dst = reinterpret_cast<uint4*>(yrow + n0);
 #pragma unroll
                         for (int u = 0; u < 4; ++u)
-                            dst[u] = make_uint4(o[4 * u], o[4 * u + 1], o[4 * u + 2], o[4 * u + 3]);
+                            st_global_v4_hint(yrow + n0 + 8 * u, o[4 * u], o[4 * u + 1], o[4 * u + 2],
+                                              o[4 * u + 3], pol_y);
                     } else {
 #pragma unroll
                         for (int j = 0; j < 32; ++j)
@@ -335,9 +347,6 @@ nvf4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                     }
                 }
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&tmem_empty[acc]);
         }
     }
 
