@@ -43,6 +43,7 @@ constexpr int kAtom = 512;           // one scale atom: 128 rows x 4 scales
 constexpr int kAtomsPerStep = 4;     // 256 values = 16 scales = 4 atoms per row block
 constexpr int kEpiWarps = 8;         // two per TMEM lane quarter, each half the columns
 constexpr int kThreads = 64 + 32 * kEpiWarps;  // producer, MMA, epilogue warps
+constexpr int kPairThreads = kThreads + 32;      // + scale-copy warp
 constexpr uint64_t kTimeoutNs = 1000000000ull;  // 1 s per wait
 
 struct GemmArgs {
@@ -99,10 +100,11 @@ struct Cfg {
 };
 
 __device__ __forceinline__ void tile_coords(int t, const GemmArgs& a, int& mt, int& nt) {
-    const int per_group = a.group_m * a.n_tiles;
+    const int group_m = min(a.group_m, a.m_tiles);
+    const int per_group = group_m * a.n_tiles;
     const int grp = t / per_group;
-    const int first_m = grp * a.group_m;
-    const int gsize = min(a.group_m, a.m_tiles - first_m);
+    const int first_m = grp * group_m;
+    const int gsize = min(group_m, a.m_tiles - first_m);
     const int local = t - grp * per_group;
     mt = first_m + local % gsize;
     nt = local / gsize;
@@ -363,6 +365,320 @@ nvf4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
 
 
 // ---------------------------------------------------------------------------
+// CTA-pair kernel (cta_group::2): a cluster of two CTAs on two SMs computes a
+// 256 x 256 output tile.  Each CTA loads its own 128 rows of A, its 128-row
+// half of the tile's B rows, its own A scale atoms and the B scale atoms of
+// the whole 256-row N tile; every load is a 2-D TMA whose bytes are counted on
+// the even CTA's full barrier.  A dedicated copy thread of the even CTA copies
+// each stage's scale atoms into that stage's own 48-column TMEM region of both
+// CTAs (each CTA's shared memory at the same offset into its own TMEM) and
+// signals sf_ready; the MMA thread, which then issues nothing but
+// tcgen05.mma.cta_group::2 (M = 256, N = 256, K = 64), overlaps with those
+// copies (issued from one thread, the copies and MMAs would run one after the
+// other; the copies alone cost more than the MMAs).  Accumulator rows 0..127
+// live in the even CTA's TMEM and 128..255 in the odd CTA's.  Commits are multicast to both CTAs'
+// barriers; both CTAs' epilogue warps release the accumulator on the even
+// CTA's barrier.  Per CTA and k-step this moves 38 KB from L2 for 128 x 256 x
+// 256 multiply-adds (the single-CTA 128 x 256 tile moves 54 KB).
+// ---------------------------------------------------------------------------
+template <int STAGES>
+struct PairCfg {
+    static constexpr int BN = 256;
+    static constexpr int A_BYTES = kBM * kBKBytes;                 // own 128 rows of A
+    static constexpr int B_BYTES = 128 * kBKBytes;                 // own half of the N tile
+    static constexpr int SFA_BYTES = kAtomsPerStep * kAtom;        // own 128-row block
+    static constexpr int SFB_BYTES = 2 * kAtomsPerStep * kAtom;    // both 128-row blocks of N
+    static constexpr int STAGE_TX = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+    static constexpr int OFF_A = 0;
+    static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
+    static constexpr int OFF_SFA = OFF_B + STAGES * B_BYTES;
+    static constexpr int OFF_SFB = OFF_SFA + STAGES * SFA_BYTES;
+    static constexpr int OFF_BAR = OFF_SFB + STAGES * SFB_BYTES;
+    static constexpr int NBAR = 3 * STAGES + 4;                  // full, empty, sf_ready, tmem_full, tmem_empty, drain x2
+    static constexpr int OFF_SEGA = OFF_BAR + NBAR * 8;
+    static constexpr int OFF_SEGE = OFF_SEGA + NVFP4_MAX_SEGMENTS * 4;
+    static constexpr int OFF_MISC = OFF_SEGE + NVFP4_MAX_SEGMENTS * 4;
+    static constexpr int SMEM = OFF_MISC + 16 + 1024;
+    static constexpr int SFA_COL = BN;                           // one accumulator of 256 columns
+    static constexpr int SFB_COL = SFA_COL + kAtomsPerStep * 4;
+    static constexpr int SF_STRIDE = kAtomsPerStep * 12;         // 48 columns per stage region
+    static constexpr int TMEM_COLS = 512;
+    static_assert(BN + STAGES * SF_STRIDE <= TMEM_COLS, "tensor memory overflow");
+    static_assert(SMEM <= 232448, "shared memory overflow");
+};
+
+// kind::mxf4nvf4 descriptor for the pair MMA: M = 256, N = 256.
+__host__ __device__ constexpr uint32_t make_idesc_pair() {
+    return (1u << 7) | (1u << 10) | (static_cast<uint32_t>(256 >> 3) << 17) |
+           (static_cast<uint32_t>(256 >> 4) << 24);
+}
+
+template <int STAGES>
+__global__ void __launch_bounds__(kPairThreads, 1)
+nvf4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a,
+                      const __grid_constant__ CUtensorMap tmap_b,
+                      const __grid_constant__ CUtensorMap tmap_sfa,
+                      const __grid_constant__ CUtensorMap tmap_sfb, const GemmArgs args) {
+    using C = PairCfg<STAGES>;
+    constexpr int BN = C::BN;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+    uint64_t* full = bars;
+    uint64_t* empty = bars + STAGES;
+    uint64_t* sf_ready = bars + 2 * STAGES;
+    uint64_t* tmem_full = bars + 3 * STAGES;
+    uint64_t* tmem_empty = bars + 3 * STAGES + 1;
+    uint64_t* drain = bars + 3 * STAGES + 2;
+    uint64_t* drain2 = bars + 3 * STAGES + 3;
+    float* s_seg_alpha = reinterpret_cast<float*>(smem + C::OFF_SEGA);
+    int* s_seg_end = reinterpret_cast<int*>(smem + C::OFF_SEGE);
+    uint32_t* s_tmem_base = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+    volatile int* s_abort = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();             // 0: issues the pair's MMAs
+    const int pair = blockIdx.x >> 1;
+    const int npairs = gridDim.x >> 1;
+    const int total_tiles = args.m_tiles * args.n_tiles;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < STAGES; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], 1);
+            mbar_init(&sf_ready[i], 1);
+        }
+        mbar_init(tmem_full, 1);
+        mbar_init(tmem_empty, 2 * kEpiWarps);            // both CTAs' epilogue warps
+        mbar_init(drain, 1);
+        mbar_init(drain2, 1);
+        *s_abort = 0;
+        fence_mbar_init();
+        prefetch_tmap(&tmap_a);
+        prefetch_tmap(&tmap_b);
+        prefetch_tmap(&tmap_sfa);
+        prefetch_tmap(&tmap_sfb);
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(s_tmem_base, C::TMEM_COLS);
+        tmem_relinquish_pair();
+    }
+    if (threadIdx.x >= 64 && threadIdx.x < 64 + NVFP4_MAX_SEGMENTS) {
+        const int s = threadIdx.x - 64;
+        s_seg_alpha[s] = (s < args.nseg) ? __fmul_rn(*args.a_g, *args.seg_g[s]) : 0.0f;
+        s_seg_end[s] = (s < args.nseg) ? args.seg_end[s] : 0x7FFFFFFF;
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();                                      // barriers of both CTAs initialised
+    tc_fence_after();
+    const uint32_t tmem_base = *s_tmem_base;
+    const uint32_t full0_leader = mapa_shared(smem_u32(&full[0]), 0);
+    const uint32_t tmem_empty_leader = mapa_shared(smem_u32(tmem_empty), 0);
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ---------------- TMA producer (both CTAs) ----------------
+            const uint64_t pol = l2_policy_evict_last();
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t armed = 0, armed_parity = 0;   // stages the even CTA expects bytes on
+            bool ok = true;
+            for (int t = pair; t < total_tiles && ok; t += npairs) {
+                int mt, nt;
+                tile_coords(t, args, mt, nt);
+                for (int kb = 0; kb < args.k_steps; ++kb) {
+                    if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, args.timeout_ns, s_abort,
+                                           args.status)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t fb = full0_leader + stage * 8;
+                    if (rank == 0) {
+                        mbar_arrive_expect_tx(&full[stage], 2 * C::STAGE_TX);
+                        armed |= 1u << stage;
+                        armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+                    }
+                    tma_load_2d_pair(smem + C::OFF_A + stage * C::A_BYTES, &tmap_a, fb,
+                                     kb * kBKBytes, mt * 256 + rank * 128, pol);
+                    tma_load_2d_pair(smem + C::OFF_B + stage * C::B_BYTES, &tmap_b, fb,
+                                     kb * kBKBytes, nt * BN + rank * 128, pol);
+                    tma_load_2d_pair(smem + C::OFF_SFA + stage * C::SFA_BYTES, &tmap_sfa, fb,
+                                     kb * 256, mt * 2 + rank, pol);
+                    tma_load_2d_pair(smem + C::OFF_SFB + stage * C::SFB_BYTES, &tmap_sfb, fb,
+                                     kb * 256, nt * 2, pol);
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (!ok && rank == 0) {
+                // leave no copy of either CTA in flight on the stages armed here
+                int local_abort = 0;
+                for (int s = 0; s < STAGES; ++s)
+                    if (armed & (1u << s))
+                        mbar_wait_bounded(&full[s], (armed_parity >> s) & 1u, args.timeout_ns,
+                                          &local_abort, args.status);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && rank == 0) {
+            // ---------------- MMA issuer (even CTA) ----------------
+            constexpr uint32_t idesc = make_idesc_pair();
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            int i = 0;
+            for (int t = pair; t < total_tiles && ok; t += npairs, ++i) {
+                if (!mbar_wait_bounded(tmem_empty, (i & 1) ^ 1u, args.timeout_ns, s_abort,
+                                       args.status)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                for (int kb = 0; kb < args.k_steps; ++kb) {
+                    if (!mbar_wait_bounded(&sf_ready[stage], phase, args.timeout_ns, s_abort,
+                                           args.status)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const int natoms = min(kAtomsPerStep, args.atoms_per_rb - kb * kAtomsPerStep);
+                    const uint32_t sa = smem_u32(smem + C::OFF_A + stage * C::A_BYTES);
+                    const uint32_t sb = smem_u32(smem + C::OFF_B + stage * C::B_BYTES);
+                    const uint32_t sfr = tmem_base + C::BN + stage * C::SF_STRIDE;
+                    for (int j = 0; j < natoms; ++j)
+                        tc_mma_nvf4_pair(tmem_base, sdesc_kmajor_sw128(sa + j * 32),
+                                         sdesc_kmajor_sw128(sb + j * 32), idesc,
+                                         sfr + j * 4, sfr + 16 + j * 8, (kb | j) != 0);
+                    tc_commit_pair(&empty[stage], 0x3);
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (ok) tc_commit_pair(tmem_full, 0x3);
+            }
+            tc_commit_pair(drain, 0x1);
+            int local_abort = 0;
+            mbar_wait_bounded(drain, 0, args.timeout_ns, &local_abort, args.status);
+        }
+    } else if (warp == 2 + kEpiWarps) {
+        if (lane == 0 && rank == 0) {
+            // ---------------- scale copies (even CTA) ----------------
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (int t = pair; t < total_tiles && ok; t += npairs) {
+                for (int kb = 0; kb < args.k_steps; ++kb) {
+                    if (!mbar_wait_bounded(&full[stage], phase, args.timeout_ns, s_abort,
+                                           args.status)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const int natoms = min(kAtomsPerStep, args.atoms_per_rb - kb * kAtomsPerStep);
+                    const uint32_t ssfa = smem_u32(smem + C::OFF_SFA + stage * C::SFA_BYTES);
+                    const uint32_t ssfb = smem_u32(smem + C::OFF_SFB + stage * C::SFB_BYTES);
+                    const uint32_t sfr = tmem_base + C::BN + stage * C::SF_STRIDE;
+                    for (int j = 0; j < natoms; ++j) {
+                        tc_copy_scales_pair(sfr + j * 4, sdesc_scales(ssfa + j * kAtom));
+                        tc_copy_scales_pair(sfr + 16 + j * 8, sdesc_scales(ssfb + j * kAtom));
+                        tc_copy_scales_pair(sfr + 16 + j * 8 + 4,
+                                            sdesc_scales(ssfb + kAtomsPerStep * kAtom + j * kAtom));
+                    }
+                    tc_commit_pair(&sf_ready[stage], 0x1);
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            tc_commit_pair(drain2, 0x1);
+            int local_abort = 0;
+            mbar_wait_bounded(drain2, 0, args.timeout_ns, &local_abort, args.status);
+        }
+    } else {
+        // ---------------- epilogue (warps 2..9, both CTAs) ----------------
+        constexpr int kHalf = BN / 2;
+        constexpr int kChunks = kHalf / 32;
+        const int q = warp & 3;
+        const int half = (warp - 2) >> 2;
+        const int row = q * 32 + lane;
+        const uint64_t pol_y = l2_policy_evict_first();
+        int i = 0;
+        for (int t = pair; t < total_tiles; t += npairs, ++i) {
+            int mt, nt;
+            tile_coords(t, args, mt, nt);
+            int ok = 1;
+            if (lane == 0)
+                ok = mbar_wait_bounded(tmem_full, i & 1, args.timeout_ns, s_abort, args.status);
+            ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+            if (!ok) break;
+            tc_fence_after();
+            uint32_t r[kChunks][32];
+            const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + half * kHalf;
+#pragma unroll
+            for (int ch = 0; ch < kChunks; ++ch) tmem_ld_32cols(taddr + ch * 32, r[ch]);
+            tmem_ld_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(tmem_empty_leader);
+            const int m = mt * 256 + static_cast<int>(rank) * 128 + row;
+            uint16_t* yrow = args.y + static_cast<int64_t>(m) * args.ldy;
+#pragma unroll
+            for (int ch = 0; ch < kChunks; ++ch) {
+                const int n0 = nt * BN + half * kHalf + ch * 32;
+                int s0 = 0;
+                while (s0 < args.nseg - 1 && n0 >= s_seg_end[s0]) ++s0;
+                const bool one_seg = (s0 == args.nseg - 1) || (n0 + 31 < s_seg_end[s0]);
+                if (m < args.M && n0 < args.N) {
+                    float v[32];
+                    if (one_seg) {
+                        const float al = s_seg_alpha[s0];
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) v[j] = __fmul_rn(__uint_as_float(r[ch][j]), al);
+                    } else {
+                        int s = s0;
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) {
+                            while (s < args.nseg - 1 && n0 + j >= s_seg_end[s]) ++s;
+                            v[j] = __fmul_rn(__uint_as_float(r[ch][j]), s_seg_alpha[s]);
+                        }
+                    }
+                    uint32_t o[16];
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) o[j] = pack_bf16x2(v[2 * j], v[2 * j + 1]);
+                    if (n0 + 32 <= args.N) {
+#pragma unroll
+                        for (int u = 0; u < 4; ++u)
+                            st_global_v4_hint(yrow + n0 + 8 * u, o[4 * u], o[4 * u + 1], o[4 * u + 2],
+                                              o[4 * u + 3], pol_y);
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j)
+                            if (n0 + j < args.N)
+                                yrow[n0 + j] = static_cast<uint16_t>((o[j >> 1] >> (16 * (j & 1))) & 0xFFFFu);
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();                                      // no CTA leaves while its peer may signal it
+    tc_fence_after();
+    if (warp == 1) {
+        __syncwarp();
+        tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
+    }
+}
+
+// ---------------------------------------------------------------------------
 // Bounded-wait self-test: one thread waits on a barrier nothing arrives on.
 // The wait must give up after limit_ns and set the device status word; the
 // context stays usable.  Lets the timeout path be tested without a fault.
@@ -417,6 +733,25 @@ bool make_code_map(CUtensorMap* m, const uint8_t* base, int64_t rows, int64_t ro
     return r == CUDA_SUCCESS;
 }
 
+// Scale bytes in the tensor-core layout viewed as [row blocks, atoms * 64]
+// 8-byte units: one box of 256 units (2 KB) x box_rows row blocks is one
+// 256-element k-step of box_rows 128-row blocks.  Out-of-range row blocks and
+// k positions read as zero.
+bool make_sf_map(CUtensorMap* m, const uint8_t* base, int64_t rowblocks, int64_t atoms_per_rb,
+                 int box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(atoms_per_rb * 64),
+                          static_cast<cuuint64_t>(rowblocks)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(atoms_per_rb * kAtom)};
+    cuuint32_t box[2] = {256, static_cast<cuuint32_t>(box_rows)};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT64, 2, const_cast<uint8_t*>(base), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 int* device_status_ptr() {
     static int* cache[64] = {nullptr};
     int dev = 0;
@@ -451,6 +786,48 @@ nvfp4_status launch_gemm(const uint8_t* a_codes, const uint8_t* w_codes, GemmArg
     const int tiles = args.m_tiles * args.n_tiles;
     const int grid = tiles < dev.sms ? tiles : dev.sms;
     kern<<<grid, kThreads, Cf::SMEM, stream>>>(ta, tb, args);
+    return cuda_status(cudaGetLastError());
+}
+
+template <int STAGES>
+nvfp4_status launch_gemm_pair(const uint8_t* a_codes, const uint8_t* w_codes, GemmArgs& args,
+                              const DeviceInfo& dev, cudaStream_t stream) {
+    using Cf = PairCfg<STAGES>;
+    auto kern = nvf4_gemm_pair_kernel<STAGES>;
+    static bool attr_set[64] = {false};
+    int devid = 0;
+    if (cudaGetDevice(&devid) != cudaSuccess || devid < 0 || devid >= 64) return NVFP4_ERR_CUDA;
+    if (!attr_set[devid]) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::SMEM) !=
+            cudaSuccess)
+            return NVFP4_ERR_CUDA;
+        attr_set[devid] = true;
+    }
+    CUtensorMap ta, tb, tsa, tsb;
+    const int64_t a_rb = (args.M + 127) / 128, w_rb = (args.N + 127) / 128;
+    if (!make_code_map(&ta, a_codes, args.M, args.K / 2, 128)) return NVFP4_ERR_CUDA;
+    if (!make_code_map(&tb, w_codes, args.N, args.K / 2, 128)) return NVFP4_ERR_CUDA;
+    if (!make_sf_map(&tsa, args.a_sf, a_rb, args.atoms_per_rb, 1)) return NVFP4_ERR_CUDA;
+    if (!make_sf_map(&tsb, args.w_sf, w_rb, args.atoms_per_rb, 2)) return NVFP4_ERR_CUDA;
+    args.m_tiles = (args.M + 255) / 256;
+    args.n_tiles = (args.N + Cf::BN - 1) / Cf::BN;
+    const int tiles = args.m_tiles * args.n_tiles;
+    const int max_pairs = dev.sms / 2;
+    const int pairs = tiles < max_pairs ? tiles : max_pairs;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * pairs, 1, 1);
+    cfg.blockDim = dim3(kPairThreads, 1, 1);
+    cfg.dynamicSmemBytes = Cf::SMEM;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ta, tb, tsa, tsb, args);
+    if (e != cudaSuccess) return NVFP4_ERR_CUDA;
     return cuda_status(cudaGetLastError());
 }
 
@@ -492,7 +869,10 @@ nvfp4_status gemm_impl(const uint8_t* a_codes, const uint8_t* a_sf, const float*
     args.k_steps = static_cast<int>((K + 255) / 256);
     args.atoms_per_rb = static_cast<int>((K + 63) / 64);
     args.w_rowblocks = static_cast<int>((N + 127) / 128);
-    args.group_m = 16;
+    // Raster: when the quantized activation fits comfortably in L2, sweep every
+    // M tile for each N tile (the weight then streams from HBM once);
+    // otherwise walk bands of 16 M tiles.
+    args.group_m = (M * (K / 2) <= (int64_t(48) << 20)) ? 1 << 30 : 16;
     args.nseg = nseg;
     for (int s = 0; s < nseg; ++s) {
         args.seg_end[s] = static_cast<int>(segs[s].n_offset + segs[s].n_size);
@@ -503,7 +883,7 @@ nvfp4_status gemm_impl(const uint8_t* a_codes, const uint8_t* a_sf, const float*
     cudaStream_t cs = as_stream(stream);
     // The configuration depends on M only, so a fused GEMM and its per-module
     // GEMMs accumulate every output element identically.
-    if (M > 256) return launch_gemm<256, 4, 1>(a_codes, w_codes, args, dev, cs);
+    if (M > 256) return launch_gemm_pair<5>(a_codes, w_codes, args, dev, cs);
     return launch_gemm<128, 6, 2>(a_codes, w_codes, args, dev, cs);
 }
 
