@@ -90,6 +90,32 @@ nvfp4_status nvfp4_global_scale(const void* x, int64_t rows, int64_t cols, int64
                                 float* g_out, float* amax_out, void* workspace,
                                 void* stream);
 
+/* Bytes of the library-owned scratch array behind nvfp4_global_scale_noalloc. */
+#define NVFP4_NOALLOC_SCRATCH_BYTES 256
+
+/* nvfp4_global_scale without a caller workspace, for callers that cannot
+ * allocate device memory -- for example code plugged into a host framework
+ * whose memory pool forbids outside cudaMalloc calls, or a hook that runs
+ * where allocation is not permitted -- and so cannot hand over the
+ * zero-initialised workspace nvfp4_global_scale needs.  The paper has no
+ * counterpart; this is a property of the library, not of the method.
+ * The workspace lives instead in a file-scope __device__ array of
+ * NVFP4_NOALLOC_SCRATCH_BYTES bytes that every GPU loading the library holds
+ * until the process exits; the call needs 8 of those bytes and returns
+ * NVFP4_ERR_UNSUPPORTED_SHAPE if its need ever exceeded the array.  The call
+ * allocates nothing (no cudaMalloc, no allocating library routine): it
+ * clears the part of the array that must start at zero with a
+ * cudaMemsetAsync on `stream`, then launches the same kernel as
+ * nvfp4_global_scale.  The first call on each device looks up the array's
+ * device address (cudaGetSymbolAddress) with that device current; make that
+ * first call before any stream capture.  All calls on a device share the one
+ * array, which keeps the last call's contents: calls that overlap on the GPU
+ * (different streams, no ordering between them) race and may return a wrong
+ * g; serialize them.  Arguments, results and requirements as
+ * nvfp4_global_scale, without `workspace`. */
+nvfp4_status nvfp4_global_scale_noalloc(const void* x, int64_t rows, int64_t cols, int64_t ld,
+                                        float* g_out, float* amax_out, void* stream);
+
 /* Bytes of the scale buffer for a [rows, cols] tensor in `layout`:
  * LINEAR rows * cols/16; TCGEN05 roundup(rows,128) * roundup(cols/16,4).
  * cols must be a multiple of 16. */

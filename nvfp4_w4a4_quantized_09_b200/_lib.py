@@ -25,6 +25,7 @@ SF_TCGEN05 = 1
 
 MAX_SEGMENTS = 16
 GLOBAL_SCALE_WORKSPACE_BYTES = 256
+NOALLOC_SCRATCH_BYTES = 256
 
 # Every symbol include/nvfp4.h declares, with (restype, argtypes).
 P = ctypes.c_void_p
@@ -40,6 +41,7 @@ class Segment(ctypes.Structure):
 
 SIGNATURES = {
     "nvfp4_global_scale": (ST, [P, I64, I64, I64, P, P, P, P]),
+    "nvfp4_global_scale_noalloc": (ST, [P, I64, I64, I64, P, P, P]),
     "nvfp4_sf_bytes": (ST, [I64, I64, I32, ctypes.POINTER(ctypes.c_size_t)]),
     "nvfp4_quantize": (ST, [P, I64, I64, I64, P, P, P, I32, P]),
     "nvfp4_quantize_slice": (ST, [P, I64, I64, I64, P, P, P, I32, I64, I64, P]),

@@ -409,6 +409,43 @@ nvfp4_status current_device_info(DeviceInfo* info) {
 
 using namespace nvfp4;
 
+// ---------------------------------------------------------------------------
+// Global scale for callers that cannot allocate: the workspace is a
+// file-scope device array (one per device that loads the library), whose
+// address host code must obtain with cudaGetSymbolAddress -- the array's name
+// in host code is only a host-side stand-in.
+// ---------------------------------------------------------------------------
+static __device__ __align__(256) unsigned char g_noalloc_scratch[NVFP4_NOALLOC_SCRATCH_BYTES];
+
+static nvfp4_status noalloc_scratch_ptr(void** out) {
+    static void* cache[64] = {nullptr};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return NVFP4_ERR_CUDA;
+    if (!cache[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return NVFP4_ERR_CUDA;
+        cache[dev] = p;
+    }
+    *out = cache[dev];
+    return NVFP4_OK;
+}
+
+extern "C" nvfp4_status nvfp4_global_scale_noalloc(const void* x, int64_t rows, int64_t cols,
+                                                   int64_t ld, float* g_out, float* amax_out,
+                                                   void* stream) {
+    static_assert(sizeof(GlobalScaleWorkspace) <= NVFP4_NOALLOC_SCRATCH_BYTES,
+                  "scratch array too small for the global-scale workspace");
+    if (sizeof(GlobalScaleWorkspace) > NVFP4_NOALLOC_SCRATCH_BYTES) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (!g_out || rows < 0 || cols < 0) return NVFP4_ERR_INVALID_ARG;
+    void* ws = nullptr;
+    nvfp4_status st = noalloc_scratch_ptr(&ws);
+    if (st != NVFP4_OK) return st;
+    // the workspace must start at zero: clear it on the stream (no allocation)
+    if (cudaMemsetAsync(ws, 0, sizeof(GlobalScaleWorkspace), as_stream(stream)) != cudaSuccess)
+        return NVFP4_ERR_CUDA;
+    return nvfp4_global_scale(x, rows, cols, ld, g_out, amax_out, ws, stream);
+}
+
 extern "C" nvfp4_status nvfp4_sf_bytes(int64_t rows, int64_t cols, nvfp4_sf_layout layout,
                                        size_t* bytes) {
     if (!bytes || rows < 0 || cols < 0) return NVFP4_ERR_INVALID_ARG;
