@@ -39,6 +39,25 @@ WORKLOAD = "fused GDN input projection prefill: X bf16 [8192,5120] -> W q/k/v/z/
 L2_FLUSH_BYTES = 256 << 20
 
 
+def gemm_traffic():
+    """DRAM bytes per launch of the fused GEMM from the committed ncu record,
+    or None when the kernel source changed since the counters were taken."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "traffic_gemm_pair_fused_gdn_8192x24704x5120.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+        h = hashlib.sha256()
+        for src in rec["sources"]:
+            with open(os.path.join(ROOT, src), "rb") as f:
+                h.update(f.read())
+        if h.hexdigest()[:16] != rec["source_sha256_16"]:
+            return None
+        return int(rec["dram_bytes_read"] + rec["dram_bytes_write"])
+    except (OSError, KeyError, ValueError):
+        return None
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -195,7 +214,8 @@ def run_ours(args, dev, world, rank):
     fp4_peak = peaks["bf16_tflops"] * 4.0
     roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(fp4_peak, 1),
                 "unit": "TFLOP/s", "frac": round(achieved / fp4_peak, 4),
-                "traffic": None, "kernel": "nvf4_gemm_kernel (fused, 8192x24704x5120)",
+                "traffic": gemm_traffic(), "kernel": "nvf4_gemm_pair_kernel (fused, 8192x24704x5120)",
+                "algorithmic_flop_per_launch": flops,
                 "peak_source": f"{peak_src} bf16 burst x 4 (nominal dense FP4/BF16 ratio 9/2.25)"}
 
     # quantizer alone on the [32768, 5120] activation: global scale + quantize
