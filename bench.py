@@ -250,6 +250,99 @@ def run_ours(args, dev, world, rank):
         "hbm_peak_GBps": hbm, "peak_source": peak_src}
     del xq, cq, sq
 
+    # decode-shaped sweep (weight-bandwidth bound): K = 5120, M tokens, rotating
+    # weight copies (together larger than 2 x L2) so the weights come from HBM
+    decode = []
+    if not args.no_decode:
+        for Nd in (5120, 24640, 34816):
+            copies = max(4, int((300 << 20) // (Nd * 2880)) + 1)
+            if Nd == 24640:
+                mods = synth.GDN_MODULES_DECODE
+                wsets = [nv.FusedWeight.from_modules(
+                    [w for _, w in synth.gdn_weights(mods, device=dev)]) for _ in range(copies)]
+            else:
+                w = synth.gaussian_weights(Nd, K_HID, 0.015, seed=20, device=dev)
+                wq0 = nv.quantize_tensor(w)
+                wsets = [nv.QuantizedTensor(wq0.codes.clone(), wq0.sf.clone(), wq0.g, Nd, K_HID)
+                         for _ in range(copies)]
+                del w
+            for Mtok in (1, 8, 32, 128):
+                xd = synth.student_t_activations(Mtok, K_HID, seed=100 + Mtok, device=dev)
+                ad = nv.quantize_tensor(xd)
+                yd = torch.empty(Mtok, Nd, dtype=torch.bfloat16, device=dev)
+                evs = []
+                for it in range(3 * copies + 30):
+                    wq = wsets[it % copies]
+                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    e0.record(stream)
+                    if isinstance(wq, nv.FusedWeight):
+                        nv.fused_gemm(ad, wq.codes, wq.sf, wq.segments(), yd)
+                    else:
+                        nv.gemm(ad, wq, yd)
+                    e1.record(stream)
+                    evs.append((e0, e1))
+                torch.cuda.synchronize()
+                us = float(np.median([a_.elapsed_time(b_) for a_, b_ in evs[copies:]])) * 1e3
+                nbytes = Nd * K_HID * 0.5625 + Mtok * K_HID * 0.5625 + 2 * Mtok * Nd
+                decode.append({"M": Mtok, "N": Nd, "us": round(us, 2),
+                               "GBps": round(nbytes / (us * 1e-6) / 1e9, 1),
+                               "frac_hbm": round(nbytes / (us * 1e-6) / 1e9 / peaks["hbm_gbs"], 3)})
+            del wsets
+        torch.cuda.empty_cache()
+
+    # the 32K-token MLP (gate_up GEMM, SiLU(gate)*up, requantization, down GEMM)
+    mlp_line = None
+    if not args.no_mlp:
+        Mm, Hm, Fm = 32768, K_HID, synth.MLP_WIDTH
+        xm = synth.student_t_activations(Mm, Hm, seed=1, device=dev)
+        wq_gu = nv.quantize_tensor(synth.gaussian_weights(2 * Fm, Hm, 0.015, seed=20, device=dev))
+        wq_dn = nv.quantize_tensor(synth.gaussian_weights(Hm, Fm, 0.01, seed=21, device=dev))
+        am = nv.quantize_tensor(xm)
+        gu = torch.empty(Mm, 2 * Fm, dtype=torch.bfloat16, device=dev)
+        hm = torch.empty(Mm, Fm, dtype=torch.bfloat16, device=dev)
+        ym = torch.empty(Mm, Hm, dtype=torch.bfloat16, device=dev)
+        hcodes = torch.empty(Mm, Fm // 2, dtype=torch.uint8, device=dev)
+        hsf = torch.empty(nv.sf_bytes(Mm, Fm), dtype=torch.uint8, device=dev)
+        hg = torch.empty(1, dtype=torch.float32, device=dev)
+        hq = nv.QuantizedTensor(hcodes, hsf, hg, Mm, Fm)
+        recs = []
+        for it in range(args.warmup + 5):
+            flush.zero_()
+            e = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+            e[0].record(stream)
+            nv.gemm(am, wq_gu, gu)
+            e[1].record(stream)
+            nv.silu_mul(gu, hm)
+            e[2].record(stream)
+            nv.global_scale(hm, hg, amax)
+            e[3].record(stream)
+            nv.quantize(hm, hg, nv.SF_TCGEN05, hcodes, hsf)
+            e[4].record(stream)
+            nv.gemm(hq, wq_dn, ym)
+            e[5].record(stream)
+            recs.append(e)
+        torch.cuda.synchronize()
+        recs = recs[args.warmup:]
+        t = [float(np.median([r[i].elapsed_time(r[i + 1]) for r in recs])) * 1e3 for i in range(5)]
+        f_gu = 2.0 * Mm * 2 * Fm * Hm
+        f_dn = 2.0 * Mm * Hm * Fm
+        fp4 = peaks["bf16_tflops"] * 4.0
+        hbytes = Mm * Fm * 2
+        mlp_line = {
+            "workload": "MLP 32K prefill: X [32768,5120] -> gate_up [34816,5120] -> SiLU*up -> down [5120,17408]",
+            "gate_up_us": round(t[0], 1), "gate_up_TFLOPs": round(f_gu / (t[0] * 1e-6) / 1e12, 1),
+            "gate_up_frac": round(f_gu / (t[0] * 1e-6) / 1e12 / fp4, 4),
+            "silu_mul_us": round(t[1], 1),
+            "silu_mul_GBps": round(3 * hbytes / (t[1] * 1e-6) / 1e9, 1),
+            "h_global_scale_us": round(t[2], 1), "h_quantize_us": round(t[3], 1),
+            "h_quantize_GBps": round(hbytes * 1.28125 / (t[3] * 1e-6) / 1e9, 1),
+            "down_us": round(t[4], 1), "down_TFLOPs": round(f_dn / (t[4] * 1e-6) / 1e12, 1),
+            "down_frac": round(f_dn / (t[4] * 1e-6) / 1e12 / fp4, 4),
+            "total_us": round(sum(t), 1),
+            "total_TFLOPs": round((f_gu + f_dn) / (sum(t) * 1e-6) / 1e12, 1)}
+        del xm, wq_gu, wq_dn, am, gu, hm, ym, hcodes, hsf
+        torch.cuda.empty_cache()
+
     # end to end through the public API with host buffers: pinned X in, Y out
     x_host = x.cpu().pin_memory()
     y_host = torch.empty(M, N, dtype=torch.bfloat16).pin_memory()
@@ -290,7 +383,7 @@ def run_ours(args, dev, world, rank):
                    "l2": "flushed between timed steps (256 MB write)"},
         "components_us": {"global_scale+quantize": round(float(np.mean(quant_ms)) * 1e3, 2),
                           "fused_gemm": round(gemm_avg_ms * 1e3, 2)},
-        "roofline": roofline, "quantizer": quantizer, "e2e": e2e,
+        "roofline": roofline, "quantizer": quantizer, "e2e": e2e, "decode_sweep": decode, "mlp_32k": mlp_line,
         "gpu_launches": 3 * args.steps,
         "clocks": clk.summary(),
         "activation_stats": act_stats(x),
@@ -381,6 +474,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-mlp", action="store_true")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -192,6 +192,19 @@ nvfp4_status nvfp4_fused_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const
                               void* y, int64_t ldy, int64_t M, int64_t K,
                               void* stream);
 
+/* MLP intermediate for the W4A4 down projection: h[r, c] = BF16_RNE(
+ * fl32(SiLU(gate) * up)) with gate = gate_up[r, c], up = gate_up[r, f + c]
+ * (BF16, row stride ld elements, device) and SiLU(v) = v / (1 + e^-v)
+ * evaluated in FP32 (expf, IEEE division); h is BF16 [rows, f], row stride
+ * ldh (device).  Within one BF16 ulp of the value rounded once from exact
+ * arithmetic.  Requirements: f, ld, ldh multiples of 8; ld >= 2f, ldh >= f;
+ * pointers 16-byte aligned.
+ * Source: W4A4 on every linear layer, the MLP down projection included
+ * (chatpaper.ai abstract); the SiLU-gated MLP is the plain reading of the
+ * 27B hybrid's MLP block, which the pages do not describe. */
+nvfp4_status nvfp4_silu_mul(const void* gate_up, int64_t rows, int64_t f, int64_t ld, void* h,
+                            int64_t ldh, void* stream);
+
 /* Synchronizes `stream`, then reads and clears the library's device status
  * word on the current device: NVFP4_ERR_TIMEOUT if a bounded wait inside a
  * kernel gave up since the last call (that kernel's output is then invalid),

@@ -27,7 +27,7 @@ from ._lib import SF_LINEAR, SF_TCGEN05, MAX_SEGMENTS, Nvfp4Error
 __all__ = [
     "SF_LINEAR", "SF_TCGEN05", "MAX_SEGMENTS", "Nvfp4Error", "QuantizedTensor",
     "global_scale", "sf_bytes", "quantize", "quantize_into", "quantize_tensor",
-    "gemm", "fused_gemm", "FusedWeight", "linear", "last_device_status",
+    "gemm", "fused_gemm", "FusedWeight", "linear", "silu_mul", "mlp", "last_device_status",
     "debug_wait_timeout", "library_path",
 ]
 
@@ -216,6 +216,25 @@ def linear(x: torch.Tensor, w, y: Optional[torch.Tensor] = None, stream=None) ->
     if isinstance(w, FusedWeight):
         return fused_gemm(a, w.codes, w.sf, w.segments(), y, stream)
     return gemm(a, w, y, stream)
+
+
+def silu_mul(gate_up: torch.Tensor, h: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """h = SiLU(gate_up[:, :f]) * gate_up[:, f:] in BF16 (the MLP intermediate)."""
+    _check_bf16_matrix(gate_up, "gate_up")
+    rows, two_f = gate_up.shape
+    f = two_f // 2
+    if h is None:
+        h = torch.empty(rows, f, dtype=torch.bfloat16, device=gate_up.device)
+    _lib.check("nvfp4_silu_mul", _lib.lib().nvfp4_silu_mul(
+        _ptr(gate_up), rows, f, gate_up.stride(0), _ptr(h), h.stride(0), _stream(stream)))
+    return h
+
+
+def mlp(x: torch.Tensor, w_gate_up, w_down, stream=None) -> torch.Tensor:
+    """W4A4 SiLU-gated MLP: gate_up GEMM, SiLU(gate)*up, requantization, down GEMM."""
+    gu = linear(x, w_gate_up, stream=stream)
+    h = silu_mul(gu, stream=stream)
+    return linear(h, w_down, stream=stream)
 
 
 def last_device_status(stream=None) -> int:

@@ -87,6 +87,8 @@ def _L():
         lib.oracle_e4m3_encode_array.argtypes = [P, I64, P]
         lib.oracle_bf16_from_double_array.argtypes = [P, I64, P]
         lib.oracle_num_threads.restype = ctypes.c_int
+        lib.oracle_silu_mul.argtypes = [P, I64, I64, I64, P]
+        lib.oracle_silu_mul.restype = None
         _lib = lib
     return _lib
 
@@ -227,6 +229,17 @@ def linear(a_codes, a_sf, g_a, w_codes, w_sf, segments, row_ids=None):
     alpha = segment_alpha(g_a, segments)
     y64 = gemm_f64(A, W, alpha, row_ids)
     return y64, bf16_from_double(y64)
+
+
+def silu_mul(gate_up_bf16: np.ndarray) -> np.ndarray:
+    """h = bf16(SiLU(gate) * up) from a BF16 [rows, 2f] gate_up matrix (uint16 bits)."""
+    gu = _c(gate_up_bf16, np.uint16)
+    rows, two_f = gu.shape
+    assert two_f % 2 == 0
+    f = two_f // 2
+    h = np.empty((rows, f), np.uint16)
+    _L().oracle_silu_mul(_ptr(gu), rows, f, two_f, _ptr(h))
+    return h
 
 
 def num_threads() -> int:

@@ -330,3 +330,25 @@ int oracle_num_threads(void)
     return 1;
 #endif
 }
+
+/* ---------------------------------------------------------------------- */
+/* MLP intermediate: h = SiLU(gate) * up                                   */
+/* ---------------------------------------------------------------------- */
+
+/* The MLP's down projection consumes h = SiLU(gate) * up, with gate the
+ * first f columns and up the next f columns of the BF16 gate_up output
+ * (row stride ld elements); SiLU(v) = v / (1 + e^-v).  Computed in FP64 from
+ * the exact BF16 values and rounded once to BF16.  The pages quantize every
+ * linear layer, the down projection included (chatpaper.ai abstract: W4A4 on
+ * all linear layers); the SiLU-gated MLP is the plain reading of a Qwen-style
+ * MLP block, which the pages do not describe. */
+void oracle_silu_mul(const uint16_t* gu, int64_t rows, int64_t f, int64_t ld, uint16_t* h)
+{
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t c = 0; c < f; ++c) {
+            double g = (double)bf16_to_float(gu[r * ld + c]);
+            double u = (double)bf16_to_float(gu[r * ld + f + c]);
+            double s = g / (1.0 + exp(-g));
+            h[r * f + c] = oracle_bf16_from_double(s * u);
+        }
+}

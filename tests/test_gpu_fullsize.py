@@ -118,3 +118,46 @@ def test_decode_sweep(which, M):
     alpha = oracle.segment_alpha(ga, segs)
     assert_gemm_matches(host_bits(y[torch.from_numpy(rows).to(DEV)]), A, W, alpha,
                         label=f"decode M={M} {which}")
+
+
+def test_mlp_32k_prefill_sampled():
+    # the 32K-token MLP: gate_up [34816, 5120], SiLU(gate)*up, requantization of
+    # h [32768, 17408], down [5120, 17408]; every stage on sampled rows
+    M, H, F = 32768, 5120, 17408
+    x = synth.student_t_activations(M, H, seed=1, device=DEV)
+    w_gu = synth.gaussian_weights(2 * F, H, 0.015, seed=20, device=DEV)
+    w_dn = synth.gaussian_weights(H, F, 0.01, seed=21, device=DEV)
+    a = nv.quantize_tensor(x)
+    wq_gu = nv.quantize_tensor(w_gu)
+    wq_dn = nv.quantize_tensor(w_dn)
+    gu = nv.gemm(a, wq_gu)
+    h = nv.silu_mul(gu)
+    hq = nv.quantize_tensor(h)
+    y = nv.gemm(hq, wq_dn)
+    torch.cuda.synchronize()
+    rows = sample_rows(M, 6, 7)
+    rid = torch.from_numpy(rows).to(DEV)
+    xb = host_bits(x)
+    ga, _ = oracle.global_scale(xb)
+    ca, sa = oracle.quantize(xb[rows], ga)
+    wgb = host_bits(w_gu)
+    gw, _ = oracle.global_scale(wgb)
+    cw, sw = oracle.quantize(wgb, gw)
+    assert np.array_equal(np_u8(wq_gu.codes), cw)
+    assert_gemm_matches(host_bits(gu[rid]), dequant(ca, sa), dequant(cw, sw),
+                        oracle.segment_alpha(ga, [(0, 2 * F, gw)]), label="gate_up 32K")
+    del cw, sw
+    hb_rows = host_bits(h[rid])
+    ref_h = oracle.silu_mul(host_bits(gu[rid]))
+    assert np.max(np.abs(hb_rows.astype(np.int32) - ref_h.astype(np.int32))) <= 1
+    hb = host_bits(h)
+    gh, _ = oracle.global_scale(hb)
+    assert np_f32(hq.g)[0] == gh
+    ch, sh = oracle.quantize(hb_rows, gh)
+    assert np.array_equal(np_u8(hq.codes)[rows], ch)
+    del hb
+    wdb = host_bits(w_dn)
+    gd, _ = oracle.global_scale(wdb)
+    cd, sd = oracle.quantize(wdb, gd)
+    assert_gemm_matches(host_bits(y[rid]), dequant(ch, sh), dequant(cd, sd),
+                        oracle.segment_alpha(gh, [(0, H, gd)]), label="down 32K")

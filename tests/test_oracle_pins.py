@@ -419,3 +419,50 @@ def test_quantized_gemm_close_to_bf16_gemm():
     ref = oracle.bf16_bits_to_f64(bf16_bits_of(x)) @ oracle.bf16_bits_to_f64(bf16_bits_of(w)).T
     rel = np.linalg.norm(y64 - ref) / np.linalg.norm(ref)
     assert 0.01 < rel < 0.2
+
+
+# ---------------------------------------------------------------------------
+# MLP intermediate h = SiLU(gate) * up
+# ---------------------------------------------------------------------------
+
+def test_silu_mul_closed_forms():
+    # SiLU(0) = 0; SiLU(v) - SiLU(-v) = v (odd part of v*sigmoid(v)); up = 1 and
+    # up = -1 mirror; large |v| limits (SiLU -> v, SiLU -> 0)
+    v = np.array([0.0, 0.5, 1.0, 2.0, 3.0, 8.0, 40.0, -40.0, 100.0], np.float32)
+    gu = np.concatenate([np.concatenate([v, -v])[None, :],
+                         np.ones((1, 2 * v.size), np.float32)], axis=1)
+    # rows: [gate = (v, -v), up = 1]
+    bits = bf16_bits_of(gu)
+    h = oracle.bf16_bits_to_f64(oracle.silu_mul(bits))[0]
+    n = v.size
+    assert h[0] == 0.0
+    for i in range(n):
+        pos, neg = h[i], h[n + i]
+        # difference is v up to the BF16 rounding of both terms
+        assert abs((pos - neg) - v[i]) <= 2.0 ** -8 * (abs(pos) + abs(neg)) + 1e-30
+    assert h[6] == 40.0 and h[n + 6] == 0.0 or abs(h[n + 6]) < 1e-15
+    assert h[8] == 100.0
+    up = np.concatenate([np.full(2 * n, 3.0, np.float32)])
+    gu3 = np.concatenate([np.concatenate([v, -v]), -up])[None, :]
+    h3 = oracle.bf16_bits_to_f64(oracle.silu_mul(bf16_bits_of(gu3)))[0]
+    # up = -3: h = -3 SiLU(v), exact to one BF16 rounding of the FP64 product
+    assert np.all(np.abs(h3 + 3 * oracle.bf16_bits_to_f64(oracle.silu_mul(bits))[0]) <=
+                  2.0 ** -7 * np.abs(h3) + 1e-30)
+
+
+def test_silu_mul_single_rounding_matches_exact_value():
+    # for random inputs, h is the BF16 value nearest to g*sigmoid(g)*u (checked
+    # through the neighbours of the returned BF16 value, in FP64)
+    rng = np.random.default_rng(17)
+    gu = (rng.standard_normal((16, 64)) * 3).astype(np.float32)
+    bits = bf16_bits_of(gu)
+    h = oracle.silu_mul(bits)
+    vals = oracle.bf16_bits_to_f64(bits)
+    g, u = vals[:, :32], vals[:, 32:]
+    exact = g / (1 + np.exp(-g)) * u
+    hv = oracle.bf16_bits_to_f64(h)
+    up = oracle.bf16_bits_to_f64(h + 1)
+    dn = oracle.bf16_bits_to_f64(h - 1)
+    d0 = np.abs(hv - exact)
+    assert np.all((d0 <= np.abs(up - exact)) | (h == 0x7F7F))
+    assert np.all((d0 <= np.abs(dn - exact)) | ((h & 0x7FFF) == 0))
