@@ -270,21 +270,41 @@ def run_ours(args, dev, world, rank):
                 xd = synth.student_t_activations(Mtok, K_HID, seed=100 + Mtok, device=dev)
                 ad = nv.quantize_tensor(xd)
                 yd = torch.empty(Mtok, Nd, dtype=torch.bfloat16, device=dev)
-                evs = []
-                for it in range(3 * copies + 30):
-                    wq = wsets[it % copies]
-                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                    e0.record(stream)
+
+                def launch(wq):
                     if isinstance(wq, nv.FusedWeight):
                         nv.fused_gemm(ad, wq.codes, wq.sf, wq.segments(), yd)
                     else:
                         nv.gemm(ad, wq, yd)
+                # eager: one call at a time, host launch cost included
+                evs = []
+                for it in range(3 * copies + 30):
+                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    e0.record(stream)
+                    launch(wsets[it % copies])
                     e1.record(stream)
                     evs.append((e0, e1))
                 torch.cuda.synchronize()
-                us = float(np.median([a_.elapsed_time(b_) for a_, b_ in evs[copies:]])) * 1e3
+                us_eager = float(np.median([a_.elapsed_time(b_) for a_, b_ in evs[copies:]])) * 1e3
+                # device: the launches over all weight copies captured in one CUDA
+                # graph and replayed back to back (how a decode loop issues them)
+                graph = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(graph):
+                    for wq in wsets:
+                        launch(wq)
+                graph.replay()
+                torch.cuda.synchronize()
+                reps = 20
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                for _ in range(reps):
+                    graph.replay()
+                e1.record(stream)
+                torch.cuda.synchronize()
+                us = e0.elapsed_time(e1) * 1e3 / (reps * copies)
+                del graph
                 nbytes = Nd * K_HID * 0.5625 + Mtok * K_HID * 0.5625 + 2 * Mtok * Nd
-                decode.append({"M": Mtok, "N": Nd, "us": round(us, 2),
+                decode.append({"M": Mtok, "N": Nd, "us": round(us, 2), "us_eager": round(us_eager, 2),
                                "GBps": round(nbytes / (us * 1e-6) / 1e9, 1),
                                "frac_hbm": round(nbytes / (us * 1e-6) / 1e9 / peaks["hbm_gbs"], 3)})
             del wsets

@@ -361,6 +361,8 @@ nvf4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
     }
 }
 
+#include "gemm_decode.cuh"
+
 }  // namespace
 
 
@@ -831,6 +833,63 @@ nvfp4_status launch_gemm_pair(const uint8_t* a_codes, const uint8_t* w_codes, Ge
     return cuda_status(cudaGetLastError());
 }
 
+// Few tokens (M <= 128): operands swapped, K split over a cluster.  NT, the
+// ring depth and the split depend on M and K only.
+nvfp4_status launch_gemm_decode(const uint8_t* a_codes, const uint8_t* w_codes,
+                                GemmArgs& args, cudaStream_t stream) {
+    auto kern = nvf4_gemm_decode_kernel;
+    static bool attr_set[64] = {false};
+    static int max_clusters[64][kDecMaxSplit + 1][9];   // [device][split][nt_tok / 16]
+    int devid = 0;
+    if (cudaGetDevice(&devid) != cudaSuccess || devid < 0 || devid >= 64) return NVFP4_ERR_CUDA;
+    if (!attr_set[devid]) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(kDecStageBudget + 4096)) != cudaSuccess)
+            return NVFP4_ERR_CUDA;
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100) !=
+            cudaSuccess)
+            return NVFP4_ERR_CUDA;
+        attr_set[devid] = true;
+    }
+    DecodeArgs d;
+    d.g = args;
+    d.nt_tok = ((args.M + 15) / 16) * 16;
+    dec_config(d.nt_tok, &d.stages, &d.nparts, &d.nacc);
+    d.split = 1;
+    while (d.split < kDecMaxSplit && args.k_steps / (2 * d.split) >= 4) d.split *= 2;
+    d.g.m_tiles = 1;
+    d.g.n_tiles = (args.N + kBM - 1) / kBM;
+    const uint32_t smem = dec_layout(d.nt_tok, d.stages, d.nparts).bytes;
+
+    cudaLaunchConfig_t cfg = {};
+    cfg.blockDim = dim3(kDecThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = static_cast<unsigned>(d.split);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    // persistent: as many clusters as can be resident at once
+    int& slots = max_clusters[devid][d.split][d.nt_tok / 16];
+    if (slots <= 0) {
+        cfg.gridDim = dim3(static_cast<unsigned>(d.split), 1, 1);
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0)
+            return NVFP4_ERR_CUDA;
+        slots = n;
+    }
+    const int clusters = d.g.n_tiles < slots ? d.g.n_tiles : slots;
+    cfg.gridDim = dim3(static_cast<unsigned>(clusters * d.split), 1, 1);
+    CUtensorMap tw, tx;
+    if (!make_code_map(&tw, w_codes, args.N, args.K / 2, kBM)) return NVFP4_ERR_CUDA;
+    if (!make_code_map(&tx, a_codes, args.M, args.K / 2, d.nt_tok)) return NVFP4_ERR_CUDA;
+    if (cudaLaunchKernelEx(&cfg, kern, tw, tx, d) != cudaSuccess) return NVFP4_ERR_CUDA;
+    return cuda_status(cudaGetLastError());
+}
+
 nvfp4_status gemm_impl(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_g,
                        const uint8_t* w_codes, const uint8_t* w_sf, const nvfp4_segment* segs,
                        int nseg, void* y, int64_t ldy, int64_t M, int64_t K, void* stream) {
@@ -884,6 +943,7 @@ nvfp4_status gemm_impl(const uint8_t* a_codes, const uint8_t* a_sf, const float*
     // The configuration depends on M only, so a fused GEMM and its per-module
     // GEMMs accumulate every output element identically.
     if (M > 256) return launch_gemm_pair<5>(a_codes, w_codes, args, dev, cs);
+    if (M <= kBM) return launch_gemm_decode(a_codes, w_codes, args, cs);
     return launch_gemm<128, 6, 2>(a_codes, w_codes, args, dev, cs);
 }
 

@@ -1,0 +1,436 @@
+// gemm_decode.cuh -- the W4A4 GEMM for few tokens (M <= 128), where the
+// weights stream from HBM once and nothing else matters.  Included by gemm.cu
+// (shares GemmArgs and the tile constants); same result formula:
+//
+// Y[m, n] = bf16( fl32( acc[m, n] * fl32(gA * gW[seg(n)]) ) ).
+//
+// Layout of the work (sm_100a):
+//   * Operands swapped: 128 weight rows sit on the MMA's M side and the tokens,
+//     padded to NT = 16..128, on its N side, so a tile is 128 outputs wide in n
+//     whatever the token count.
+//   * K is split over a cluster of S CTAs (S = 1, 2, 4 or 8, chosen from K
+//     alone); each CTA accumulates its fixed K slice of a tile in TMEM.
+//   * Persistent: one cluster per scheduling slot; cluster c takes weight
+//     tiles c, c + C, c + 2C, ...  The shared-memory ring runs across tiles, so
+//     weight loads stay in flight while earlier tiles drain.
+//   * Split-K reduction through distributed shared memory: every CTA pushes its
+//     FP32 partial of each row to the CTA owning that row (128/S rows each);
+//     the owner adds the S partials in rank order 0..S-1 (a fixed order: the
+//     result depends on neither N nor the segment table nor timing), applies
+//     alpha and writes BF16.  Handshakes are mbarriers arrived on across the
+//     cluster, so no role waits on a cluster-wide barrier inside the loop.
+//   * The block scales go shared -> registers -> TMEM with tcgen05.st from four
+//     warps (one per TMEM lane quarter) instead of tcgen05.cp, writing the same
+//     replicated layout the copy would: lane l of every quarter holds bytes
+//     [16 l, 16 l + 16) of each 512-byte scale atom in four columns.
+//
+// Roles (14 warps): 0 TMA producer; 1 TMEM owner and MMA issuer; 2..5 scale
+// writers; 6..9 pushers (accumulator -> owners' shared memory); 10..13
+// reducers (rank-order sum, alpha, BF16 store).  Up to four accumulators and
+// four partial buffers keep several tiles in flight between the MMA and the
+// store, so the cluster handshakes overlap the weight stream.
+// TMEM (512 columns, one CTA per SM): the accumulators in columns 0..255,
+// then one 32-column scale slot per ring stage.  Every wait is bounded; on a
+// timeout all roles stop, drain what is in flight and meet at the final
+// cluster barrier.
+
+constexpr int kDecThreads = 448;
+constexpr int kDecSfCol = 256;        // TMEM column of the first scale slot
+constexpr int kDecSfSlot = 32;        // columns per stage: 16 weight + 16 token scales
+constexpr int kDecTmemCols = 512;
+constexpr int kDecMaxSplit = 8;
+constexpr int kDecMaxStages = 8;
+constexpr int kDecMaxAcc = 4;
+constexpr int kDecMaxParts = 4;
+constexpr int kDecHeld = 8;           // reduced outputs a reducer holds before its stores
+constexpr uint32_t kDecStageBudget = 210 * 1024;   // ring + partial buffers
+constexpr uint32_t kDecMinSmem = 116 * 1024;       // > half an SM: one CTA per SM
+
+struct DecodeArgs {
+    GemmArgs g;
+    int nt_tok;      // MMA N: tokens padded to a multiple of 16 (16..128)
+    int split;       // CTAs per cluster along K
+    int stages;      // shared-memory ring depth
+    int nparts;      // partial-sum buffers
+    int nacc;        // TMEM accumulators (256 / nacc columns apart)
+};
+
+struct DecLayout {
+    uint32_t off_w, off_x, off_sfw, off_sfx, off_part, off_bar, off_seg, off_misc, bytes;
+};
+
+__host__ __device__ inline uint32_t dec_stage_bytes(int nt_tok) {
+    return kBM * kBKBytes + nt_tok * kBKBytes + 2 * kAtomsPerStep * kAtom;
+}
+
+__host__ __device__ inline uint32_t dec_part_bytes(int nt_tok) {
+    return static_cast<uint32_t>(nt_tok) * kBM * 4;
+}
+
+__host__ __device__ inline DecLayout dec_layout(int nt_tok, int stages, int nparts) {
+    DecLayout L;
+    L.off_w = 0;
+    L.off_x = L.off_w + stages * kBM * kBKBytes;
+    L.off_sfw = L.off_x + stages * nt_tok * kBKBytes;
+    L.off_sfx = L.off_sfw + stages * kAtomsPerStep * kAtom;
+    L.off_part = L.off_sfx + stages * kAtomsPerStep * kAtom;
+    L.off_bar = L.off_part + nparts * dec_part_bytes(nt_tok);
+    // full, empty, sf_ready per stage; tmem_full, tmem_empty per accumulator;
+    // part_full, part_free per partial buffer; drain
+    L.off_seg = L.off_bar + (3 * stages + 2 * kDecMaxAcc + 2 * nparts + 1) * 8;
+    L.off_misc = L.off_seg + 2 * NVFP4_MAX_SEGMENTS * 4;
+    uint32_t bytes = L.off_misc + 16 + 1024;   // + slack for 1024-byte alignment
+    L.bytes = bytes < kDecMinSmem ? kDecMinSmem : bytes;
+    return L;
+}
+
+// Accumulators, partial buffers and ring depth for a token width.
+__host__ __device__ inline void dec_config(int nt_tok, int* stages, int* nparts, int* nacc) {
+    const int np = nt_tok <= 32 ? 4 : (nt_tok <= 64 ? 2 : 1);
+    int st = static_cast<int>((kDecStageBudget - np * dec_part_bytes(nt_tok)) / dec_stage_bytes(nt_tok));
+    st = st > kDecMaxStages ? kDecMaxStages : st;
+    *stages = st < 2 ? 2 : st;
+    *nparts = np;
+    *nacc = nt_tok <= 64 ? 4 : 2;
+}
+
+__device__ __forceinline__ uint32_t make_idesc_dec(int nt_tok) {
+    return (1u << 7) | (1u << 10) | (static_cast<uint32_t>(nt_tok >> 3) << 17) |
+           (static_cast<uint32_t>(kBM >> 4) << 24);
+}
+
+__global__ void __launch_bounds__(kDecThreads, 1)
+nvf4_gemm_decode_kernel(const __grid_constant__ CUtensorMap tmap_w,
+                        const __grid_constant__ CUtensorMap tmap_x,
+                        const __grid_constant__ DecodeArgs dargs) {
+    const GemmArgs& args = dargs.g;
+    const int NT = dargs.nt_tok;
+    const int S = dargs.split;
+    const int STAGES = dargs.stages;
+    const int NPART = dargs.nparts;
+    const int NACC = dargs.nacc;
+    const int ACC_STRIDE = 256 / NACC;
+    const DecLayout L = dec_layout(NT, STAGES, NPART);
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.off_bar);
+    uint64_t* full = bars;
+    uint64_t* empty = bars + STAGES;
+    uint64_t* sf_ready = bars + 2 * STAGES;
+    uint64_t* tmem_full = bars + 3 * STAGES;          // [kDecMaxAcc]
+    uint64_t* tmem_empty = tmem_full + kDecMaxAcc;    // [kDecMaxAcc]
+    uint64_t* part_full = tmem_empty + kDecMaxAcc;    // [NPART]: partials of my rows landed
+    uint64_t* part_free = part_full + NPART;          // [NPART]: every owner done with a buffer
+    uint64_t* drain = part_free + NPART;
+    float* s_seg_alpha = reinterpret_cast<float*>(smem + L.off_seg);
+    int* s_seg_end = reinterpret_cast<int*>(smem + L.off_seg + NVFP4_MAX_SEGMENTS * 4);
+    uint32_t* s_tmem_base = reinterpret_cast<uint32_t*>(smem + L.off_misc);
+    volatile int* s_abort = reinterpret_cast<volatile int*>(smem + L.off_misc + 4);
+    float* part = reinterpret_cast<float*>(smem + L.off_part);   // [NPART][S][NT][128/S]
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int rank = static_cast<int>(cluster_ctarank());
+    const int cluster_id = blockIdx.x / S;
+    const int num_clusters = gridDim.x / S;
+    const int k_begin = (rank * args.k_steps) / S;
+    const int k_end = ((rank + 1) * args.k_steps) / S;
+    const int nsteps = k_end - k_begin;
+    const int R = kBM / S;                  // rows of a tile owned by each CTA
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < STAGES; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], 1);
+            mbar_init(&sf_ready[i], 4);
+        }
+        for (int i = 0; i < kDecMaxAcc; ++i) {
+            mbar_init(&tmem_full[i], 1);
+            mbar_init(&tmem_empty[i], 4);         // the four pusher warps
+        }
+        for (int i = 0; i < NPART; ++i) {
+            mbar_init(&part_full[i], kBM);        // R rows from each of the S CTAs
+            mbar_init(&part_free[i], 4 * S);      // the 4 reducer warps of each of the S CTAs
+        }
+        mbar_init(drain, 1);
+        *s_abort = 0;
+        fence_mbar_init();
+        prefetch_tmap(&tmap_w);
+        prefetch_tmap(&tmap_x);
+    }
+    if (warp == 1) {
+        tmem_alloc(s_tmem_base, kDecTmemCols);
+        tmem_relinquish();
+    }
+    if (threadIdx.x >= 64 && threadIdx.x < 64 + NVFP4_MAX_SEGMENTS) {
+        const int s = threadIdx.x - 64;
+        s_seg_alpha[s] = (s < args.nseg) ? __fmul_rn(*args.a_g, *args.seg_g[s]) : 0.0f;
+        s_seg_end[s] = (s < args.nseg) ? args.seg_end[s] : 0x7FFFFFFF;
+    }
+    tc_fence_before();
+    __syncthreads();
+    // the peers' barriers are initialised before anyone arrives on them remotely
+    cluster_sync();
+    tc_fence_after();
+    const uint32_t tmem_base = *s_tmem_base;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ---------------- TMA producer ----------------
+            const uint64_t pol_w = l2_policy_evict_first();   // each weight byte is read once
+            const uint64_t pol_x = l2_policy_evict_last();    // tokens are read by every tile
+            uint32_t issued = 0, issued_parity = 0;
+            bool ok = true;
+            int g = 0;
+            for (int nt = cluster_id; nt < args.n_tiles && ok; nt += num_clusters) {
+                for (int s = 0; s < nsteps; ++s, ++g) {
+                    const int stage = g % STAGES;
+                    const uint32_t phase = (g / STAGES) & 1u;
+                    if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, args.timeout_ns, s_abort,
+                                           args.status)) {
+                        ok = false;
+                        break;
+                    }
+                    const int kb = k_begin + s;
+                    const int natoms = min(kAtomsPerStep, args.atoms_per_rb - kb * kAtomsPerStep);
+                    const uint32_t bytes = kBM * kBKBytes + NT * kBKBytes + 2 * natoms * kAtom;
+                    mbar_arrive_expect_tx(&full[stage], bytes);
+                    tma_load_2d(smem + L.off_w + stage * kBM * kBKBytes, &tmap_w, &full[stage],
+                                kb * kBKBytes, nt * kBM, pol_w);
+                    tma_load_2d(smem + L.off_x + stage * NT * kBKBytes, &tmap_x, &full[stage],
+                                kb * kBKBytes, 0, pol_x);
+                    const size_t w_off =
+                        (static_cast<size_t>(nt) * args.atoms_per_rb + kb * kAtomsPerStep) * kAtom;
+                    bulk_load(smem + L.off_sfw + stage * kAtomsPerStep * kAtom, args.w_sf + w_off,
+                              natoms * kAtom, &full[stage], pol_w);
+                    bulk_load(smem + L.off_sfx + stage * kAtomsPerStep * kAtom,
+                              args.a_sf + static_cast<size_t>(kb) * kAtomsPerStep * kAtom,
+                              natoms * kAtom, &full[stage], pol_x);
+                    issued |= 1u << stage;
+                    issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+                }
+            }
+            if (!ok) {
+                // leave no copy in flight: wait (bounded) for every stage issued
+                int local_abort = 0;
+                for (int s = 0; s < STAGES; ++s)
+                    if (issued & (1u << s))
+                        mbar_wait_bounded(&full[s], (issued_parity >> s) & 1u, args.timeout_ns,
+                                          &local_abort, args.status);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ---------------- MMA issuer ----------------
+            const uint32_t idesc = make_idesc_dec(NT);
+            bool ok = true;
+            int g = 0, i = 0;
+            for (int nt = cluster_id; nt < args.n_tiles && ok; nt += num_clusters, ++i) {
+                const int acc = i % NACC;
+                if (!mbar_wait_bounded(&tmem_empty[acc], ((i / NACC) & 1u) ^ 1u, args.timeout_ns,
+                                       s_abort, args.status)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + acc * ACC_STRIDE;
+                for (int s = 0; s < nsteps; ++s, ++g) {
+                    const int stage = g % STAGES;
+                    const uint32_t phase = (g / STAGES) & 1u;
+                    if (!mbar_wait_bounded(&sf_ready[stage], phase, args.timeout_ns, s_abort,
+                                           args.status)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const int kb = k_begin + s;
+                    const int natoms = min(kAtomsPerStep, args.atoms_per_rb - kb * kAtomsPerStep);
+                    const uint32_t sw = smem_u32(smem + L.off_w + stage * kBM * kBKBytes);
+                    const uint32_t sx = smem_u32(smem + L.off_x + stage * NT * kBKBytes);
+                    const uint32_t sf = tmem_base + kDecSfCol + stage * kDecSfSlot;
+                    for (int j = 0; j < natoms; ++j)
+                        tc_mma_nvf4(d_tmem, sdesc_kmajor_sw128(sw + j * 32),
+                                    sdesc_kmajor_sw128(sx + j * 32), idesc, sf + j * 4,
+                                    sf + 16 + j * 4, (s | j) != 0);
+                    tc_commit(&empty[stage]);
+                }
+                if (ok) tc_commit(&tmem_full[acc]);
+            }
+            // every tcgen05 operation issued above has finished before TMEM is freed
+            tc_commit(drain);
+            int local_abort = 0;
+            mbar_wait_bounded(drain, 0, args.timeout_ns, &local_abort, args.status);
+        }
+        __syncwarp();
+    } else if (warp < 6) {
+        // ---------------- scale writers (warps 2..5) ----------------
+        const int q = warp & 3;                   // TMEM lane quarter of this warp
+        const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
+        int g = 0;
+        bool ok = true;
+        for (int nt = cluster_id; nt < args.n_tiles && ok; nt += num_clusters) {
+            for (int s = 0; s < nsteps; ++s, ++g) {
+                const int stage = g % STAGES;
+                const uint32_t phase = (g / STAGES) & 1u;
+                int got = 1;
+                if (lane == 0)
+                    got = mbar_wait_bounded(&full[stage], phase, args.timeout_ns, s_abort,
+                                            args.status);
+                got = __shfl_sync(0xFFFFFFFFu, got, 0);
+                if (!got) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();   // the MMAs that last read this scale slot have completed
+                const int kb = k_begin + s;
+                const int natoms = min(kAtomsPerStep, args.atoms_per_rb - kb * kAtomsPerStep);
+                const uint32_t sfw = smem_u32(smem + L.off_sfw + stage * kAtomsPerStep * kAtom);
+                const uint32_t sfx = smem_u32(smem + L.off_sfx + stage * kAtomsPerStep * kAtom);
+                uint32_t rw[16], rx[16];
+#pragma unroll
+                for (int j = 0; j < kAtomsPerStep; ++j) {
+                    uint4 a = make_uint4(0, 0, 0, 0), b = make_uint4(0, 0, 0, 0);
+                    if (j < natoms) {
+                        a = lds128(sfw + j * kAtom + lane * 16);
+                        b = lds128(sfx + j * kAtom + lane * 16);
+                    }
+                    rw[4 * j] = a.x; rw[4 * j + 1] = a.y; rw[4 * j + 2] = a.z; rw[4 * j + 3] = a.w;
+                    rx[4 * j] = b.x; rx[4 * j + 1] = b.y; rx[4 * j + 2] = b.z; rx[4 * j + 3] = b.w;
+                }
+                const uint32_t sf = tmem_base + lane_base + kDecSfCol + stage * kDecSfSlot;
+                tmem_st_16cols(sf, rw);
+                tmem_st_16cols(sf + 16, rx);
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sf_ready[stage]);
+            }
+        }
+    } else if (warp < 10) {
+        // ---------------- pushers (warps 6..9) ----------------
+        // accumulator row `row` (this thread's TMEM lane) -> slot [rank][t][rr]
+        // of the CTA that owns the row, then one arrival on the owner's part_full
+        const int q = warp & 3;
+        const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
+        const int row = q * 32 + lane;
+        const int owner = row / R;
+        const int rr = row - owner * R;
+        const uint32_t part_owner = mapa_shared(smem_u32(part), static_cast<uint32_t>(owner));
+        const uint32_t full_owner0 = mapa_shared(smem_u32(part_full), static_cast<uint32_t>(owner));
+        int i = 0;
+        for (int nt = cluster_id; nt < args.n_tiles; nt += num_clusters, ++i) {
+            const int acc = i % NACC;
+            const int pb = i % NPART;
+            const int puse = i / NPART;
+            int got = 1;
+            if (lane == 0)
+                got = mbar_wait_bounded(&tmem_full[acc], (i / NACC) & 1u, args.timeout_ns, s_abort,
+                                        args.status);
+            if (puse > 0 && got && lane == 0)
+                got = mbar_wait_cluster_bounded(&part_free[pb], (puse - 1) & 1u, args.timeout_ns,
+                                                s_abort, args.status);
+            got = __shfl_sync(0xFFFFFFFFu, got, 0);
+            if (!got) break;
+            tc_fence_after();
+            const uint32_t dst = part_owner + static_cast<uint32_t>(
+                pb * dec_part_bytes(NT) + ((rank * NT) * R + rr) * 4);
+            for (int c = 0; c < NT; c += 16) {
+                uint32_t r[16];
+                tmem_ld_16cols(tmem_base + lane_base + acc * ACC_STRIDE + c, r);
+                tmem_ld_wait();
+#pragma unroll
+                for (int j = 0; j < 16; ++j)
+                    st_shared_cluster_f32(dst + static_cast<uint32_t>((c + j) * R * 4),
+                                          __uint_as_float(r[j]));
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tmem_empty[acc]);       // the MMA may reuse it
+            mbar_arrive_cluster(full_owner0 + pb * 8);          // my row's partial has landed
+        }
+    } else {
+        // ---------------- reducers (warps 10..13) ----------------
+        // thread -> 4 consecutive owned rows (alpha looked up once per tile) and
+        // every (4 S)-th token; partials read as float4, sums in rank order.
+        // The results stay in registers until this warp has released the
+        // partial buffer, so that release never waits on the global stores.
+        const int red_tid = threadIdx.x - 10 * 32;
+        const int ngroups = R / 4;
+        const int rg = red_tid % ngroups;
+        const int tstep = 128 / ngroups;
+        const int t_first = red_tid / ngroups;
+        int i = 0;
+        for (int nt = cluster_id; nt < args.n_tiles; nt += num_clusters, ++i) {
+            const int pb = i % NPART;
+            const int puse = i / NPART;
+            const int got = mbar_wait_cluster_bounded(&part_full[pb], puse & 1u, args.timeout_ns,
+                                                      s_abort, args.status);
+            if (!__all_sync(0xFFFFFFFFu, got)) break;
+            const float* pbuf = part + pb * (dec_part_bytes(NT) / 4);
+            const int n0 = nt * kBM + rank * R + 4 * rg;
+            float al[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                int sgi = 0;
+                while (sgi < args.nseg - 1 && n0 + u >= s_seg_end[sgi]) ++sgi;
+                al[u] = s_seg_alpha[sgi];
+            }
+            const bool full4 = n0 + 3 < args.N;
+            const int t_end = NT < args.M ? NT : args.M;
+            const int niter = t_first < t_end ? (t_end - t_first + tstep - 1) / tstep : 0;
+            auto reduce_one = [&](int t) -> uint2 {
+                float4 sum = *reinterpret_cast<const float4*>(pbuf + t * R + 4 * rg);
+                for (int qq = 1; qq < S; ++qq) {
+                    const float4 p = *reinterpret_cast<const float4*>(pbuf + (qq * NT + t) * R + 4 * rg);
+                    sum.x = __fadd_rn(sum.x, p.x);
+                    sum.y = __fadd_rn(sum.y, p.y);
+                    sum.z = __fadd_rn(sum.z, p.z);
+                    sum.w = __fadd_rn(sum.w, p.w);
+                }
+                return make_uint2(pack_bf16x2(__fmul_rn(sum.x, al[0]), __fmul_rn(sum.y, al[1])),
+                                  pack_bf16x2(__fmul_rn(sum.z, al[2]), __fmul_rn(sum.w, al[3])));
+            };
+            auto store_one = [&](int t, uint2 o) {
+                uint16_t* yp = args.y + static_cast<int64_t>(t) * args.ldy + n0;
+                if (full4) {
+                    *reinterpret_cast<uint2*>(yp) = o;
+                } else {
+                    const uint16_t v[4] = {static_cast<uint16_t>(o.x & 0xFFFFu), static_cast<uint16_t>(o.x >> 16),
+                                           static_cast<uint16_t>(o.y & 0xFFFFu), static_cast<uint16_t>(o.y >> 16)};
+#pragma unroll
+                    for (int u = 0; u < 4; ++u)
+                        if (n0 + u < args.N) yp[u] = v[u];
+                }
+            };
+            uint2 held[kDecHeld];
+#pragma unroll
+            for (int h = 0; h < kDecHeld; ++h)
+                if (h < niter) held[h] = reduce_one(t_first + h * tstep);
+            // more outputs than registers hold (one-CTA clusters with wide token
+            // counts): those are stored before the release
+            for (int h = kDecHeld; h < niter; ++h) store_one(t_first + h * tstep, reduce_one(t_first + h * tstep));
+            __syncwarp();
+            // this warp is done reading buffer pb: tell every CTA of the cluster.
+            // Relaxed: every partial read above was consumed before this point
+            // (in-order issue), and a release would wait for the global stores
+            // of the previous tile.
+            if (lane < S)
+                mbar_arrive_cluster_relaxed(
+                    mapa_shared(smem_u32(&part_free[pb]), static_cast<uint32_t>(lane)));
+#pragma unroll
+            for (int h = 0; h < kDecHeld; ++h)
+                if (h < niter) store_one(t_first + h * tstep, held[h]);
+        }
+    }
+
+    // no CTA leaves while a peer may still write into its shared memory or
+    // arrive on its barriers
+    tc_fence_before();
+    __syncwarp();
+    cluster_sync();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem_base, kDecTmemCols);
+}

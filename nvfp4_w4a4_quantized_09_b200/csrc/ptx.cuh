@@ -43,31 +43,83 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
+// Suspend-time hint for try_wait, in ns: a waiting thread sleeps in hardware
+// until the phase completes (it is woken then) or this much time has passed,
+// instead of spinning and loading the shared-memory pipe the working warps need.
+constexpr uint32_t kWaitHintNs = 20000;
+
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     uint32_t done;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(done)
-        : "r"(smem_u32(bar)), "r"(parity)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(kWaitHintNs)
         : "memory");
     return done != 0;
 }
 
+// SM cycle counter: cheap to read (unlike %globaltimer, whose reads are slow
+// and which advances in coarse steps), so polling loops can consult it on
+// every iteration without adding latency to the handshake they wait for.
+__device__ __forceinline__ uint64_t clock_cycles() {
+    uint64_t c;
+    asm volatile("mov.u64 %0, %%clock64;" : "=l"(c));
+    return c;
+}
+
+// A wait limit given in nanoseconds as SM cycles: 2 cycles per ns, so the
+// bound is the requested time at 2 GHz and proportionally longer at lower
+// clocks -- always finite.
+__device__ __forceinline__ uint64_t limit_cycles(uint64_t limit_ns) { return limit_ns * 2; }
+
 // Wait until the phase with the given parity has completed, or give up after
-// `limit_ns` of wall time or when *abort becomes non-zero.  On a timeout the
-// device status word is set and *abort raised so that every role of the CTA
-// stops.  Returns true when the phase completed.
+// `limit_ns` (see limit_cycles) or when *abort becomes non-zero.  On a
+// timeout the device status word is set and *abort raised so that every role
+// of the CTA stops.  Returns true when the phase completed.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
                                                   uint64_t limit_ns, volatile int* abort,
                                                   int* dev_status) {
     if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = globaltimer_ns();
+    const uint64_t t0 = clock_cycles();
+    const uint64_t lim = limit_cycles(limit_ns);
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
         if (*abort) return false;
-        if (globaltimer_ns() - t0 > limit_ns) {
+        if (clock_cycles() - t0 > lim) {
+            *abort = 1;
+            atomicExch(dev_status, kDevTimeout);
+            return false;
+        }
+    }
+}
+
+// Wait variant for barriers that other CTAs of the cluster arrive on (with
+// release.cluster) after writing into this CTA's shared memory: the acquire
+// is at cluster scope so those writes are visible once the phase completes.
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(kWaitHintNs)
+        : "memory");
+    return done != 0;
+}
+
+__device__ __forceinline__ bool mbar_wait_cluster_bounded(uint64_t* bar, uint32_t parity,
+                                                          uint64_t limit_ns, volatile int* abort,
+                                                          int* dev_status) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    const uint64_t t0 = clock_cycles();
+    const uint64_t lim = limit_cycles(limit_ns);
+    while (true) {
+        if (mbar_try_wait_cluster(bar, parity)) return true;
+        if (*abort) return false;
+        if (clock_cycles() - t0 > lim) {
             *abort = 1;
             atomicExch(dev_status, kDevTimeout);
             return false;
@@ -258,6 +310,15 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_saddr) {
                  : "memory");
 }
 
+// Arrive with relaxed ordering: for signals that only say "I have finished
+// reading" where every value read was already consumed by this thread before
+// the arrive issues.  Unlike the release form it does not wait for this
+// thread's earlier global stores to complete.
+__device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t cluster_saddr) {
+    asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_saddr)
+                 : "memory");
+}
+
 __device__ __forceinline__ void cluster_sync() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
                      : "memory");
@@ -344,6 +405,24 @@ __device__ __forceinline__ uint4 lds128(uint32_t saddr) {
                  : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                  : "r"(saddr));
     return v;
+}
+
+// 32-bit store into the shared memory of a CTA of the cluster (a
+// shared::cluster address from mapa_shared).
+__device__ __forceinline__ void st_shared_cluster_f32(uint32_t cluster_saddr, float v) {
+    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(cluster_saddr), "f"(v) : "memory");
+}
+
+// Each thread of the warp reads 16 consecutive 32-bit columns of its own TMEM
+// lane (the warp's 32-lane quarter).
+__device__ __forceinline__ void tmem_ld_16cols(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
 }
 
 }  // namespace nvfp4

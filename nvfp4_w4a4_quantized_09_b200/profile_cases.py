@@ -6,6 +6,7 @@ CASE:
   gemm_gdn        fused GEMM, X [8192,5120] x W q/k/v/z/b/a [24704,5120]
   gemm_gateup     GEMM, X [8192,5120] x W [34816,5120]
   gemm_decode     fused GEMM, X [32,5120] x W [24640,5120]
+  gemm_decode_m1  fused GEMM, X [1,5120] x W [24640,5120]
   quantize_act    quantizer on the activation [32768,5120]
   global_scale_act  global scale of the activation [32768,5120]
 
@@ -25,8 +26,8 @@ from nvfp4_w4a4_quantized_09_b200 import synth
 def main(case: str, launches: int = 3) -> None:
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
-    if case in ("gemm_gdn", "gemm_decode"):
-        M = 8192 if case == "gemm_gdn" else 32
+    if case in ("gemm_gdn", "gemm_decode", "gemm_decode_m1"):
+        M = {"gemm_gdn": 8192, "gemm_decode": 32, "gemm_decode_m1": 1}[case]
         mods = synth.GDN_MODULES if case == "gemm_gdn" else synth.GDN_MODULES_DECODE
         x = synth.student_t_activations(M, 5120, seed=3, device=dev)
         fw = nv.FusedWeight.from_modules([w for _, w in synth.gdn_weights(mods, device=dev)])
