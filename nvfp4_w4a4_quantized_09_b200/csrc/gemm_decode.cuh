@@ -42,7 +42,7 @@ constexpr int kDecMaxSplit = 8;
 constexpr int kDecMaxStages = 8;
 constexpr int kDecMaxAcc = 4;
 constexpr int kDecMaxParts = 4;
-constexpr int kDecHeld = 8;           // reduced outputs a reducer holds before its stores
+constexpr int kDecHeld = 4;           // reduced outputs a reducer holds before its stores
 constexpr uint32_t kDecStageBudget = 210 * 1024;   // ring + partial buffers
 constexpr uint32_t kDecMinSmem = 116 * 1024;       // > half an SM: one CTA per SM
 
@@ -137,7 +137,6 @@ nvf4_gemm_decode_kernel(const __grid_constant__ CUtensorMap tmap_w,
     const int num_clusters = gridDim.x / S;
     const int k_begin = (rank * args.k_steps) / S;
     const int k_end = ((rank + 1) * args.k_steps) / S;
-    const int nsteps = k_end - k_begin;
     const int R = kBM / S;                  // rows of a tile owned by each CTA
 
     if (threadIdx.x == 0) {
@@ -176,90 +175,124 @@ nvf4_gemm_decode_kernel(const __grid_constant__ CUtensorMap tmap_w,
     tc_fence_after();
     const uint32_t tmem_base = *s_tmem_base;
 
+    // Loop-invariant step data.  Every role walks the same (tile, k-step)
+    // sequence with incremental ring counters -- no division in the loops;
+    // only the last k-step of K can carry fewer than four scale atoms.
+    const int last_kb = args.k_steps - 1;
+    const int last_natoms = args.atoms_per_rb - last_kb * kAtomsPerStep;
+    const uint32_t s_w0 = smem_u32(smem + L.off_w);
+    const uint32_t s_x0 = smem_u32(smem + L.off_x);
+    const uint32_t s_sfw0 = smem_u32(smem + L.off_sfw);
+    const uint32_t s_sfx0 = smem_u32(smem + L.off_sfx);
+    const uint32_t x_stride = static_cast<uint32_t>(NT) * kBKBytes;
+
     if (warp == 0) {
-        if (lane == 0) {
-            // ---------------- TMA producer ----------------
-            const uint64_t pol_w = l2_policy_evict_first();   // each weight byte is read once
-            const uint64_t pol_x = l2_policy_evict_last();    // tokens are read by every tile
-            uint32_t issued = 0, issued_parity = 0;
-            bool ok = true;
-            int g = 0;
-            for (int nt = cluster_id; nt < args.n_tiles && ok; nt += num_clusters) {
-                for (int s = 0; s < nsteps; ++s, ++g) {
-                    const int stage = g % STAGES;
-                    const uint32_t phase = (g / STAGES) & 1u;
-                    if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, args.timeout_ns, s_abort,
-                                           args.status)) {
-                        ok = false;
-                        break;
-                    }
-                    const int kb = k_begin + s;
-                    const int natoms = min(kAtomsPerStep, args.atoms_per_rb - kb * kAtomsPerStep);
-                    const uint32_t bytes = kBM * kBKBytes + NT * kBKBytes + 2 * natoms * kAtom;
-                    mbar_arrive_expect_tx(&full[stage], bytes);
-                    tma_load_2d(smem + L.off_w + stage * kBM * kBKBytes, &tmap_w, &full[stage],
+        // ---------------- TMA producer (whole warp; one elected lane issues) ----------------
+        const uint64_t pol_w = l2_policy_evict_first();   // each weight byte is read once
+        const uint64_t pol_x = l2_policy_evict_last();    // tokens are read by every tile
+        const uint32_t full_bytes = kBM * kBKBytes + NT * kBKBytes + 2 * kAtomsPerStep * kAtom;
+        const uint32_t last_bytes = kBM * kBKBytes + NT * kBKBytes + 2 * last_natoms * kAtom;
+        uint32_t issued = 0, issued_parity = 0;
+        bool ok = true;
+        int stage = 0;
+        uint32_t phase = 0;
+        for (int nt = cluster_id; nt < args.n_tiles && ok; nt += num_clusters) {
+            const uint8_t* wsf = args.w_sf + (static_cast<size_t>(nt) * args.atoms_per_rb +
+                                              static_cast<size_t>(k_begin) * kAtomsPerStep) * kAtom;
+            const uint8_t* xsf = args.a_sf + static_cast<size_t>(k_begin) * kAtomsPerStep * kAtom;
+            for (int kb = k_begin; kb < k_end; ++kb) {
+                if (!mbar_wait_warp(&empty[stage], phase ^ 1u, args.timeout_ns, s_abort, args.status)) {
+                    ok = false;
+                    break;
+                }
+                const bool last = kb == last_kb;
+                const uint32_t sf_bytes = (last ? last_natoms : kAtomsPerStep) * kAtom;
+                uint64_t* fb = &full[stage];
+                if (elect_one()) {
+                    mbar_arrive_expect_tx(fb, last ? last_bytes : full_bytes);
+                    tma_load_2d(smem + L.off_w + stage * (kBM * kBKBytes), &tmap_w, fb,
                                 kb * kBKBytes, nt * kBM, pol_w);
-                    tma_load_2d(smem + L.off_x + stage * NT * kBKBytes, &tmap_x, &full[stage],
-                                kb * kBKBytes, 0, pol_x);
-                    const size_t w_off =
-                        (static_cast<size_t>(nt) * args.atoms_per_rb + kb * kAtomsPerStep) * kAtom;
-                    bulk_load(smem + L.off_sfw + stage * kAtomsPerStep * kAtom, args.w_sf + w_off,
-                              natoms * kAtom, &full[stage], pol_w);
-                    bulk_load(smem + L.off_sfx + stage * kAtomsPerStep * kAtom,
-                              args.a_sf + static_cast<size_t>(kb) * kAtomsPerStep * kAtom,
-                              natoms * kAtom, &full[stage], pol_x);
-                    issued |= 1u << stage;
-                    issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+                    tma_load_2d(smem + L.off_x + stage * x_stride, &tmap_x, fb, kb * kBKBytes, 0, pol_x);
+                    bulk_load(smem + L.off_sfw + stage * (kAtomsPerStep * kAtom), wsf, sf_bytes, fb, pol_w);
+                    bulk_load(smem + L.off_sfx + stage * (kAtomsPerStep * kAtom), xsf, sf_bytes, fb, pol_x);
+                }
+                __syncwarp();
+                wsf += kAtomsPerStep * kAtom;
+                xsf += kAtomsPerStep * kAtom;
+                issued |= 1u << stage;
+                issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
                 }
             }
-            if (!ok) {
-                // leave no copy in flight: wait (bounded) for every stage issued
-                int local_abort = 0;
-                for (int s = 0; s < STAGES; ++s)
-                    if (issued & (1u << s))
-                        mbar_wait_bounded(&full[s], (issued_parity >> s) & 1u, args.timeout_ns,
-                                          &local_abort, args.status);
-            }
+        }
+        if (!ok && lane == 0) {
+            // leave no copy in flight: wait (bounded) for every stage issued
+            int local_abort = 0;
+            for (int st = 0; st < STAGES; ++st)
+                if (issued & (1u << st))
+                    mbar_wait_bounded(&full[st], (issued_parity >> st) & 1u, args.timeout_ns,
+                                      &local_abort, args.status);
         }
         __syncwarp();
     } else if (warp == 1) {
-        if (lane == 0) {
-            // ---------------- MMA issuer ----------------
-            const uint32_t idesc = make_idesc_dec(NT);
-            bool ok = true;
-            int g = 0, i = 0;
-            for (int nt = cluster_id; nt < args.n_tiles && ok; nt += num_clusters, ++i) {
-                const int acc = i % NACC;
-                if (!mbar_wait_bounded(&tmem_empty[acc], ((i / NACC) & 1u) ^ 1u, args.timeout_ns,
-                                       s_abort, args.status)) {
+        // ---------------- MMA issuer (whole warp; one elected lane issues) ----------------
+        const uint32_t idesc = make_idesc_dec(NT);
+        // descriptor start-address fields advance by 2 per 32 bytes of K
+        const uint64_t dw0 = sdesc_kmajor_sw128(s_w0);
+        const uint64_t dx0 = sdesc_kmajor_sw128(s_x0);
+        const uint32_t sf0 = tmem_base + kDecSfCol;
+        bool ok = true;
+        int stage = 0, acc = 0;
+        uint32_t phase = 0, acc_phase = 0;
+        for (int nt = cluster_id; nt < args.n_tiles && ok; nt += num_clusters) {
+            if (!mbar_wait_warp(&tmem_empty[acc], acc_phase ^ 1u, args.timeout_ns, s_abort,
+                                args.status)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t d_tmem = tmem_base + acc * ACC_STRIDE;
+            for (int kb = k_begin; kb < k_end; ++kb) {
+                if (!mbar_wait_warp(&sf_ready[stage], phase, args.timeout_ns, s_abort, args.status)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const uint32_t d_tmem = tmem_base + acc * ACC_STRIDE;
-                for (int s = 0; s < nsteps; ++s, ++g) {
-                    const int stage = g % STAGES;
-                    const uint32_t phase = (g / STAGES) & 1u;
-                    if (!mbar_wait_bounded(&sf_ready[stage], phase, args.timeout_ns, s_abort,
-                                           args.status)) {
-                        ok = false;
-                        break;
+                const uint64_t dw = dw0 + static_cast<uint64_t>(stage * (kBM * kBKBytes / 16));
+                const uint64_t dx = dx0 + static_cast<uint64_t>(stage * (x_stride / 16));
+                const uint32_t sf = sf0 + stage * kDecSfSlot;
+                const uint32_t first = kb != k_begin;
+                const int natoms = kb == last_kb ? last_natoms : kAtomsPerStep;
+                if (elect_one()) {
+                    if (natoms == kAtomsPerStep) {
+#pragma unroll
+                        for (int j = 0; j < kAtomsPerStep; ++j)
+                            tc_mma_nvf4(d_tmem, dw + 2 * j, dx + 2 * j, idesc, sf + j * 4,
+                                        sf + 16 + j * 4, first | static_cast<uint32_t>(j));
+                    } else {
+                        for (int j = 0; j < natoms; ++j)
+                            tc_mma_nvf4(d_tmem, dw + 2 * j, dx + 2 * j, idesc, sf + j * 4,
+                                        sf + 16 + j * 4, first | static_cast<uint32_t>(j));
                     }
-                    tc_fence_after();
-                    const int kb = k_begin + s;
-                    const int natoms = min(kAtomsPerStep, args.atoms_per_rb - kb * kAtomsPerStep);
-                    const uint32_t sw = smem_u32(smem + L.off_w + stage * kBM * kBKBytes);
-                    const uint32_t sx = smem_u32(smem + L.off_x + stage * NT * kBKBytes);
-                    const uint32_t sf = tmem_base + kDecSfCol + stage * kDecSfSlot;
-                    for (int j = 0; j < natoms; ++j)
-                        tc_mma_nvf4(d_tmem, sdesc_kmajor_sw128(sw + j * 32),
-                                    sdesc_kmajor_sw128(sx + j * 32), idesc, sf + j * 4,
-                                    sf + 16 + j * 4, (s | j) != 0);
                     tc_commit(&empty[stage]);
                 }
-                if (ok) tc_commit(&tmem_full[acc]);
+                __syncwarp();
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
             }
-            // every tcgen05 operation issued above has finished before TMEM is freed
+            if (ok && elect_one()) tc_commit(&tmem_full[acc]);
+            __syncwarp();
+            if (++acc == NACC) {
+                acc = 0;
+                acc_phase ^= 1u;
+            }
+        }
+        // every tcgen05 operation issued above has finished before TMEM is freed
+        if (elect_one()) {
             tc_commit(drain);
             int local_abort = 0;
             mbar_wait_bounded(drain, 0, args.timeout_ns, &local_abort, args.status);
@@ -268,13 +301,13 @@ nvf4_gemm_decode_kernel(const __grid_constant__ CUtensorMap tmap_w,
     } else if (warp < 6) {
         // ---------------- scale writers (warps 2..5) ----------------
         const int q = warp & 3;                   // TMEM lane quarter of this warp
-        const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
-        int g = 0;
+        const uint32_t sf0 = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + kDecSfCol;
+        const uint32_t lane_off = lane * 16;
+        int stage = 0;
+        uint32_t phase = 0;
         bool ok = true;
         for (int nt = cluster_id; nt < args.n_tiles && ok; nt += num_clusters) {
-            for (int s = 0; s < nsteps; ++s, ++g) {
-                const int stage = g % STAGES;
-                const uint32_t phase = (g / STAGES) & 1u;
+            for (int kb = k_begin; kb < k_end; ++kb) {
                 int got = 1;
                 if (lane == 0)
                     got = mbar_wait_bounded(&full[stage], phase, args.timeout_ns, s_abort,
@@ -285,28 +318,31 @@ nvf4_gemm_decode_kernel(const __grid_constant__ CUtensorMap tmap_w,
                     break;
                 }
                 tc_fence_after();   // the MMAs that last read this scale slot have completed
-                const int kb = k_begin + s;
-                const int natoms = min(kAtomsPerStep, args.atoms_per_rb - kb * kAtomsPerStep);
-                const uint32_t sfw = smem_u32(smem + L.off_sfw + stage * kAtomsPerStep * kAtom);
-                const uint32_t sfx = smem_u32(smem + L.off_sfx + stage * kAtomsPerStep * kAtom);
+                const int natoms = kb == last_kb ? last_natoms : kAtomsPerStep;
+                const uint32_t sfw = s_sfw0 + stage * (kAtomsPerStep * kAtom) + lane_off;
+                const uint32_t sfx = s_sfx0 + stage * (kAtomsPerStep * kAtom) + lane_off;
                 uint32_t rw[16], rx[16];
 #pragma unroll
                 for (int j = 0; j < kAtomsPerStep; ++j) {
                     uint4 a = make_uint4(0, 0, 0, 0), b = make_uint4(0, 0, 0, 0);
                     if (j < natoms) {
-                        a = lds128(sfw + j * kAtom + lane * 16);
-                        b = lds128(sfx + j * kAtom + lane * 16);
+                        a = lds128(sfw + j * kAtom);
+                        b = lds128(sfx + j * kAtom);
                     }
                     rw[4 * j] = a.x; rw[4 * j + 1] = a.y; rw[4 * j + 2] = a.z; rw[4 * j + 3] = a.w;
                     rx[4 * j] = b.x; rx[4 * j + 1] = b.y; rx[4 * j + 2] = b.z; rx[4 * j + 3] = b.w;
                 }
-                const uint32_t sf = tmem_base + lane_base + kDecSfCol + stage * kDecSfSlot;
+                const uint32_t sf = sf0 + stage * kDecSfSlot;
                 tmem_st_16cols(sf, rw);
                 tmem_st_16cols(sf + 16, rx);
                 tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sf_ready[stage]);
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
             }
         }
     } else if (warp < 10) {
@@ -381,14 +417,23 @@ nvf4_gemm_decode_kernel(const __grid_constant__ CUtensorMap tmap_w,
             const bool full4 = n0 + 3 < args.N;
             const int t_end = NT < args.M ? NT : args.M;
             const int niter = t_first < t_end ? (t_end - t_first + tstep - 1) / tstep : 0;
+            const int slot_stride = NT * R;          // floats between the partials of two ranks
             auto reduce_one = [&](int t) -> uint2 {
-                float4 sum = *reinterpret_cast<const float4*>(pbuf + t * R + 4 * rg);
-                for (int qq = 1; qq < S; ++qq) {
-                    const float4 p = *reinterpret_cast<const float4*>(pbuf + (qq * NT + t) * R + 4 * rg);
-                    sum.x = __fadd_rn(sum.x, p.x);
-                    sum.y = __fadd_rn(sum.y, p.y);
-                    sum.z = __fadd_rn(sum.z, p.z);
-                    sum.w = __fadd_rn(sum.w, p.w);
+                // all S partials are loaded before the rank-ordered adds
+                const float* p0 = pbuf + t * R + 4 * rg;
+                float4 p[kDecMaxSplit];
+#pragma unroll
+                for (int qq = 0; qq < kDecMaxSplit; ++qq)
+                    if (qq < S) p[qq] = *reinterpret_cast<const float4*>(p0 + qq * slot_stride);
+                float4 sum = p[0];
+#pragma unroll
+                for (int qq = 1; qq < kDecMaxSplit; ++qq) {
+                    if (qq < S) {
+                        sum.x = __fadd_rn(sum.x, p[qq].x);
+                        sum.y = __fadd_rn(sum.y, p[qq].y);
+                        sum.z = __fadd_rn(sum.z, p[qq].z);
+                        sum.w = __fadd_rn(sum.w, p[qq].w);
+                    }
                 }
                 return make_uint2(pack_bf16x2(__fmul_rn(sum.x, al[0]), __fmul_rn(sum.y, al[1])),
                                   pack_bf16x2(__fmul_rn(sum.z, al[2]), __fmul_rn(sum.w, al[3])));

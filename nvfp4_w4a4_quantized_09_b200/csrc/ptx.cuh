@@ -127,6 +127,28 @@ __device__ __forceinline__ bool mbar_wait_cluster_bounded(uint64_t* bar, uint32_
     }
 }
 
+// True in exactly one active lane of the warp.  Issue code of the form
+// "the whole warp computes, one elected lane issues" keeps descriptors and
+// addresses warp-uniform, so tensor-core and TMA instructions take them from
+// uniform registers without per-instruction moves.
+__device__ __forceinline__ bool elect_one() {
+    uint32_t pred = 0;
+    asm volatile(
+        "{\n\t.reg .pred P;\n\t"
+        "elect.sync _|P, 0xffffffff;\n\t"
+        "selp.u32 %0, 1, 0, P;\n\t}"
+        : "=r"(pred));
+    return pred != 0;
+}
+
+// Bounded wait by the whole warp: lane 0 polls, the verdict is broadcast.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, uint64_t limit_ns,
+                                               volatile int* abort, int* dev_status) {
+    int ok = 1;
+    if ((threadIdx.x & 31) == 0) ok = mbar_wait_bounded(bar, parity, limit_ns, abort, dev_status);
+    return __shfl_sync(0xFFFFFFFFu, ok, 0) != 0;
+}
+
 // ----------------------------------------------------------------------------
 // TMA and bulk copies (global -> shared), completion counted in bytes on an
 // mbarrier.  No multicast anywhere: each CTA loads its own tiles.
