@@ -480,29 +480,30 @@ nvf4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a,
     const uint32_t full0_leader = mapa_shared(smem_u32(&full[0]), 0);
     const uint32_t tmem_empty_leader = mapa_shared(smem_u32(tmem_empty), 0);
 
+    // The issuing roles run as whole warps with one elected lane issuing, so
+    // ring counters, descriptors and addresses stay warp-uniform; only the
+    // last k-step of K can carry fewer than four scale atoms.
+    const int last_kb = args.k_steps - 1;
+    const int last_natoms = args.atoms_per_rb - last_kb * kAtomsPerStep;
+
     if (warp == 0) {
-        if (lane == 0) {
-            // ---------------- TMA producer (both CTAs) ----------------
-            const uint64_t pol = l2_policy_evict_last();
-            int stage = 0;
-            uint32_t phase = 0;
-            uint32_t armed = 0, armed_parity = 0;   // stages the even CTA expects bytes on
-            bool ok = true;
-            for (int t = pair; t < total_tiles && ok; t += npairs) {
-                int mt, nt;
-                tile_coords(t, args, mt, nt);
-                for (int kb = 0; kb < args.k_steps; ++kb) {
-                    if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, args.timeout_ns, s_abort,
-                                           args.status)) {
-                        ok = false;
-                        break;
-                    }
-                    const uint32_t fb = full0_leader + stage * 8;
-                    if (rank == 0) {
-                        mbar_arrive_expect_tx(&full[stage], 2 * C::STAGE_TX);
-                        armed |= 1u << stage;
-                        armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
-                    }
+        // ---------------- TMA producer (both CTAs) ----------------
+        const uint64_t pol = l2_policy_evict_last();
+        int stage = 0;
+        uint32_t phase = 0;
+        uint32_t armed = 0, armed_parity = 0;   // stages the even CTA expects bytes on
+        bool ok = true;
+        for (int t = pair; t < total_tiles && ok; t += npairs) {
+            int mt, nt;
+            tile_coords(t, args, mt, nt);
+            for (int kb = 0; kb < args.k_steps; ++kb) {
+                if (!mbar_wait_warp(&empty[stage], phase ^ 1u, args.timeout_ns, s_abort, args.status)) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t fb = full0_leader + stage * 8;
+                if (elect_one()) {
+                    if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * C::STAGE_TX);
                     tma_load_2d_pair(smem + C::OFF_A + stage * C::A_BYTES, &tmap_a, fb,
                                      kb * kBKBytes, mt * 256 + rank * 128, pol);
                     tma_load_2d_pair(smem + C::OFF_B + stage * C::B_BYTES, &tmap_b, fb,
@@ -511,97 +512,124 @@ nvf4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a,
                                      kb * 256, mt * 2 + rank, pol);
                     tma_load_2d_pair(smem + C::OFF_SFB + stage * C::SFB_BYTES, &tmap_sfb, fb,
                                      kb * 256, nt * 2, pol);
-                    if (++stage == STAGES) {
-                        stage = 0;
-                        phase ^= 1u;
-                    }
+                }
+                __syncwarp();
+                if (rank == 0) {
+                    armed |= 1u << stage;
+                    armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+                }
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
                 }
             }
-            if (!ok && rank == 0) {
-                // leave no copy of either CTA in flight on the stages armed here
-                int local_abort = 0;
-                for (int s = 0; s < STAGES; ++s)
-                    if (armed & (1u << s))
-                        mbar_wait_bounded(&full[s], (armed_parity >> s) & 1u, args.timeout_ns,
-                                          &local_abort, args.status);
-            }
         }
+        if (!ok && rank == 0 && lane == 0) {
+            // leave no copy of either CTA in flight on the stages armed here
+            int local_abort = 0;
+            for (int s = 0; s < STAGES; ++s)
+                if (armed & (1u << s))
+                    mbar_wait_bounded(&full[s], (armed_parity >> s) & 1u, args.timeout_ns,
+                                      &local_abort, args.status);
+        }
+        __syncwarp();
     } else if (warp == 1) {
-        if (lane == 0 && rank == 0) {
+        if (rank == 0) {
             // ---------------- MMA issuer (even CTA) ----------------
             constexpr uint32_t idesc = make_idesc_pair();
+            // descriptor start-address fields advance by 2 per 32 bytes of K
+            const uint64_t da0 = sdesc_kmajor_sw128(smem_u32(smem + C::OFF_A));
+            const uint64_t db0 = sdesc_kmajor_sw128(smem_u32(smem + C::OFF_B));
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
             int i = 0;
             for (int t = pair; t < total_tiles && ok; t += npairs, ++i) {
-                if (!mbar_wait_bounded(tmem_empty, (i & 1) ^ 1u, args.timeout_ns, s_abort,
-                                       args.status)) {
+                if (!mbar_wait_warp(tmem_empty, (i & 1) ^ 1u, args.timeout_ns, s_abort, args.status)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
                 for (int kb = 0; kb < args.k_steps; ++kb) {
-                    if (!mbar_wait_bounded(&sf_ready[stage], phase, args.timeout_ns, s_abort,
-                                           args.status)) {
+                    if (!mbar_wait_warp(&sf_ready[stage], phase, args.timeout_ns, s_abort, args.status)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const int natoms = min(kAtomsPerStep, args.atoms_per_rb - kb * kAtomsPerStep);
-                    const uint32_t sa = smem_u32(smem + C::OFF_A + stage * C::A_BYTES);
-                    const uint32_t sb = smem_u32(smem + C::OFF_B + stage * C::B_BYTES);
+                    const uint64_t da = da0 + static_cast<uint64_t>(stage * (C::A_BYTES / 16));
+                    const uint64_t db = db0 + static_cast<uint64_t>(stage * (C::B_BYTES / 16));
                     const uint32_t sfr = tmem_base + C::BN + stage * C::SF_STRIDE;
-                    for (int j = 0; j < natoms; ++j)
-                        tc_mma_nvf4_pair(tmem_base, sdesc_kmajor_sw128(sa + j * 32),
-                                         sdesc_kmajor_sw128(sb + j * 32), idesc,
-                                         sfr + j * 4, sfr + 16 + j * 8, (kb | j) != 0);
-                    tc_commit_pair(&empty[stage], 0x3);
+                    const uint32_t first = kb != 0;
+                    if (elect_one()) {
+                        if (kb != last_kb) {
+#pragma unroll
+                            for (int j = 0; j < kAtomsPerStep; ++j)
+                                tc_mma_nvf4_pair(tmem_base, da + 2 * j, db + 2 * j, idesc, sfr + j * 4,
+                                                 sfr + 16 + j * 8, first | static_cast<uint32_t>(j));
+                        } else {
+                            for (int j = 0; j < last_natoms; ++j)
+                                tc_mma_nvf4_pair(tmem_base, da + 2 * j, db + 2 * j, idesc, sfr + j * 4,
+                                                 sfr + 16 + j * 8, first | static_cast<uint32_t>(j));
+                        }
+                        tc_commit_pair(&empty[stage], 0x3);
+                    }
+                    __syncwarp();
                     if (++stage == STAGES) {
                         stage = 0;
                         phase ^= 1u;
                     }
                 }
-                if (ok) tc_commit_pair(tmem_full, 0x3);
+                if (ok && elect_one()) tc_commit_pair(tmem_full, 0x3);
+                __syncwarp();
             }
-            tc_commit_pair(drain, 0x1);
-            int local_abort = 0;
-            mbar_wait_bounded(drain, 0, args.timeout_ns, &local_abort, args.status);
+            if (elect_one()) {
+                tc_commit_pair(drain, 0x1);
+                int local_abort = 0;
+                mbar_wait_bounded(drain, 0, args.timeout_ns, &local_abort, args.status);
+            }
+            __syncwarp();
         }
     } else if (warp == 2 + kEpiWarps) {
-        if (lane == 0 && rank == 0) {
+        if (rank == 0) {
             // ---------------- scale copies (even CTA) ----------------
+            const uint32_t ssfa0 = smem_u32(smem + C::OFF_SFA);
+            const uint32_t ssfb0 = smem_u32(smem + C::OFF_SFB);
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
             for (int t = pair; t < total_tiles && ok; t += npairs) {
                 for (int kb = 0; kb < args.k_steps; ++kb) {
-                    if (!mbar_wait_bounded(&full[stage], phase, args.timeout_ns, s_abort,
-                                           args.status)) {
+                    if (!mbar_wait_warp(&full[stage], phase, args.timeout_ns, s_abort, args.status)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const int natoms = min(kAtomsPerStep, args.atoms_per_rb - kb * kAtomsPerStep);
-                    const uint32_t ssfa = smem_u32(smem + C::OFF_SFA + stage * C::SFA_BYTES);
-                    const uint32_t ssfb = smem_u32(smem + C::OFF_SFB + stage * C::SFB_BYTES);
+                    const int natoms = kb == last_kb ? last_natoms : kAtomsPerStep;
+                    const uint32_t ssfa = ssfa0 + stage * C::SFA_BYTES;
+                    const uint32_t ssfb = ssfb0 + stage * C::SFB_BYTES;
                     const uint32_t sfr = tmem_base + C::BN + stage * C::SF_STRIDE;
-                    for (int j = 0; j < natoms; ++j) {
-                        tc_copy_scales_pair(sfr + j * 4, sdesc_scales(ssfa + j * kAtom));
-                        tc_copy_scales_pair(sfr + 16 + j * 8, sdesc_scales(ssfb + j * kAtom));
-                        tc_copy_scales_pair(sfr + 16 + j * 8 + 4,
-                                            sdesc_scales(ssfb + kAtomsPerStep * kAtom + j * kAtom));
+                    if (elect_one()) {
+                        for (int j = 0; j < natoms; ++j) {
+                            tc_copy_scales_pair(sfr + j * 4, sdesc_scales(ssfa + j * kAtom));
+                            tc_copy_scales_pair(sfr + 16 + j * 8, sdesc_scales(ssfb + j * kAtom));
+                            tc_copy_scales_pair(sfr + 16 + j * 8 + 4,
+                                                sdesc_scales(ssfb + kAtomsPerStep * kAtom + j * kAtom));
+                        }
+                        tc_commit_pair(&sf_ready[stage], 0x1);
                     }
-                    tc_commit_pair(&sf_ready[stage], 0x1);
+                    __syncwarp();
                     if (++stage == STAGES) {
                         stage = 0;
                         phase ^= 1u;
                     }
                 }
             }
-            tc_commit_pair(drain2, 0x1);
-            int local_abort = 0;
-            mbar_wait_bounded(drain2, 0, args.timeout_ns, &local_abort, args.status);
+            if (elect_one()) {
+                tc_commit_pair(drain2, 0x1);
+                int local_abort = 0;
+                mbar_wait_bounded(drain2, 0, args.timeout_ns, &local_abort, args.status);
+            }
+            __syncwarp();
         }
     } else {
         // ---------------- epilogue (warps 2..9, both CTAs) ----------------
