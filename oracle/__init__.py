@@ -89,6 +89,8 @@ def _L():
         lib.oracle_num_threads.restype = ctypes.c_int
         lib.oracle_silu_mul.argtypes = [P, I64, I64, I64, P]
         lib.oracle_silu_mul.restype = None
+        lib.oracle_harmonize_scales.argtypes = [P, I64, I64, P, P, ctypes.c_int, P]
+        lib.oracle_harmonize_scales.restype = ctypes.c_float
         _lib = lib
     return _lib
 
@@ -240,6 +242,27 @@ def silu_mul(gate_up_bf16: np.ndarray) -> np.ndarray:
     h = np.empty((rows, f), np.uint16)
     _L().oracle_silu_mul(_ptr(gu), rows, f, two_f, _ptr(h))
     return h
+
+
+def harmonize_scales(sf_linear: np.ndarray, segments):
+    """Checkpoint-side harmonisation of a fused weight's block scales.
+
+    sf_linear: linear [rows, sfcols] scale bytes of the fused weight;
+    segments: [(n_offset, n_size, g)] tiling the rows in order.  Returns
+    (g_c, sf') with g_c = max g and every module's scales re-expressed
+    against g_c, codes unchanged (oracle_harmonize_scales in the C file)."""
+    sf = _c(sf_linear, np.uint8)
+    rows, sfcols = sf.shape
+    expect = 0
+    for off, size, _ in segments:
+        assert int(off) == expect, "segments must tile the rows in order"
+        expect += int(size)
+    seg_rows = np.array([int(s[1]) for s in segments], np.int64)
+    seg_g = np.array([float(np.float32(s[2])) for s in segments], np.float32)
+    out = np.empty_like(sf)
+    gc = _L().oracle_harmonize_scales(_ptr(sf), rows, sfcols, _ptr(seg_rows), _ptr(seg_g),
+                                      len(segments), _ptr(out))
+    return np.float32(gc), out
 
 
 def num_threads() -> int:

@@ -352,3 +352,44 @@ void oracle_silu_mul(const uint16_t* gu, int64_t rows, int64_t f, int64_t ld, ui
             h[r * f + c] = oracle_bf16_from_double(s * u);
         }
 }
+
+/* ---------------------------------------------------------------------- */
+/* Checkpoint-side scale harmonisation                                     */
+/* ---------------------------------------------------------------------- */
+
+/* A fused multi-module GEMM that applies ONE global scale to a weight whose
+ * modules were quantized with their own scales is the global-scale mismatch
+ * the pages repair (chatpaper.ai abstract).  Besides applying each module's
+ * scale per N-segment in the epilogue, the repair can be made on the
+ * checkpoint: re-express every module's block scales against one common
+ * scale and keep the codes.  The pages give no formula; the plainest reading
+ * that never saturates a scale takes the largest module scale as common:
+ *   g_c = max_i g_i
+ *   r_i = fl32(g_i / g_c)                          (one binary32 division)
+ *   s8' = E4M3_RNE_satfinite(fl32(E4M3(s8) * r_i)) (one binary32 multiply)
+ * E4M3(s8') * g_c then approximates E4M3(s8) * g_i, exactly when the product
+ * is an E4M3 value; r_i <= 1, so modules with small scales drift into the
+ * E4M3 subnormals and lose precision.
+ * sf_in/sf_out: linear [rows, sfcols] scale bytes (codes 0..0x7E); the
+ * modules are consecutive row ranges of seg_rows[i] rows with scales
+ * seg_g[i].  Returns g_c. */
+float oracle_harmonize_scales(const uint8_t* sf_in, int64_t rows, int64_t sfcols,
+                              const int64_t* seg_rows, const float* seg_g, int nseg,
+                              uint8_t* sf_out)
+{
+    float gc = seg_g[0];
+    for (int i = 1; i < nseg; ++i)
+        if (seg_g[i] > gc) gc = seg_g[i];
+    int64_t r0 = 0;
+    for (int i = 0; i < nseg; ++i) {
+        const float ratio = seg_g[i] / gc;
+        for (int64_t r = r0; r < r0 + seg_rows[i] && r < rows; ++r)
+            for (int64_t c = 0; c < sfcols; ++c) {
+                const float dec = (float)oracle_e4m3_value(sf_in[r * sfcols + c]);  /* exact */
+                const float prod = dec * ratio;
+                sf_out[r * sfcols + c] = (uint8_t)oracle_e4m3_encode(prod);
+            }
+        r0 += seg_rows[i];
+    }
+    return gc;
+}

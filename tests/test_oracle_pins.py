@@ -466,3 +466,62 @@ def test_silu_mul_single_rounding_matches_exact_value():
     d0 = np.abs(hv - exact)
     assert np.all((d0 <= np.abs(up - exact)) | (h == 0x7F7F))
     assert np.all((d0 <= np.abs(dn - exact)) | ((h & 0x7FFF) == 0))
+
+
+# --------------------------------------------------------------------------
+# checkpoint-side scale harmonisation (chatpaper.ai abstract: the fused-module
+# global-scale mismatch and its repair; reading: common scale = max module scale)
+# --------------------------------------------------------------------------
+
+def _harm_one(s8, gi, gc):
+    sf = np.array([[s8], [0]], np.uint8)
+    g_c, out = oracle.harmonize_scales(sf, [(0, 1, np.float32(gi)), (1, 1, np.float32(gc))])
+    return g_c, int(out[0, 0])
+
+
+def test_harmonize_golden(golden_dir):
+    for line in read_golden(os.path.join(golden_dir, "harmonize_points.txt")):
+        gi, gc, s8, expect = line.split()[:4]
+        g_c, got = _harm_one(int(s8, 16), float(gi), float(gc))
+        assert g_c == np.float32(max(float(gi), float(gc)))
+        assert got == int(expect, 16), line
+
+
+def test_harmonize_matches_torch_cast_exhaustive():
+    # every scale byte x several ratios against an independent library path:
+    # decode by the format's bit fields, one float32 multiply, torch's RNE cast
+    codes = np.arange(0x7F, dtype=np.uint8)
+    dec = torch.from_numpy(codes.copy()).view(torch.float8_e4m3fn).float()
+    for gi, gc in [(0.3, 1.0), (1.0, 3.0), (0.01, 1.0), (0.77, 0.8), (1e-3, 0.2), (0.015, 0.02)]:
+        ratio = np.float32(np.float32(gi) / np.float32(gc))
+        prod = (dec * torch.tensor(ratio, dtype=torch.float32)).numpy()
+        ref = torch.from_numpy(prod).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+        sf = np.stack([codes, np.zeros_like(codes)])
+        g_c, out = oracle.harmonize_scales(sf, [(0, 1, np.float32(gi)), (1, 1, np.float32(gc))])
+        assert np.array_equal(out[0], ref), (gi, gc)
+        assert np.all(out[1] == 0)
+
+
+def test_harmonize_power_of_two_ratio_closed_form():
+    # ratio 2^-k moves a normal scale k binades down: the code drops by 8k while
+    # the exponent field stays >= 1, and the value is exactly E4M3(s8) * 2^-k
+    for k in (1, 2, 3):
+        for s8 in range(8 * (k + 1), 0x7F):
+            _, got = _harm_one(s8, 2.0 ** -k, 1.0)
+            assert got == s8 - 8 * k
+            assert oracle.e4m3_value(got) == oracle.e4m3_value(s8) * 2.0 ** -k
+
+
+def test_harmonize_max_module_unchanged_and_shape():
+    rng = np.random.default_rng(7)
+    sf = rng.integers(0, 0x7F, size=(40, 12), dtype=np.uint8)
+    segs = [(0, 10, np.float32(0.02)), (10, 25, np.float32(0.2)), (35, 5, np.float32(0.002))]
+    g_c, out = oracle.harmonize_scales(sf, segs)
+    assert g_c == np.float32(0.2)
+    assert np.array_equal(out[10:35], sf[10:35])            # the max-scale module
+    assert np.all(out[:10] <= sf[:10]) and np.all(out[35:] <= sf[35:])   # ratio <= 1 never grows a scale
+    # the other modules are the single-module formula row range by row range
+    for off, n, g in segs:
+        _, ref = oracle.harmonize_scales(np.concatenate([sf[off:off + n], np.zeros((1, 12), np.uint8)]),
+                                         [(0, n, g), (n, 1, g_c)])
+        assert np.array_equal(out[off:off + n], ref[:n])
