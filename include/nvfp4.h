@@ -192,6 +192,34 @@ nvfp4_status nvfp4_fused_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const
                               void* y, int64_t ldy, int64_t M, int64_t K,
                               void* stream);
 
+/* Checkpoint-side repair of the global-scale mismatch: rewrite the block
+ * scales of a fused weight so that ONE global scale serves all its modules.
+ *   g_c  = max_i *segs[i].w_gscale                 (written to *g_common)
+ *   r_i  = fl32(g_i / g_c)
+ *   s8' = E4M3_RNE_satfinite(fl32(E4M3(s8) * r_i)) for every scale byte of
+ *          module i's rows; the codes are not touched.
+ * Afterwards nvfp4_gemm(..., w_sf, g_common, ...) serves the fused weight
+ * with a single scale; E4M3(s8') * g_c equals E4M3(s8) * g_i where that
+ * product is an E4M3 value and rounds it otherwise (modules with small
+ * scales lose precision in the E4M3 subnormals).  This is the alternative to
+ * the per-segment epilogue of nvfp4_fused_gemm.
+ *   w_sf     (device, in/out) scale bytes of the fused [N, K] weight in
+ *            `layout`, N = sum of n_size (padding bytes of the tensor-core
+ *            layout stay 0).  16-byte aligned.
+ *   K        multiple of 16 (so cols/16 scales per row).
+ *   segs     (host, nseg entries, copied during the call): as for
+ *            nvfp4_fused_gemm; the w_gscale pointers are device FP32.
+ *   g_common (device) receives g_c.
+ * Errors: NVFP4_ERR_INVALID_ARG (null pointer, bad segment table, bad
+ * layout), NVFP4_ERR_UNSUPPORTED_SHAPE (K), NVFP4_ERR_ALIGNMENT, CUDA errors.
+ * Asynchronous on `stream`.
+ * Source: chatpaper.ai abstract (per-module-calibrated checkpoints, fused
+ * multi-module kernels, the global-scale mismatch and its repair); the choice
+ * of the largest module scale as the common one is a reading -- the pages
+ * give no formula. */
+nvfp4_status nvfp4_harmonize_scales(uint8_t* w_sf, int64_t K, const nvfp4_segment* segs, int nseg,
+                                    nvfp4_sf_layout layout, float* g_common, void* stream);
+
 /* MLP intermediate for the W4A4 down projection: h[r, c] = BF16_RNE(
  * fl32(SiLU(gate) * up)) with gate = gate_up[r, c], up = gate_up[r, f + c]
  * (BF16, row stride ld elements, device) and SiLU(v) = v / (1 + e^-v)

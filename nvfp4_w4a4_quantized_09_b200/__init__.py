@@ -27,7 +27,7 @@ from ._lib import SF_LINEAR, SF_TCGEN05, MAX_SEGMENTS, Nvfp4Error
 __all__ = [
     "SF_LINEAR", "SF_TCGEN05", "MAX_SEGMENTS", "Nvfp4Error", "QuantizedTensor",
     "global_scale", "sf_bytes", "quantize", "quantize_into", "quantize_tensor",
-    "gemm", "fused_gemm", "FusedWeight", "linear", "silu_mul", "mlp", "last_device_status",
+    "gemm", "fused_gemm", "FusedWeight", "linear", "silu_mul", "mlp", "harmonize", "last_device_status",
     "debug_wait_timeout", "library_path",
 ]
 
@@ -185,6 +185,27 @@ class FusedWeight:
             out.append((off, n, g))
             off += n
         return out
+
+
+def _segment_array(segments):
+    arr = (_lib.Segment * max(len(segments), 1))()
+    for i, (off, n, g) in enumerate(segments):
+        arr[i].n_offset = int(off)
+        arr[i].n_size = int(n)
+        arr[i].w_gscale = g.data_ptr()
+    return arr
+
+
+def harmonize(w: "FusedWeight", layout: int = SF_TCGEN05, stream=None) -> QuantizedTensor:
+    """Checkpoint-side repair of the global-scale mismatch: a copy of the
+    fused weight's block scales re-expressed against g_c = max_i g_i (codes
+    shared, not copied), served afterwards by the single-scale GEMM."""
+    sf = w.sf.clone()
+    g_c = torch.empty(1, dtype=torch.float32, device=w.sf.device)
+    segs = w.segments()
+    _lib.check("nvfp4_harmonize_scales", _lib.lib().nvfp4_harmonize_scales(
+        _ptr(sf), w.cols, _segment_array(segs), len(segs), layout, _ptr(g_c), _stream(stream)))
+    return QuantizedTensor(w.codes, sf, g_c, w.rows, w.cols, layout)
 
 
 def fused_gemm(a: QuantizedTensor, w_codes: torch.Tensor, w_sf: torch.Tensor,

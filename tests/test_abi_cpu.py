@@ -125,6 +125,24 @@ def test_fused_gemm_validates_segment_table(L):
     assert f(*args, good, 2, FAKE, 128, 0, 64, NUL) == _lib.NVFP4_OK                   # M = 0
 
 
+def test_harmonize_rejects_bad_arguments(L):
+    f = L.nvfp4_harmonize_scales
+    good = seg_array([(0, 64, 0x10000), (64, 64, 0x10010)])
+    T, LIN = _lib.SF_TCGEN05, _lib.SF_LINEAR
+    assert f(NUL, 64, good, 2, T, FAKE, NUL) == _lib.NVFP4_ERR_INVALID_ARG     # no scales
+    assert f(FAKE, 64, good, 2, T, NUL, NUL) == _lib.NVFP4_ERR_INVALID_ARG     # no g_common
+    assert f(FAKE, 64, good, 0, T, FAKE, NUL) == _lib.NVFP4_ERR_INVALID_ARG    # nseg 0
+    assert f(FAKE, 64, good, 17, T, FAKE, NUL) == _lib.NVFP4_ERR_INVALID_ARG   # > max
+    assert f(FAKE, 64, good, 2, 7, FAKE, NUL) == _lib.NVFP4_ERR_INVALID_ARG    # layout
+    gap = seg_array([(0, 64, 0x10000), (72, 64, 0x10010)])
+    assert f(FAKE, 64, gap, 2, LIN, FAKE, NUL) == _lib.NVFP4_ERR_INVALID_ARG   # not contiguous
+    noscale = seg_array([(0, 64, 0x10000), (64, 64, 0)])
+    assert f(FAKE, 64, noscale, 2, LIN, FAKE, NUL) == _lib.NVFP4_ERR_INVALID_ARG
+    assert f(FAKE, 24, good, 2, T, FAKE, NUL) == _lib.NVFP4_ERR_UNSUPPORTED_SHAPE   # K % 16
+    assert f(FAKE, 0, good, 2, T, FAKE, NUL) == _lib.NVFP4_ERR_UNSUPPORTED_SHAPE
+    assert f(ctypes.c_void_p(0x10008), 64, good, 2, T, FAKE, NUL) == _lib.NVFP4_ERR_ALIGNMENT
+
+
 def test_debug_wait_rejects_bad_limits(L):
     assert L.nvfp4_debug_wait_timeout(0, NUL) == _lib.NVFP4_ERR_INVALID_ARG
     assert L.nvfp4_debug_wait_timeout(2_000_000_000, NUL) == _lib.NVFP4_ERR_INVALID_ARG
