@@ -782,6 +782,8 @@ bool make_sf_map(CUtensorMap* m, const uint8_t* base, int64_t rowblocks, int64_t
     return r == CUDA_SUCCESS;
 }
 
+}  // namespace
+
 int* device_status_ptr() {
     static int* cache[64] = {nullptr};
     int dev = 0;
@@ -793,6 +795,8 @@ int* device_status_ptr() {
     }
     return cache[dev];
 }
+
+namespace {
 
 template <int BN, int STAGES, int ACC>
 nvfp4_status launch_gemm(const uint8_t* a_codes, const uint8_t* w_codes, GemmArgs& args,

@@ -25,6 +25,10 @@ struct DeviceInfo {
 
 nvfp4_status current_device_info(DeviceInfo* info);
 
+// Device address of the library's status word (set by kernels whose bounded
+// waits gave up), looked up once per device; nullptr on a CUDA error.
+int* device_status_ptr();
+
 // The block-scaled FP4 tensor-core path needs an sm_100 device.
 inline nvfp4_status require_sm100(DeviceInfo* info) {
     nvfp4_status st = current_device_info(info);
