@@ -91,6 +91,10 @@ def _L():
         lib.oracle_silu_mul.restype = None
         lib.oracle_harmonize_scales.argtypes = [P, I64, I64, P, P, ctypes.c_int, P]
         lib.oracle_harmonize_scales.restype = ctypes.c_float
+        lib.oracle_kv_scale.argtypes = [ctypes.c_float]
+        lib.oracle_kv_scale.restype = ctypes.c_float
+        lib.oracle_kv_quantize.argtypes = [P, I64, I64, I64, ctypes.c_float, P]
+        lib.oracle_kv_quantize.restype = None
         _lib = lib
     return _lib
 
@@ -263,6 +267,20 @@ def harmonize_scales(sf_linear: np.ndarray, segments):
     gc = _L().oracle_harmonize_scales(_ptr(sf), rows, sfcols, _ptr(seg_rows), _ptr(seg_g),
                                       len(segments), _ptr(out))
     return np.float32(gc), out
+
+
+def kv_scale(amax: float) -> np.float32:
+    """Calibrated per-tensor FP8 KV-cache scale fl32(amax / 448) (1 if amax = 0)."""
+    return np.float32(_L().oracle_kv_scale(ctypes.c_float(float(np.float32(amax)))))
+
+
+def kv_quantize(x_bf16: np.ndarray, s: float) -> np.ndarray:
+    """Signed E4M3 bytes of fl32(x / s), RNE, saturating at 448 (oracle_kv_quantize)."""
+    x = _c(x_bf16, np.uint16)
+    rows, cols = x.shape
+    out = np.empty((rows, cols), np.uint8)
+    _L().oracle_kv_quantize(_ptr(x), rows, cols, cols, ctypes.c_float(float(np.float32(s))), _ptr(out))
+    return out
 
 
 def num_threads() -> int:

@@ -525,3 +525,50 @@ def test_harmonize_max_module_unchanged_and_shape():
         _, ref = oracle.harmonize_scales(np.concatenate([sf[off:off + n], np.zeros((1, 12), np.uint8)]),
                                          [(0, n, g), (n, 1, g_c)])
         assert np.array_equal(out[off:off + n], ref[:n])
+
+
+# --------------------------------------------------------------------------
+# FP8 E4M3 KV-cache quantization with a calibrated per-tensor scale
+# (evolve.pub, Key claims under review, last bullet; reading beside the oracle)
+# --------------------------------------------------------------------------
+
+def _bf16(vals):
+    return torch.tensor(vals, dtype=torch.float32).to(torch.bfloat16).view(torch.int16).numpy() \
+        .astype(np.uint16)
+
+
+def test_kv_quantize_golden(golden_dir):
+    for line in read_golden(os.path.join(golden_dir, "kv_e4m3_points.txt")):
+        xv, sv, expect = line.split()[:3]
+        got = oracle.kv_quantize(_bf16([[float(xv)]]), float(sv))[0, 0]
+        assert got == int(expect, 16), line
+
+
+@pytest.mark.parametrize("s", [1.0, 0.37, 3.1e-3, 41.0])
+def test_kv_quantize_matches_torch_cast_exhaustive_bf16(s):
+    # every finite BF16 value: the quotient by one float32 division, then
+    # torch's RNE float8_e4m3fn cast in range and +-448 beyond (satfinite)
+    bits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    vals = (bits.astype(np.uint32) << 16).view(np.float32)
+    keep = np.isfinite(vals)
+    bits, vals = bits[keep], vals[keep]
+    with np.errstate(over="ignore"):                 # quotients beyond float32 saturate too
+        t = (vals / np.float32(s)).astype(np.float32)
+    got = oracle.kv_quantize(bits.reshape(1, -1), s)[0]
+    inr = np.abs(t) <= 448
+    ref = torch.from_numpy(t[inr].copy()).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(got[inr], ref)
+    sat = np.where(np.signbit(t[~inr]), 0xFE, 0x7E).astype(np.uint8)
+    assert np.array_equal(got[~inr], sat)
+
+
+def test_kv_scale_maps_amax_to_448():
+    rng = np.random.default_rng(3)
+    for amax in [1.0, 448.0, 0.0123, 7.5e3, float(rng.uniform(0.1, 100))]:
+        s = oracle.kv_scale(amax)
+        assert s == np.float32(np.float32(amax) / np.float32(448.0))
+        b = _bf16([[amax, -amax]])
+        a_b = float(torch.from_numpy(b.view(np.int16)).view(torch.bfloat16).float()[0, 0])
+        codes = oracle.kv_quantize(b, oracle.kv_scale(a_b))[0]
+        assert codes[0] == 0x7E and codes[1] == 0xFE     # the calibration absmax is the largest code
+    assert oracle.kv_scale(0.0) == np.float32(1.0)
