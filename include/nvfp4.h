@@ -220,6 +220,28 @@ nvfp4_status nvfp4_fused_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const
 nvfp4_status nvfp4_harmonize_scales(uint8_t* w_sf, int64_t K, const nvfp4_segment* segs, int nseg,
                                     nvfp4_sf_layout layout, float* g_common, void* stream);
 
+/* FP8 E4M3 KV cache with a calibrated per-tensor scale.
+ *
+ * nvfp4_kv_scale_from_amax: *scale = fl32(*amax / 448), or 1 when *amax is 0
+ * (both device FP32; amax as written by nvfp4_global_scale's amax_out over the
+ * calibration tensor).  Errors: NVFP4_ERR_INVALID_ARG (null), CUDA errors.
+ *
+ * nvfp4_kv_quantize_e4m3: out[r, c] = signed E4M3 byte of fl32(x[r, c] /
+ * *scale), round to nearest even, saturating at +-448 (the NaN code is never
+ * written), bit 7 the sign of the quotient (kept for zero).  Every byte
+ * equals the one an IEEE division would give.
+ *   x      (device) BF16 [rows, cols], row stride ld elements; 16-byte aligned.
+ *   scale  (device) FP32 per-tensor scale, positive and finite.
+ *   out    (device) bytes [rows, cols], row stride ldo bytes; 8-byte aligned.
+ * Requirements: cols, ld, ldo multiples of 8; ld >= cols, ldo >= cols.
+ * Errors: NVFP4_ERR_INVALID_ARG, NVFP4_ERR_ALIGNMENT, CUDA errors.  Both calls
+ * are asynchronous on `stream`.
+ * Source: evolve.pub, Key claims under review (calibrated per-tensor FP8
+ * KV-cache scales); the formula is a reading -- the pages give none. */
+nvfp4_status nvfp4_kv_scale_from_amax(const float* amax, float* scale, void* stream);
+nvfp4_status nvfp4_kv_quantize_e4m3(const void* x, int64_t rows, int64_t cols, int64_t ld,
+                                    const float* scale, uint8_t* out, int64_t ldo, void* stream);
+
 /* MLP intermediate for the W4A4 down projection: h[r, c] = BF16_RNE(
  * fl32(SiLU(gate) * up)) with gate = gate_up[r, c], up = gate_up[r, f + c]
  * (BF16, row stride ld elements, device) and SiLU(v) = v / (1 + e^-v)

@@ -27,7 +27,7 @@ from ._lib import SF_LINEAR, SF_TCGEN05, MAX_SEGMENTS, Nvfp4Error
 __all__ = [
     "SF_LINEAR", "SF_TCGEN05", "MAX_SEGMENTS", "Nvfp4Error", "QuantizedTensor",
     "global_scale", "sf_bytes", "quantize", "quantize_into", "quantize_tensor",
-    "gemm", "fused_gemm", "FusedWeight", "linear", "silu_mul", "mlp", "harmonize", "last_device_status",
+    "gemm", "fused_gemm", "FusedWeight", "linear", "silu_mul", "mlp", "harmonize", "kv_scale", "kv_quantize", "last_device_status",
     "debug_wait_timeout", "library_path",
 ]
 
@@ -256,6 +256,28 @@ def mlp(x: torch.Tensor, w_gate_up, w_down, stream=None) -> torch.Tensor:
     gu = linear(x, w_gate_up, stream=stream)
     h = silu_mul(gu, stream=stream)
     return linear(h, w_down, stream=stream)
+
+
+def kv_scale(calibration: torch.Tensor, stream=None) -> torch.Tensor:
+    """Calibrated per-tensor FP8 KV-cache scale fl32(amax / 448) of a BF16
+    calibration tensor (device FP32, 1 element)."""
+    _, amax = global_scale(calibration, stream=stream)
+    s = torch.empty(1, dtype=torch.float32, device=calibration.device)
+    _lib.check("nvfp4_kv_scale_from_amax",
+               _lib.lib().nvfp4_kv_scale_from_amax(_ptr(amax), _ptr(s), _stream(stream)))
+    return s
+
+
+def kv_quantize(x: torch.Tensor, scale: torch.Tensor, out: Optional[torch.Tensor] = None,
+                stream=None) -> torch.Tensor:
+    """Signed E4M3 bytes of x / scale (RNE, saturating at 448) as uint8 [rows, cols]."""
+    _check_bf16_matrix(x, "x")
+    rows, cols = x.shape
+    if out is None:
+        out = torch.empty(rows, cols, dtype=torch.uint8, device=x.device)
+    _lib.check("nvfp4_kv_quantize_e4m3", _lib.lib().nvfp4_kv_quantize_e4m3(
+        _ptr(x), rows, cols, x.stride(0), _ptr(scale), _ptr(out), out.stride(0), _stream(stream)))
+    return out
 
 
 def last_device_status(stream=None) -> int:

@@ -49,6 +49,8 @@ SIGNATURES = {
     "nvfp4_fused_gemm": (ST, [P, P, P, P, P, ctypes.POINTER(Segment), I32, P, I64, I64, I64, P]),
     "nvfp4_silu_mul": (ST, [P, I64, I64, I64, P, I64, P]),
     "nvfp4_harmonize_scales": (ST, [P, I64, ctypes.POINTER(Segment), I32, I32, P, P]),
+    "nvfp4_kv_scale_from_amax": (ST, [P, P, P]),
+    "nvfp4_kv_quantize_e4m3": (ST, [P, I64, I64, I64, P, P, I64, P]),
     "nvfp4_last_device_status": (ST, [P]),
     "nvfp4_debug_wait_timeout": (ST, [I64, P]),
     "nvfp4_status_string": (ctypes.c_char_p, [ST]),

@@ -143,6 +143,22 @@ def test_harmonize_rejects_bad_arguments(L):
     assert f(ctypes.c_void_p(0x10008), 64, good, 2, T, FAKE, NUL) == _lib.NVFP4_ERR_ALIGNMENT
 
 
+def test_kv_cache_entries_reject_bad_arguments(L):
+    q = L.nvfp4_kv_quantize_e4m3
+    assert q(FAKE, -1, 8, 8, FAKE, FAKE, 8, NUL) == _lib.NVFP4_ERR_INVALID_ARG
+    assert q(FAKE, 4, 8, 8, NUL, FAKE, 8, NUL) == _lib.NVFP4_ERR_INVALID_ARG      # no scale
+    assert q(FAKE, 4, 12, 16, FAKE, FAKE, 16, NUL) == _lib.NVFP4_ERR_ALIGNMENT    # cols % 8
+    assert q(FAKE, 4, 8, 12, FAKE, FAKE, 8, NUL) == _lib.NVFP4_ERR_ALIGNMENT      # ld % 8
+    assert q(FAKE, 4, 8, 8, FAKE, FAKE, 12, NUL) == _lib.NVFP4_ERR_ALIGNMENT      # ldo % 8
+    assert q(NUL, 4, 8, 8, FAKE, FAKE, 8, NUL) == _lib.NVFP4_ERR_INVALID_ARG      # no x
+    assert q(FAKE, 4, 16, 8, FAKE, FAKE, 16, NUL) == _lib.NVFP4_ERR_INVALID_ARG   # ld < cols
+    assert q(ODD, 4, 8, 8, FAKE, FAKE, 8, NUL) == _lib.NVFP4_ERR_ALIGNMENT        # x not 16-aligned
+    assert q(FAKE, 4, 8, 8, FAKE, ctypes.c_void_p(0x10004), 8, NUL) == _lib.NVFP4_ERR_ALIGNMENT
+    assert q(FAKE, 0, 8, 8, FAKE, FAKE, 8, NUL) == _lib.NVFP4_OK                 # nothing to do
+    assert L.nvfp4_kv_scale_from_amax(NUL, FAKE, NUL) == _lib.NVFP4_ERR_INVALID_ARG
+    assert L.nvfp4_kv_scale_from_amax(FAKE, NUL, NUL) == _lib.NVFP4_ERR_INVALID_ARG
+
+
 def test_debug_wait_rejects_bad_limits(L):
     assert L.nvfp4_debug_wait_timeout(0, NUL) == _lib.NVFP4_ERR_INVALID_ARG
     assert L.nvfp4_debug_wait_timeout(2_000_000_000, NUL) == _lib.NVFP4_ERR_INVALID_ARG
