@@ -95,6 +95,8 @@ def _L():
         lib.oracle_kv_scale.restype = ctypes.c_float
         lib.oracle_kv_quantize.argtypes = [P, I64, I64, I64, ctypes.c_float, P]
         lib.oracle_kv_quantize.restype = None
+        lib.oracle_gdn_gates.argtypes = [P, I64, I64, I64, P, P, ctypes.c_int, P]
+        lib.oracle_gdn_gates.restype = None
         _lib = lib
     return _lib
 
@@ -280,6 +282,21 @@ def kv_quantize(x_bf16: np.ndarray, s: float) -> np.ndarray:
     rows, cols = x.shape
     out = np.empty((rows, cols), np.uint8)
     _L().oracle_kv_quantize(_ptr(x), rows, cols, cols, ctypes.c_float(float(np.float32(s))), _ptr(out))
+    return out
+
+
+GATE_DECAY, GATE_SIGMOID = 1, 2
+
+
+def gdn_gates(y64: np.ndarray, kind: int, a_log=None, dt_bias=None) -> np.ndarray:
+    """BF16 bits of the gate functions on FP64 GEMM values y64 [rows, ncols]:
+    kind 1 g = -exp(A_log) softplus(y + dt_bias) per column, kind 2 sigmoid(y)."""
+    y = _c(y64, np.float64)
+    rows, ncols = y.shape
+    al = _c(np.zeros(ncols) if a_log is None else a_log, np.float32)
+    db = _c(np.zeros(ncols) if dt_bias is None else dt_bias, np.float32)
+    out = np.empty((rows, ncols), np.uint16)
+    _L().oracle_gdn_gates(_ptr(y), rows, ncols, ncols, _ptr(al), _ptr(db), int(kind), _ptr(out))
     return out
 
 

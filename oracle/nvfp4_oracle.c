@@ -422,3 +422,38 @@ void oracle_kv_quantize(const uint16_t* x, int64_t rows, int64_t cols, int64_t l
             out[r * cols + c] = (uint8_t)code;
         }
 }
+
+/* ---------------------------------------------------------------------- */
+/* Gated DeltaNet gate epilogue                                            */
+/* ---------------------------------------------------------------------- */
+
+/* The fused GDN input projection carries the two gate projections: a (one
+ * column per head) feeds the log-space decay gate and b feeds the sigmoid
+ * write strength; the pages credit these "log-space softplus/exponential and
+ * sigmoid parameterizations" with compressing ~11 % GEMM error to ~2 % output
+ * error (evolve.pub, Key claims under review, second bullet; Report preview,
+ * Table 3).  They give no formula; the plain reading is the Gated DeltaNet
+ * parameterisation:
+ *   decay (kind 1): g    = -exp(A_log[c]) * softplus(y + dt_bias[c]),
+ *                   softplus(z) = log(1 + e^z), per column c of the segment
+ *   sigmoid (kind 2): beta = 1 / (1 + e^-y)
+ * evaluated in FP64 on the exact GEMM value y (row-major [rows, ncols], row
+ * stride ld) and rounded once to BF16 (bits in out, [rows, ncols]). */
+void oracle_gdn_gates(const double* y, int64_t rows, int64_t ncols, int64_t ld,
+                      const float* a_log, const float* dt_bias, int kind, uint16_t* out)
+{
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t c = 0; c < ncols; ++c) {
+            const double v = y[r * ld + c];
+            double o;
+            if (kind == 1) {
+                const double z = v + (double)dt_bias[c];
+                /* log(1 + e^z) written so that neither branch overflows */
+                const double sp = z > 0.0 ? z + log1p(exp(-z)) : log1p(exp(z));
+                o = -exp((double)a_log[c]) * sp;
+            } else {
+                o = 1.0 / (1.0 + exp(-v));
+            }
+            out[r * ncols + c] = oracle_bf16_from_double(o);
+        }
+}

@@ -572,3 +572,55 @@ def test_kv_scale_maps_amax_to_448():
         codes = oracle.kv_quantize(b, oracle.kv_scale(a_b))[0]
         assert codes[0] == 0x7E and codes[1] == 0xFE     # the calibration absmax is the largest code
     assert oracle.kv_scale(0.0) == np.float32(1.0)
+
+
+# --------------------------------------------------------------------------
+# Gated DeltaNet gate epilogue (evolve.pub, Key claims under review, second
+# bullet: log-space softplus/exponential decay and sigmoid parameterizations)
+# --------------------------------------------------------------------------
+
+def test_gates_closed_forms():
+    # sigmoid: exact values 1/2, 3/4, 1/4 at 0, +-ln 3
+    y = np.array([[0.0, np.log(3.0), -np.log(3.0)]])
+    assert list(oracle.gdn_gates(y, oracle.GATE_SIGMOID)[0]) == [0x3F00, 0x3F40, 0x3E80]
+    # decay: softplus(ln(e - 1)) = 1, so g = -exp(A_log); softplus(0) = ln 2
+    z = np.log(np.e - 1.0)
+    a_log = np.array([0.0, np.log(np.float32(4.0)), 0.0], np.float32)
+    g = oracle.gdn_gates(np.array([[z, z, 0.0]]), oracle.GATE_DECAY, a_log=a_log,
+                         dt_bias=np.zeros(3, np.float32))[0]
+    assert g[0] == 0xBF80 and g[1] == 0xC080                      # -1, -4
+    assert g[2] == oracle.bf16_from_double(np.array([-np.log(2.0)]))[0]
+    # dt_bias shifts the argument: y + b = 0 gives ln 2 whatever the split
+    g2 = oracle.gdn_gates(np.array([[1.5]]), oracle.GATE_DECAY, a_log=np.zeros(1, np.float32),
+                          dt_bias=np.array([-1.5], np.float32))[0, 0]
+    assert g2 == g[2]
+
+
+def test_gates_match_torch_float64():
+    rng = np.random.default_rng(11)
+    y = rng.uniform(-20, 20, size=(64, 48))
+    a_log = rng.uniform(0.0, 2.8, size=48).astype(np.float32)
+    dt_bias = rng.uniform(-7.0, -2.0, size=48).astype(np.float32)
+    yt = torch.from_numpy(y)
+    sig = torch.sigmoid(yt).numpy()
+    assert np.array_equal(oracle.gdn_gates(y, oracle.GATE_SIGMOID), oracle.bf16_from_double(sig))
+    z = yt + torch.from_numpy(dt_bias.astype(np.float64))
+    dec = (-torch.exp(torch.from_numpy(a_log.astype(np.float64))) *
+           torch.nn.functional.softplus(z, beta=1.0, threshold=50.0)).numpy()
+    assert np.array_equal(oracle.gdn_gates(y, oracle.GATE_DECAY, a_log, dt_bias),
+                          oracle.bf16_from_double(dec))
+
+
+def test_gates_monotone_signs_and_tails():
+    y = np.linspace(-60, 60, 4001).reshape(1, -1)
+    s = oracle.bf16_bits_to_f64(oracle.gdn_gates(y, oracle.GATE_SIGMOID))[0]
+    assert np.all(np.diff(s) >= 0) and s.min() >= 0 and s.max() <= 1
+    n = y.shape[1]
+    g = oracle.bf16_bits_to_f64(oracle.gdn_gates(y, oracle.GATE_DECAY, np.full(n, 0.5, np.float32),
+                                                 np.zeros(n, np.float32)))[0]
+    assert np.all(np.diff(g) <= 0) and g.max() <= 0
+    # far tails: softplus(z) -> z for large z, -> e^z for very negative z
+    big = oracle.gdn_gates(np.array([[300.0, -300.0]]), oracle.GATE_DECAY,
+                           np.zeros(2, np.float32), np.zeros(2, np.float32))[0]
+    assert big[0] == oracle.bf16_from_double(np.array([-300.0]))[0]
+    assert big[1] == oracle.bf16_from_double(np.array([-np.exp(-300.0)]))[0]
