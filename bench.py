@@ -393,6 +393,50 @@ def run_ours(args, dev, world, rank):
     sanity = float((y[rows].float() - ref).norm() / ref.norm())
     del w_bf16
 
+    # gate epilogue (Gated DeltaNet decay gate on segment a, sigmoid on b):
+    # the pages' GEMM-error -> gate-output-error compression (Table 3: 11.0 % /
+    # 8.5 % GEMM error -> 2.1 % / 2.6 % output), here on the synthetic workload,
+    # against gates computed in FP32 from the unquantized BF16 GEMM
+    gates = None
+    if not args.no_gates:
+        a_off, a_n, _ = segs[5]
+        b_off, b_n, _ = segs[4]
+        a_log, dt_bias = synth.gdn_gate_params(a_n, seed=40, device=dev)
+        acts = [(nv.ACT_NONE, None, None)] * 4 + [(nv.ACT_SIGMOID, None, None),
+                                                  (nv.ACT_DECAY_GATE, a_log, dt_bias)]
+        aq = nv.quantize_tensor(x)
+        y_g = nv.fused_gemm(aq, fw.codes, fw.sf, segs, acts=acts)
+        torch.cuda.synchronize()
+
+        def rel(p_, r_):
+            return float((p_.double() - r_.double()).norm() / r_.double().norm())
+        ya_ref, yb_ref = ref[:, a_off:a_off + a_n], ref[:, b_off:b_off + b_n]
+        g_ref = -torch.exp(a_log)[None, :] * torch.nn.functional.softplus(ya_ref + dt_bias[None, :])
+        beta_ref = torch.sigmoid(yb_ref)
+        g_q = y_g[rows, a_off:a_off + a_n].float()
+        beta_q = y_g[rows, b_off:b_off + b_n].float()
+        tg = []
+        for act_on in (False, True):
+            evs_g = []
+            for it in range(12):
+                flush.zero_()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                nv.fused_gemm(aq, fw.codes, fw.sf, segs, y_g, acts=acts if act_on else None)
+                e1.record(stream)
+                evs_g.append((e0, e1))
+            torch.cuda.synchronize()
+            tg.append(float(np.median([a_.elapsed_time(b_) for a_, b_ in evs_g[2:]])) * 1e3)
+        gates = {"workload": "fused GDN projection with gate epilogue (a: decay gate, b: sigmoid), 16 sampled rows",
+                 "a_gemm_rel_err_vs_bf16": rel(y[rows, a_off:a_off + a_n], ya_ref),
+                 "a_gate_g_rel_err": rel(g_q, g_ref),
+                 "a_gate_exp_g_rel_err": rel(torch.exp(g_q), torch.exp(g_ref)),
+                 "b_gemm_rel_err_vs_bf16": rel(y[rows, b_off:b_off + b_n], yb_ref),
+                 "b_gate_beta_rel_err": rel(beta_q, beta_ref),
+                 "pages_table3": {"gemm_err": [0.110, 0.085], "output_err": [0.021, 0.026]},
+                 "fused_gemm_us": round(tg[0], 2), "fused_gemm_with_gates_us": round(tg[1], 2)}
+        del y_g, aq
+
     # checkpoint-side harmonisation (the single-scale repair, done once per
     # checkpoint): its kernel on the fused GDN weight's scales, and the error of
     # the single-scale GEMM against the per-segment epilogue, per module
@@ -468,7 +512,7 @@ def run_ours(args, dev, world, rank):
         "components_us": {"global_scale+quantize": round(float(np.mean(quant_ms)) * 1e3, 2),
                           "fused_gemm": round(gemm_avg_ms * 1e3, 2)},
         "roofline": roofline, "quantizer": quantizer, "e2e": e2e, "decode_sweep": decode, "mlp_32k": mlp_line,
-        "harmonize": harm, "kv_cache_fp8": kv,
+        "harmonize": harm, "kv_cache_fp8": kv, "gate_epilogue": gates,
         "gpu_launches": 3 * args.steps,
         "clocks": clk.summary(),
         "activation_stats": act_stats(x),
@@ -563,6 +607,7 @@ def main():
     ap.add_argument("--no-mlp", action="store_true")
     ap.add_argument("--no-harmonize", action="store_true")
     ap.add_argument("--no-kv", action="store_true")
+    ap.add_argument("--no-gates", action="store_true")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -71,6 +71,23 @@ typedef struct {
 } nvfp4_segment;
 
 #define NVFP4_MAX_SEGMENTS 16
+
+/* Elementwise function a fused GEMM may apply to one segment's outputs after
+ * the global scales (see nvfp4_fused_gemm_act). */
+typedef enum {
+    NVFP4_ACT_NONE = 0,
+    /* Gated DeltaNet log-space decay gate, per column c of the segment:
+     * g = -exp(a_log[c]) * softplus(y + dt_bias[c]), softplus(z) = log(1 + e^z). */
+    NVFP4_ACT_DECAY_GATE = 1,
+    /* Gated DeltaNet write strength: beta = 1 / (1 + e^-y). */
+    NVFP4_ACT_SIGMOID = 2
+} nvfp4_act_kind;
+
+typedef struct {
+    int kind;              /* nvfp4_act_kind */
+    const float* a_log;    /* NVFP4_ACT_DECAY_GATE: device FP32 [n_size], else unused */
+    const float* dt_bias;  /* NVFP4_ACT_DECAY_GATE: device FP32 [n_size], else unused */
+} nvfp4_segment_act;
 /* Bytes of the zero-initialised workspace nvfp4_global_scale needs. */
 #define NVFP4_GLOBAL_SCALE_WORKSPACE_BYTES 256
 
@@ -191,6 +208,27 @@ nvfp4_status nvfp4_fused_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const
                               const nvfp4_segment* segs, int nseg,
                               void* y, int64_t ldy, int64_t M, int64_t K,
                               void* stream);
+
+/* Fused multi-module GEMM with gate functions in the epilogue: as
+ * nvfp4_fused_gemm, then each output of segment i is replaced by
+ * f_i(fl32(acc * alpha_n)) evaluated in FP32 (expf, log1pf, IEEE division)
+ * and rounded once to BF16, f_i given by acts[i] (nvfp4_act_kind; NONE is the
+ * identity).  For the fused Gated DeltaNet input projection this yields the
+ * log-space decay gate g (segment a) and the write strength beta (segment b)
+ * directly, without a BF16 round trip of the raw gate projections.
+ *   acts (host, nseg entries, copied during the call) or NULL (all NONE).
+ *        A DECAY_GATE entry needs a_log and dt_bias (device, n_size FP32 each).
+ * Errors: as nvfp4_fused_gemm; NVFP4_ERR_INVALID_ARG for an unknown kind or a
+ * missing parameter array.
+ * Source: evolve.pub, Key claims under review, second bullet, and Report
+ * preview, Table 3 (log-space softplus/exponential and sigmoid gate
+ * parameterizations); the formulas are the Gated DeltaNet reading -- the
+ * pages give none. */
+nvfp4_status nvfp4_fused_gemm_act(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_g,
+                                  const uint8_t* w_codes, const uint8_t* w_sf,
+                                  const nvfp4_segment* segs, const nvfp4_segment_act* acts,
+                                  int nseg, void* y, int64_t ldy, int64_t M, int64_t K,
+                                  void* stream);
 
 /* Checkpoint-side repair of the global-scale mismatch: rewrite the block
  * scales of a fused weight so that ONE global scale serves all its modules.

@@ -26,6 +26,7 @@ from ._lib import SF_LINEAR, SF_TCGEN05, MAX_SEGMENTS, Nvfp4Error
 
 __all__ = [
     "SF_LINEAR", "SF_TCGEN05", "MAX_SEGMENTS", "Nvfp4Error", "QuantizedTensor",
+    "ACT_NONE", "ACT_DECAY_GATE", "ACT_SIGMOID",
     "global_scale", "sf_bytes", "quantize", "quantize_into", "quantize_tensor",
     "gemm", "fused_gemm", "FusedWeight", "linear", "silu_mul", "mlp", "harmonize", "kv_scale", "kv_quantize", "last_device_status",
     "debug_wait_timeout", "library_path",
@@ -208,23 +209,39 @@ def harmonize(w: "FusedWeight", layout: int = SF_TCGEN05, stream=None) -> Quanti
     return QuantizedTensor(w.codes, sf, g_c, w.rows, w.cols, layout)
 
 
+ACT_NONE, ACT_DECAY_GATE, ACT_SIGMOID = _lib.ACT_NONE, _lib.ACT_DECAY_GATE, _lib.ACT_SIGMOID
+
+
 def fused_gemm(a: QuantizedTensor, w_codes: torch.Tensor, w_sf: torch.Tensor,
-               segments: List, y: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
-    """Fused multi-module GEMM; segments = [(n_offset, n_size, g_tensor)]."""
+               segments: List, y: Optional[torch.Tensor] = None, stream=None,
+               acts: Optional[List] = None) -> torch.Tensor:
+    """Fused multi-module GEMM; segments = [(n_offset, n_size, g_tensor)].
+
+    acts (optional, one per segment): (kind, a_log, dt_bias) with kind one of
+    ACT_NONE, ACT_DECAY_GATE (a_log, dt_bias: FP32 device tensors of n_size),
+    ACT_SIGMOID -- the Gated DeltaNet gate functions applied in the epilogue."""
     if a.layout != SF_TCGEN05:
         raise ValueError("the GEMM reads block scales in the tensor-core layout")
     nseg = len(segments)
-    arr = (_lib.Segment * max(nseg, 1))()
-    for i, (off, n, g) in enumerate(segments):
-        arr[i].n_offset = int(off)
-        arr[i].n_size = int(n)
-        arr[i].w_gscale = g.data_ptr()
+    arr = _segment_array(segments)
     N = sum(int(s[1]) for s in segments)
     M, K = a.rows, a.cols
     if y is None:
         y = torch.empty(M, N, dtype=torch.bfloat16, device=a.codes.device)
-    _lib.check("nvfp4_fused_gemm", _lib.lib().nvfp4_fused_gemm(
-        _ptr(a.codes), _ptr(a.sf), _ptr(a.g), _ptr(w_codes), _ptr(w_sf), arr, nseg,
+    if acts is None:
+        _lib.check("nvfp4_fused_gemm", _lib.lib().nvfp4_fused_gemm(
+            _ptr(a.codes), _ptr(a.sf), _ptr(a.g), _ptr(w_codes), _ptr(w_sf), arr, nseg,
+            _ptr(y), y.stride(0), M, K, _stream(stream)))
+        return y
+    if len(acts) != nseg:
+        raise ValueError("one activation entry per segment")
+    act_arr = (_lib.SegmentAct * max(nseg, 1))()
+    for i, (kind, a_log, dt_bias) in enumerate(acts):
+        act_arr[i].kind = int(kind)
+        act_arr[i].a_log = 0 if a_log is None else a_log.data_ptr()
+        act_arr[i].dt_bias = 0 if dt_bias is None else dt_bias.data_ptr()
+    _lib.check("nvfp4_fused_gemm_act", _lib.lib().nvfp4_fused_gemm_act(
+        _ptr(a.codes), _ptr(a.sf), _ptr(a.g), _ptr(w_codes), _ptr(w_sf), arr, act_arr, nseg,
         _ptr(y), y.stride(0), M, K, _stream(stream)))
     return y
 

@@ -39,6 +39,12 @@ class Segment(ctypes.Structure):
                 ("w_gscale", ctypes.c_void_p)]
 
 
+class SegmentAct(ctypes.Structure):
+    _fields_ = [("kind", ctypes.c_int), ("a_log", ctypes.c_void_p), ("dt_bias", ctypes.c_void_p)]
+
+
+ACT_NONE, ACT_DECAY_GATE, ACT_SIGMOID = 0, 1, 2
+
 SIGNATURES = {
     "nvfp4_global_scale": (ST, [P, I64, I64, I64, P, P, P, P]),
     "nvfp4_global_scale_noalloc": (ST, [P, I64, I64, I64, P, P, P]),
@@ -47,6 +53,8 @@ SIGNATURES = {
     "nvfp4_quantize_slice": (ST, [P, I64, I64, I64, P, P, P, I32, I64, I64, P]),
     "nvfp4_gemm": (ST, [P, P, P, P, P, P, P, I64, I64, I64, I64, P]),
     "nvfp4_fused_gemm": (ST, [P, P, P, P, P, ctypes.POINTER(Segment), I32, P, I64, I64, I64, P]),
+    "nvfp4_fused_gemm_act": (ST, [P, P, P, P, P, ctypes.POINTER(Segment), ctypes.POINTER(SegmentAct),
+                                  I32, P, I64, I64, I64, P]),
     "nvfp4_silu_mul": (ST, [P, I64, I64, I64, P, I64, P]),
     "nvfp4_harmonize_scales": (ST, [P, I64, ctypes.POINTER(Segment), I32, I32, P, P]),
     "nvfp4_kv_scale_from_amax": (ST, [P, P, P]),

@@ -22,6 +22,8 @@
 //               tile's MMAs overlap the alpha scaling and the BF16 stores.
 // Every wait is bounded; a timeout sets the device status word and all roles
 // leave their loops, drain in-flight copies and free TMEM.
+#include <algorithm>
+
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -60,8 +62,22 @@ struct GemmArgs {
     int nseg;
     int seg_end[NVFP4_MAX_SEGMENTS];
     const float* seg_g[NVFP4_MAX_SEGMENTS];
+    int any_act;                                   // some segment has a gate function
+    int gate_lo, gate_hi;                          // hull of the gated segments' columns
+    int seg_kind[NVFP4_MAX_SEGMENTS];              // nvfp4_act_kind per segment
+    const float* seg_p0[NVFP4_MAX_SEGMENTS];       // decay gate: A_log per column
+    const float* seg_p1[NVFP4_MAX_SEGMENTS];       // decay gate: dt_bias per column
     uint64_t timeout_ns;
     int* status;
+};
+
+// Per-segment epilogue data, copied to shared memory at kernel start.
+struct SegTable {
+    float alpha[NVFP4_MAX_SEGMENTS];          // fl32(gA * gW[s])
+    int end[NVFP4_MAX_SEGMENTS];              // one past the segment's last column
+    int kind[NVFP4_MAX_SEGMENTS];             // nvfp4_act_kind
+    const float* p0[NVFP4_MAX_SEGMENTS];      // decay gate: A_log per column
+    const float* p1[NVFP4_MAX_SEGMENTS];      // decay gate: dt_bias per column
 };
 
 template <int BN>
@@ -85,9 +101,8 @@ struct Cfg {
     static constexpr int OFF_SFB = OFF_SFA + STAGES * SFA_BYTES;
     static constexpr int OFF_BAR = OFF_SFB + STAGES * SFB_BYTES;
     static constexpr int NBAR = 2 * STAGES + 2 * ACC + 1;
-    static constexpr int OFF_SEGA = OFF_BAR + NBAR * 8;
-    static constexpr int OFF_SEGE = OFF_SEGA + NVFP4_MAX_SEGMENTS * 4;
-    static constexpr int OFF_MISC = OFF_SEGE + NVFP4_MAX_SEGMENTS * 4;
+    static constexpr int OFF_SEG = OFF_BAR + NBAR * 8;
+    static constexpr int OFF_MISC = OFF_SEG + static_cast<int>((sizeof(SegTable) + 15) / 16 * 16);
     static constexpr int SMEM = OFF_MISC + 16 + 1024;  // + slack for 1024-byte alignment
     static constexpr int SFA_COL = ACC * BN;
     static constexpr int SFB_COL = SFA_COL + kAtomsPerStep * 4;
@@ -116,6 +131,49 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return l | (h << 16);
 }
 
+// Fill the table: thread t < NVFP4_MAX_SEGMENTS writes entry t.
+__device__ __forceinline__ void fill_seg_table(SegTable& T, const GemmArgs& a, int t) {
+    const bool in = t < a.nseg;
+    T.alpha[t] = in ? __fmul_rn(*a.a_g, *a.seg_g[t]) : 0.0f;
+    T.end[t] = in ? a.seg_end[t] : 0x7FFFFFFF;
+    T.kind[t] = in ? a.seg_kind[t] : NVFP4_ACT_NONE;
+    T.p0[t] = in ? a.seg_p0[t] : nullptr;
+    T.p1[t] = in ? a.seg_p1[t] : nullptr;
+}
+
+// Gated DeltaNet gate functions in FP32: the log-space decay gate
+// -exp(A_log) * softplus(v + dt_bias), softplus(z) = log(1 + e^z) written so
+// that neither branch overflows, and the sigmoid 1 / (1 + e^-v).
+__device__ __forceinline__ float gate_fn(float v, int kind, float a_log, float dt_bias) {
+    if (kind == NVFP4_ACT_DECAY_GATE) {
+        const float z = __fadd_rn(v, dt_bias);
+        const float sp = z > 0.0f ? __fadd_rn(z, log1pf(expf(-z))) : log1pf(expf(z));
+        return __fmul_rn(-expf(a_log), sp);
+    }
+    if (kind == NVFP4_ACT_SIGMOID) return __fdiv_rn(1.0f, __fadd_rn(1.0f, expf(-v)));
+    return v;
+}
+
+// Apply the segments' gate functions to CNT consecutive scaled outputs
+// starting at column n0 (columns at or beyond N are left alone).
+template <int CNT>
+__device__ __forceinline__ void apply_gates(float (&v)[CNT], int n0, int N, int nseg,
+                                            const SegTable& T) {
+    int s = 0;
+#pragma unroll
+    for (int j = 0; j < CNT; ++j) {
+        const int n = n0 + j;
+        while (s < nseg - 1 && n >= T.end[s]) ++s;
+        const int kind = T.kind[s];
+        if (n < N && kind != NVFP4_ACT_NONE) {
+            const int c = n - (s == 0 ? 0 : T.end[s - 1]);
+            const float al = kind == NVFP4_ACT_DECAY_GATE ? T.p0[s][c] : 0.0f;
+            const float db = kind == NVFP4_ACT_DECAY_GATE ? T.p1[s][c] : 0.0f;
+            v[j] = gate_fn(v[j], kind, al, db);
+        }
+    }
+}
+
 template <int BN, int STAGES, int ACC>
 __global__ void __launch_bounds__(kThreads, 1)
 nvf4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
@@ -130,8 +188,9 @@ nvf4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
     uint64_t* tmem_full = bars + 2 * STAGES;
     uint64_t* tmem_empty = bars + 2 * STAGES + ACC;
     uint64_t* drain = bars + 2 * STAGES + 2 * ACC;
-    float* s_seg_alpha = reinterpret_cast<float*>(smem + C::OFF_SEGA);
-    int* s_seg_end = reinterpret_cast<int*>(smem + C::OFF_SEGE);
+    SegTable& seg_tab = *reinterpret_cast<SegTable*>(smem + C::OFF_SEG);
+    const float* s_seg_alpha = seg_tab.alpha;
+    const int* s_seg_end = seg_tab.end;
     uint32_t* s_tmem_base = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
     volatile int* s_abort = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
 
@@ -158,11 +217,8 @@ nvf4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
         tmem_alloc(s_tmem_base, C::TMEM_COLS);
         tmem_relinquish();
     }
-    if (threadIdx.x >= 64 && threadIdx.x < 64 + NVFP4_MAX_SEGMENTS) {
-        const int s = threadIdx.x - 64;
-        s_seg_alpha[s] = (s < args.nseg) ? __fmul_rn(*args.a_g, *args.seg_g[s]) : 0.0f;
-        s_seg_end[s] = (s < args.nseg) ? args.seg_end[s] : 0x7FFFFFFF;
-    }
+    if (threadIdx.x >= 64 && threadIdx.x < 64 + NVFP4_MAX_SEGMENTS)
+        fill_seg_table(seg_tab, args, threadIdx.x - 64);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -333,6 +389,8 @@ nvf4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                             v[j] = __fmul_rn(__uint_as_float(r[ch][j]), s_seg_alpha[s]);
                         }
                     }
+                    if (args.any_act && n0 < args.gate_hi && n0 + 32 > args.gate_lo)
+                        apply_gates<32>(v, n0, args.N, args.nseg, seg_tab);
                     uint32_t o[16];
 #pragma unroll
                     for (int j = 0; j < 16; ++j) o[j] = pack_bf16x2(v[2 * j], v[2 * j + 1]);
@@ -397,9 +455,8 @@ struct PairCfg {
     static constexpr int OFF_SFB = OFF_SFA + STAGES * SFA_BYTES;
     static constexpr int OFF_BAR = OFF_SFB + STAGES * SFB_BYTES;
     static constexpr int NBAR = 3 * STAGES + 4;                  // full, empty, sf_ready, tmem_full, tmem_empty, drain x2
-    static constexpr int OFF_SEGA = OFF_BAR + NBAR * 8;
-    static constexpr int OFF_SEGE = OFF_SEGA + NVFP4_MAX_SEGMENTS * 4;
-    static constexpr int OFF_MISC = OFF_SEGE + NVFP4_MAX_SEGMENTS * 4;
+    static constexpr int OFF_SEG = OFF_BAR + NBAR * 8;
+    static constexpr int OFF_MISC = OFF_SEG + static_cast<int>((sizeof(SegTable) + 15) / 16 * 16);
     static constexpr int SMEM = OFF_MISC + 16 + 1024;
     static constexpr int SFA_COL = BN;                           // one accumulator of 256 columns
     static constexpr int SFB_COL = SFA_COL + kAtomsPerStep * 4;
@@ -434,8 +491,9 @@ nvf4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a,
     uint64_t* tmem_empty = bars + 3 * STAGES + 1;
     uint64_t* drain = bars + 3 * STAGES + 2;
     uint64_t* drain2 = bars + 3 * STAGES + 3;
-    float* s_seg_alpha = reinterpret_cast<float*>(smem + C::OFF_SEGA);
-    int* s_seg_end = reinterpret_cast<int*>(smem + C::OFF_SEGE);
+    SegTable& seg_tab = *reinterpret_cast<SegTable*>(smem + C::OFF_SEG);
+    const float* s_seg_alpha = seg_tab.alpha;
+    const int* s_seg_end = seg_tab.end;
     uint32_t* s_tmem_base = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
     volatile int* s_abort = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
 
@@ -467,11 +525,8 @@ nvf4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a,
         tmem_alloc_pair(s_tmem_base, C::TMEM_COLS);
         tmem_relinquish_pair();
     }
-    if (threadIdx.x >= 64 && threadIdx.x < 64 + NVFP4_MAX_SEGMENTS) {
-        const int s = threadIdx.x - 64;
-        s_seg_alpha[s] = (s < args.nseg) ? __fmul_rn(*args.a_g, *args.seg_g[s]) : 0.0f;
-        s_seg_end[s] = (s < args.nseg) ? args.seg_end[s] : 0x7FFFFFFF;
-    }
+    if (threadIdx.x >= 64 && threadIdx.x < 64 + NVFP4_MAX_SEGMENTS)
+        fill_seg_table(seg_tab, args, threadIdx.x - 64);
     tc_fence_before();
     __syncthreads();
     cluster_sync();                                      // barriers of both CTAs initialised
@@ -679,6 +734,8 @@ nvf4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a,
                             v[j] = __fmul_rn(__uint_as_float(r[ch][j]), s_seg_alpha[s]);
                         }
                     }
+                    if (args.any_act && n0 < args.gate_hi && n0 + 32 > args.gate_lo)
+                        apply_gates<32>(v, n0, args.N, args.nseg, seg_tab);
                     uint32_t o[16];
 #pragma unroll
                     for (int j = 0; j < 16; ++j) o[j] = pack_bf16x2(v[2 * j], v[2 * j + 1]);
@@ -924,8 +981,18 @@ nvfp4_status launch_gemm_decode(const uint8_t* a_codes, const uint8_t* w_codes,
 
 nvfp4_status gemm_impl(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_g,
                        const uint8_t* w_codes, const uint8_t* w_sf, const nvfp4_segment* segs,
-                       int nseg, void* y, int64_t ldy, int64_t M, int64_t K, void* stream) {
+                       const nvfp4_segment_act* acts, int nseg, void* y, int64_t ldy, int64_t M,
+                       int64_t K, void* stream) {
     if (!segs || nseg < 1 || nseg > NVFP4_MAX_SEGMENTS) return NVFP4_ERR_INVALID_ARG;
+    if (acts) {
+        for (int s = 0; s < nseg; ++s) {
+            const int k = acts[s].kind;
+            if (k != NVFP4_ACT_NONE && k != NVFP4_ACT_DECAY_GATE && k != NVFP4_ACT_SIGMOID)
+                return NVFP4_ERR_INVALID_ARG;
+            if (k == NVFP4_ACT_DECAY_GATE && (!acts[s].a_log || !acts[s].dt_bias))
+                return NVFP4_ERR_INVALID_ARG;
+        }
+    }
     if (M < 0 || K < 0 || !a_g) return NVFP4_ERR_INVALID_ARG;
     int64_t N = 0;
     for (int s = 0; s < nseg; ++s) {
@@ -965,9 +1032,20 @@ nvfp4_status gemm_impl(const uint8_t* a_codes, const uint8_t* a_sf, const float*
     // otherwise walk bands of 16 M tiles.
     args.group_m = (M * (K / 2) <= (int64_t(48) << 20)) ? 1 << 30 : 16;
     args.nseg = nseg;
+    args.any_act = 0;
+    args.gate_lo = 0x7FFFFFFF;
+    args.gate_hi = 0;
     for (int s = 0; s < nseg; ++s) {
         args.seg_end[s] = static_cast<int>(segs[s].n_offset + segs[s].n_size);
         args.seg_g[s] = segs[s].w_gscale;
+        args.seg_kind[s] = acts ? acts[s].kind : NVFP4_ACT_NONE;
+        args.seg_p0[s] = acts ? acts[s].a_log : nullptr;
+        args.seg_p1[s] = acts ? acts[s].dt_bias : nullptr;
+        if (args.seg_kind[s] != NVFP4_ACT_NONE) {
+            args.any_act = 1;
+            args.gate_lo = std::min(args.gate_lo, static_cast<int>(segs[s].n_offset));
+            args.gate_hi = std::max(args.gate_hi, static_cast<int>(segs[s].n_offset + segs[s].n_size));
+        }
     }
     args.timeout_ns = kTimeoutNs;
     args.status = status;
@@ -991,7 +1069,7 @@ extern "C" nvfp4_status nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_sf, 
     if (N < 0 || !w_g) return NVFP4_ERR_INVALID_ARG;
     if (N == 0) return (M >= 0 && K >= 0) ? NVFP4_OK : NVFP4_ERR_INVALID_ARG;
     nvfp4_segment seg = {0, N, w_g};
-    return gemm_impl(a_codes, a_sf, a_g, w_codes, w_sf, &seg, 1, y, ldy, M, K, stream);
+    return gemm_impl(a_codes, a_sf, a_g, w_codes, w_sf, &seg, nullptr, 1, y, ldy, M, K, stream);
 }
 
 extern "C" nvfp4_status nvfp4_fused_gemm(const uint8_t* a_codes, const uint8_t* a_sf,
@@ -999,7 +1077,15 @@ extern "C" nvfp4_status nvfp4_fused_gemm(const uint8_t* a_codes, const uint8_t* 
                                          const uint8_t* w_sf, const nvfp4_segment* segs, int nseg,
                                          void* y, int64_t ldy, int64_t M, int64_t K,
                                          void* stream) {
-    return gemm_impl(a_codes, a_sf, a_g, w_codes, w_sf, segs, nseg, y, ldy, M, K, stream);
+    return gemm_impl(a_codes, a_sf, a_g, w_codes, w_sf, segs, nullptr, nseg, y, ldy, M, K, stream);
+}
+
+extern "C" nvfp4_status nvfp4_fused_gemm_act(const uint8_t* a_codes, const uint8_t* a_sf,
+                                             const float* a_g, const uint8_t* w_codes,
+                                             const uint8_t* w_sf, const nvfp4_segment* segs,
+                                             const nvfp4_segment_act* acts, int nseg, void* y,
+                                             int64_t ldy, int64_t M, int64_t K, void* stream) {
+    return gemm_impl(a_codes, a_sf, a_g, w_codes, w_sf, segs, acts, nseg, y, ldy, M, K, stream);
 }
 
 extern "C" nvfp4_status nvfp4_last_device_status(void* stream) {

@@ -42,7 +42,7 @@ constexpr int kDecMaxSplit = 8;
 constexpr int kDecMaxStages = 8;
 constexpr int kDecMaxAcc = 4;
 constexpr int kDecMaxParts = 4;
-constexpr int kDecHeld = 4;           // reduced outputs a reducer holds before its stores
+constexpr int kDecHeld = 2;           // reduced outputs a reducer holds before its stores
 constexpr uint32_t kDecStageBudget = 210 * 1024;   // ring + partial buffers
 constexpr uint32_t kDecMinSmem = 116 * 1024;       // > half an SM: one CTA per SM
 
@@ -78,7 +78,7 @@ __host__ __device__ inline DecLayout dec_layout(int nt_tok, int stages, int npar
     // full, empty, sf_ready per stage; tmem_full, tmem_empty per accumulator;
     // part_full, part_free per partial buffer; drain
     L.off_seg = L.off_bar + (3 * stages + 2 * kDecMaxAcc + 2 * nparts + 1) * 8;
-    L.off_misc = L.off_seg + 2 * NVFP4_MAX_SEGMENTS * 4;
+    L.off_misc = L.off_seg + static_cast<uint32_t>((sizeof(SegTable) + 15) / 16 * 16);
     uint32_t bytes = L.off_misc + 16 + 1024;   // + slack for 1024-byte alignment
     L.bytes = bytes < kDecMinSmem ? kDecMinSmem : bytes;
     return L;
@@ -124,8 +124,9 @@ nvf4_gemm_decode_kernel(const __grid_constant__ CUtensorMap tmap_w,
     uint64_t* part_full = tmem_empty + kDecMaxAcc;    // [NPART]: partials of my rows landed
     uint64_t* part_free = part_full + NPART;          // [NPART]: every owner done with a buffer
     uint64_t* drain = part_free + NPART;
-    float* s_seg_alpha = reinterpret_cast<float*>(smem + L.off_seg);
-    int* s_seg_end = reinterpret_cast<int*>(smem + L.off_seg + NVFP4_MAX_SEGMENTS * 4);
+    SegTable& seg_tab = *reinterpret_cast<SegTable*>(smem + L.off_seg);
+    const float* s_seg_alpha = seg_tab.alpha;
+    const int* s_seg_end = seg_tab.end;
     uint32_t* s_tmem_base = reinterpret_cast<uint32_t*>(smem + L.off_misc);
     volatile int* s_abort = reinterpret_cast<volatile int*>(smem + L.off_misc + 4);
     float* part = reinterpret_cast<float*>(smem + L.off_part);   // [NPART][S][NT][128/S]
@@ -163,11 +164,8 @@ nvf4_gemm_decode_kernel(const __grid_constant__ CUtensorMap tmap_w,
         tmem_alloc(s_tmem_base, kDecTmemCols);
         tmem_relinquish();
     }
-    if (threadIdx.x >= 64 && threadIdx.x < 64 + NVFP4_MAX_SEGMENTS) {
-        const int s = threadIdx.x - 64;
-        s_seg_alpha[s] = (s < args.nseg) ? __fmul_rn(*args.a_g, *args.seg_g[s]) : 0.0f;
-        s_seg_end[s] = (s < args.nseg) ? args.seg_end[s] : 0x7FFFFFFF;
-    }
+    if (threadIdx.x >= 64 && threadIdx.x < 64 + NVFP4_MAX_SEGMENTS)
+        fill_seg_table(seg_tab, args, threadIdx.x - 64);
     tc_fence_before();
     __syncthreads();
     // the peers' barriers are initialised before anyone arrives on them remotely
@@ -435,8 +433,11 @@ nvf4_gemm_decode_kernel(const __grid_constant__ CUtensorMap tmap_w,
                         sum.w = __fadd_rn(sum.w, p[qq].w);
                     }
                 }
-                return make_uint2(pack_bf16x2(__fmul_rn(sum.x, al[0]), __fmul_rn(sum.y, al[1])),
-                                  pack_bf16x2(__fmul_rn(sum.z, al[2]), __fmul_rn(sum.w, al[3])));
+                float o4[4] = {__fmul_rn(sum.x, al[0]), __fmul_rn(sum.y, al[1]),
+                               __fmul_rn(sum.z, al[2]), __fmul_rn(sum.w, al[3])};
+                if (args.any_act && n0 < args.gate_hi && n0 + 4 > args.gate_lo)
+                    apply_gates<4>(o4, n0, args.N, args.nseg, seg_tab);
+                return make_uint2(pack_bf16x2(o4[0], o4[1]), pack_bf16x2(o4[2], o4[3]));
             };
             auto store_one = [&](int t, uint2 o) {
                 uint16_t* yp = args.y + static_cast<int64_t>(t) * args.ldy + n0;

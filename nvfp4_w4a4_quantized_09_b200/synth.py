@@ -21,6 +21,8 @@ max/RMS 63.5 and kurtosis ~1,564 -- evolve.pub review, Strengths, Table 2):
 """
 from __future__ import annotations
 
+import math
+
 import torch
 
 HIDDEN = 5120
@@ -88,6 +90,19 @@ def gdn_weights(modules=GDN_MODULES, cols: int = HIDDEN, first_seed: int = 10,
     """List of (name, BF16 [rows, cols]) per module, seeds first_seed, +1, ..."""
     return [(name, gaussian_weights(rows, cols, sigma, first_seed + i, device))
             for i, (name, rows, sigma) in enumerate(modules)]
+
+
+def gdn_gate_params(heads: int, seed: int = 40, device="cpu"):
+    """FP32 per-head decay-gate parameters (A_log, dt_bias) in the usual
+    Mamba-style initialisation: A ~ U(1, 16), A_log = log A; dt log-uniform in
+    [1e-3, 1e-1] and dt_bias the softplus preimage of dt.  Input generation
+    only -- seeded, float64 on the CPU, then cast."""
+    g = _gen(seed, "cpu")
+    a = 1.0 + 15.0 * torch.rand(heads, generator=g, dtype=torch.float64)
+    u = torch.rand(heads, generator=g, dtype=torch.float64)
+    dt = torch.exp(math.log(1e-3) + u * (math.log(1e-1) - math.log(1e-3)))
+    dt_bias = dt + torch.log(-torch.expm1(-dt))
+    return (torch.log(a).to(torch.float32).to(device), dt_bias.to(torch.float32).to(device))
 
 
 def random_bf16(rows: int, cols: int, seed: int, scale: float = 1.0, device="cpu"):

@@ -159,6 +159,26 @@ def test_kv_cache_entries_reject_bad_arguments(L):
     assert L.nvfp4_kv_scale_from_amax(FAKE, NUL, NUL) == _lib.NVFP4_ERR_INVALID_ARG
 
 
+def test_fused_gemm_act_validates_activations(L):
+    f = L.nvfp4_fused_gemm_act
+    args = (FAKE, FAKE, FAKE, FAKE, FAKE)
+    segs = seg_array([(0, 64, 0x10000), (64, 64, 0x10010)])
+
+    def acts(entries):
+        arr = (_lib.SegmentAct * len(entries))()
+        for i, (k, p0, p1) in enumerate(entries):
+            arr[i].kind, arr[i].a_log, arr[i].dt_bias = k, p0, p1
+        return arr
+    bad_kind = acts([(0, 0, 0), (3, 0, 0)])
+    assert f(*args, segs, bad_kind, 2, FAKE, 128, 4, 64, NUL) == _lib.NVFP4_ERR_INVALID_ARG
+    no_param = acts([(0, 0, 0), (_lib.ACT_DECAY_GATE, 0x10000, 0)])
+    assert f(*args, segs, no_param, 2, FAKE, 128, 4, 64, NUL) == _lib.NVFP4_ERR_INVALID_ARG
+    ok = acts([(_lib.ACT_SIGMOID, 0, 0), (_lib.ACT_DECAY_GATE, 0x10000, 0x10010)])
+    assert f(*args, segs, ok, 2, FAKE, 128, 0, 64, NUL) == _lib.NVFP4_OK          # M = 0
+    none = ctypes.cast(None, ctypes.POINTER(_lib.SegmentAct))
+    assert f(*args, segs, none, 2, FAKE, 128, 0, 64, NUL) == _lib.NVFP4_OK        # no table
+
+
 def test_debug_wait_rejects_bad_limits(L):
     assert L.nvfp4_debug_wait_timeout(0, NUL) == _lib.NVFP4_ERR_INVALID_ARG
     assert L.nvfp4_debug_wait_timeout(2_000_000_000, NUL) == _lib.NVFP4_ERR_INVALID_ARG
