@@ -130,13 +130,34 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------
+# ranks: one process per GPU, every rank its own batch (weak scaling)
+# ---------------------------------------------------------------------------
+def max_over_ranks(value: float, world: int, device) -> float:
+    """The largest per-rank value: the job's time is its slowest rank's."""
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world: int, flop_per_rank_step: float, steps: int, max_total_ms: float) -> float:
+    """Whole-job TFLOP/s: the work of all ranks over the slowest rank's time."""
+    return world * flop_per_rank_step * steps / (max_total_ms * 1e-3) / 1e12
+
+
+def rank_seed(rank: int) -> int:
+    """Activation seed of a rank: every rank draws its own batch."""
+    return 3 + 1000 * rank
+
+
+# ---------------------------------------------------------------------------
 # our arm
 # ---------------------------------------------------------------------------
 def build_workload(dev):
     import nvfp4_w4a4_quantized_09_b200 as nv
     from nvfp4_w4a4_quantized_09_b200 import synth
     rank = int(os.environ.get("RANK", "0"))
-    x = synth.student_t_activations(M_TOK, K_HID, seed=3 + 1000 * rank, device=dev)
+    x = synth.student_t_activations(M_TOK, K_HID, seed=rank_seed(rank), device=dev)
     ws = [w for _, w in synth.gdn_weights(synth.GDN_MODULES, device=dev)]
     fw = nv.FusedWeight.from_modules(ws)
     del ws
@@ -201,13 +222,9 @@ def run_ours(args, dev, world, rank):
     step_ms = [e0.elapsed_time(e2) for e0, _, e2 in ev]
     gemm_ms = [e1.elapsed_time(e2) for _, e1, e2 in ev]
     quant_ms = [e0.elapsed_time(e1) for e0, e1, _ in ev]
-    total_ms = float(sum(step_ms))
-    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    total_ms = float(t.item())
+    total_ms = max_over_ranks(float(sum(step_ms)), world, dev)
     ms_per_step = total_ms / args.steps
-    value = world * flops * args.steps / (total_ms * 1e-3) / 1e12
+    value = job_throughput(world, flops, args.steps, total_ms)
 
     gemm_avg_ms = float(np.mean(gemm_ms))
     achieved = flops / (gemm_avg_ms * 1e-3) / 1e12
