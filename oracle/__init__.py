@@ -97,6 +97,8 @@ def _L():
         lib.oracle_kv_quantize.restype = None
         lib.oracle_gdn_gates.argtypes = [P, I64, I64, I64, P, P, ctypes.c_int, P]
         lib.oracle_gdn_gates.restype = None
+        lib.oracle_silu_mul_f64.argtypes = [P, P, I64, I64, P]
+        lib.oracle_silu_mul_f64.restype = None
         _lib = lib
     return _lib
 
@@ -298,6 +300,17 @@ def gdn_gates(y64: np.ndarray, kind: int, a_log=None, dt_bias=None) -> np.ndarra
     out = np.empty((rows, ncols), np.uint16)
     _L().oracle_gdn_gates(_ptr(y), rows, ncols, ncols, _ptr(al), _ptr(db), int(kind), _ptr(out))
     return out
+
+
+def silu_mul_f64(gate64: np.ndarray, up64: np.ndarray) -> np.ndarray:
+    """h = bf16(SiLU(gate) * up) from FP64 gate and up [rows, f] (BF16 bits)."""
+    g = _c(gate64, np.float64)
+    u = _c(up64, np.float64)
+    assert g.shape == u.shape
+    rows, f = g.shape
+    h = np.empty((rows, f), np.uint16)
+    _L().oracle_silu_mul_f64(_ptr(g), _ptr(u), rows, f, _ptr(h))
+    return h
 
 
 def num_threads() -> int:

@@ -457,3 +457,20 @@ void oracle_gdn_gates(const double* y, int64_t rows, int64_t ncols, int64_t ld,
             out[r * ncols + c] = oracle_bf16_from_double(o);
         }
 }
+
+/* MLP intermediate straight from the gate_up GEMM: h = SiLU(gate) * up with
+ * gate and up the exact (FP64) GEMM values rather than their BF16 roundings,
+ * rounded once to BF16.  This is what a gate_up epilogue that computes h from
+ * its FP32 accumulators approximates (the fused form of the MLP companion
+ * above; W4A4 on every linear layer: chatpaper.ai abstract).  gate, up:
+ * [rows, f] row-major; h: BF16 bits [rows, f]. */
+void oracle_silu_mul_f64(const double* gate, const double* up, int64_t rows, int64_t f,
+                         uint16_t* h)
+{
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t c = 0; c < f; ++c) {
+            const double g = gate[r * f + c];
+            const double u = up[r * f + c];
+            h[r * f + c] = oracle_bf16_from_double(g / (1.0 + exp(-g)) * u);
+        }
+}

@@ -624,3 +624,24 @@ def test_gates_monotone_signs_and_tails():
                            np.zeros(2, np.float32), np.zeros(2, np.float32))[0]
     assert big[0] == oracle.bf16_from_double(np.array([-300.0]))[0]
     assert big[1] == oracle.bf16_from_double(np.array([-np.exp(-300.0)]))[0]
+
+
+def test_silu_mul_f64_agrees_with_bf16_input_form():
+    # on BF16-representable inputs it is the (pinned) BF16-input SiLU * up
+    rng = np.random.default_rng(21)
+    gb = oracle.bf16_from_double(rng.normal(0, 4, size=(32, 40)))
+    ub = oracle.bf16_from_double(rng.normal(0, 4, size=(32, 40)))
+    h1 = oracle.silu_mul_f64(oracle.bf16_bits_to_f64(gb), oracle.bf16_bits_to_f64(ub))
+    h2 = oracle.silu_mul(np.concatenate([gb, ub], axis=1))
+    assert np.array_equal(h1, h2)
+
+
+def test_silu_mul_f64_closed_forms():
+    g = np.array([[0.0, 50.0, -50.0, np.log(3.0)]])
+    u = np.array([[7.0, 2.0, 1.0, 4.0]])
+    h = oracle.bf16_bits_to_f64(oracle.silu_mul_f64(g, u))[0]
+    assert h[0] == 0.0                                        # SiLU(0) = 0
+    assert h[1] == 100.0                                      # SiLU(50) = 50 to 2^-72
+    assert h[2] == oracle.bf16_bits_to_f64(oracle.bf16_from_double(
+        np.array([-50.0 / (1.0 + np.exp(50.0))])))[0]
+    assert h[3] == oracle.bf16_bits_to_f64(oracle.bf16_from_double(np.array([np.log(3.0) * 0.75 * 4.0])))[0]
