@@ -230,6 +230,33 @@ nvfp4_status nvfp4_fused_gemm_act(const uint8_t* a_codes, const uint8_t* a_sf, c
                                   int nseg, void* y, int64_t ldy, int64_t M, int64_t K,
                                   void* stream);
 
+/* gate_up GEMM of a SiLU-gated MLP with the intermediate computed in its
+ * epilogue:  h[m, j] = BF16_RNE(fl32(SiLU(gate) * up)), gate = fl32(acc[m,
+ * gate row j] * alpha), up = fl32(acc[m, up row j] * alpha), alpha =
+ * fl32(*a_g * *w_g), SiLU evaluated as in nvfp4_silu_mul -- so no BF16
+ * [M, 2F] gate_up tensor is written or read -- plus the global scale of h
+ * for its W4A4 requantization:  *h_g = fl32(max|h| / 2688) (1 if h is all
+ * zero), what nvfp4_global_scale(h) returns, and *h_amax = max|h| (if
+ * non-null).
+ *   w_codes/w_sf: the [2F, K] gate_up weight (one global scale *w_g) with its
+ *     rows INTERLEAVED in 128-row blocks: block 2b = gate rows [128b, 128b+128),
+ *     block 2b+1 = the matching up rows.  Interleaving the BF16 rows before
+ *     quantizing changes neither the rows' codes nor the global scale.
+ *   h: device BF16 [M, F], row stride ldh elements.
+ *   workspace: as nvfp4_global_scale (NVFP4_GLOBAL_SCALE_WORKSPACE_BYTES,
+ *     zero-initialised, left zeroed); h_g, h_amax: device FP32.
+ * Requirements: M > 256 (the CTA-pair prefill kernel; smaller batches use
+ * nvfp4_gemm + nvfp4_silu_mul), F a multiple of 128, K as nvfp4_gemm,
+ * ldh >= F and a multiple of 8, pointers 16-byte aligned.
+ * Errors: NVFP4_ERR_INVALID_ARG, NVFP4_ERR_UNSUPPORTED_SHAPE,
+ * NVFP4_ERR_ALIGNMENT, CUDA errors.  Asynchronous on `stream`.
+ * Source: W4A4 on every linear layer, the MLP's included (chatpaper.ai
+ * abstract); the SiLU-gated MLP is the plain reading of the model's MLP. */
+nvfp4_status nvfp4_gemm_silu_mul(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_g,
+                                 const uint8_t* w_codes, const uint8_t* w_sf, const float* w_g,
+                                 void* h, int64_t ldh, int64_t M, int64_t F, int64_t K,
+                                 void* workspace, float* h_g, float* h_amax, void* stream);
+
 /* Checkpoint-side repair of the global-scale mismatch: rewrite the block
  * scales of a fused weight so that ONE global scale serves all its modules.
  *   g_c  = max_i *segs[i].w_gscale                 (written to *g_common)

@@ -28,7 +28,7 @@ __all__ = [
     "SF_LINEAR", "SF_TCGEN05", "MAX_SEGMENTS", "Nvfp4Error", "QuantizedTensor",
     "ACT_NONE", "ACT_DECAY_GATE", "ACT_SIGMOID",
     "global_scale", "sf_bytes", "quantize", "quantize_into", "quantize_tensor",
-    "gemm", "fused_gemm", "FusedWeight", "linear", "silu_mul", "mlp", "harmonize", "kv_scale", "kv_quantize", "last_device_status",
+    "gemm", "fused_gemm", "FusedWeight", "linear", "silu_mul", "mlp", "interleave_gate_up", "gemm_silu_mul", "harmonize", "kv_scale", "kv_quantize", "last_device_status",
     "debug_wait_timeout", "library_path",
 ]
 
@@ -266,6 +266,39 @@ def silu_mul(gate_up: torch.Tensor, h: Optional[torch.Tensor] = None, stream=Non
     _lib.check("nvfp4_silu_mul", _lib.lib().nvfp4_silu_mul(
         _ptr(gate_up), rows, f, gate_up.stride(0), _ptr(h), h.stride(0), _stream(stream)))
     return h
+
+
+def interleave_gate_up(w_gate_up: torch.Tensor, block: int = 128) -> torch.Tensor:
+    """Rows of a [2F, K] gate_up weight reordered into the 128-row-block
+    interleave nvfp4_gemm_silu_mul reads: gate block b, then up block b.
+    A row permutation of the BF16 weight before quantization (offline)."""
+    two_f = w_gate_up.shape[0]
+    f = two_f // 2
+    if two_f % 2 or f % block:
+        raise ValueError("gate_up rows must be 2F with F a multiple of 128")
+    g = w_gate_up[:f].reshape(f // block, block, -1)
+    u = w_gate_up[f:].reshape(f // block, block, -1)
+    return torch.stack([g, u], dim=1).reshape(two_f, -1).contiguous()
+
+
+def gemm_silu_mul(a: QuantizedTensor, w_interleaved: QuantizedTensor,
+                  h: Optional[torch.Tensor] = None, stream=None):
+    """h = SiLU(gate) * up straight from the gate_up GEMM's accumulators
+    (weight rows interleaved by interleave_gate_up), with the global scale of h
+    for its requantization.  Returns (h, g_h, amax_h)."""
+    if a.layout != SF_TCGEN05 or w_interleaved.layout != SF_TCGEN05:
+        raise ValueError("the GEMM reads block scales in the tensor-core layout")
+    M, K, F = a.rows, a.cols, w_interleaved.rows // 2
+    dev = a.codes.device
+    if h is None:
+        h = torch.empty(M, F, dtype=torch.bfloat16, device=dev)
+    g_h = torch.empty(1, dtype=torch.float32, device=dev)
+    amax_h = torch.empty(1, dtype=torch.float32, device=dev)
+    _lib.check("nvfp4_gemm_silu_mul", _lib.lib().nvfp4_gemm_silu_mul(
+        _ptr(a.codes), _ptr(a.sf), _ptr(a.g), _ptr(w_interleaved.codes), _ptr(w_interleaved.sf),
+        _ptr(w_interleaved.g), _ptr(h), h.stride(0), M, F, K, _ptr(_workspace(dev)), _ptr(g_h),
+        _ptr(amax_h), _stream(stream)))
+    return h, g_h, amax_h
 
 
 def mlp(x: torch.Tensor, w_gate_up, w_down, stream=None) -> torch.Tensor:

@@ -32,6 +32,7 @@
 #include "host_common.h"
 #include "nvfp4.h"
 #include "ptx.cuh"
+#include "silu.cuh"
 
 namespace nvfp4 {
 
@@ -64,6 +65,9 @@ struct GemmArgs {
     const float* seg_g[NVFP4_MAX_SEGMENTS];
     int any_act;                                   // some segment has a gate function
     int gate_lo, gate_hi;                          // hull of the gated segments' columns
+    unsigned int* h_ws;                            // SiLU epilogue: {amax bits, ticket}, zeroed
+    float* h_g;                                    // SiLU epilogue: fl32(amax(h) / 2688)
+    float* h_amax;                                 // SiLU epilogue: amax(h) (may be null)
     int seg_kind[NVFP4_MAX_SEGMENTS];              // nvfp4_act_kind per segment
     const float* seg_p0[NVFP4_MAX_SEGMENTS];       // decay gate: A_log per column
     const float* seg_p1[NVFP4_MAX_SEGMENTS];       // decay gate: dt_bias per column
@@ -472,7 +476,7 @@ __host__ __device__ constexpr uint32_t make_idesc_pair() {
            (static_cast<uint32_t>(256 >> 4) << 24);
 }
 
-template <int STAGES>
+template <int STAGES, bool kSilu>
 __global__ void __launch_bounds__(kPairThreads, 1)
 nvf4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a,
                       const __grid_constant__ CUtensorMap tmap_b,
@@ -688,6 +692,65 @@ nvf4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a,
         }
     } else {
         // ---------------- epilogue (warps 2..9, both CTAs) ----------------
+        if constexpr (kSilu) {
+            // The weight interleaves gate and up rows in 128-row blocks, so a
+            // 256-column tile holds gate columns [0, 128) and the matching up
+            // columns [128, 256).  Warp (q, half) writes h columns
+            // [64 half, 64 half + 64) of the tile's 128: h = bf16(SiLU(gate) *
+            // up) from the FP32 accumulators, and keeps the max |h| (as BF16
+            // magnitude bits) for the requantization's global scale.
+            const int q = warp & 3;
+            const int half = (warp - 2) >> 2;
+            const int row = q * 32 + lane;
+            const uint64_t pol_y = l2_policy_evict_first();
+            const float al = s_seg_alpha[0];
+            uint32_t mag = 0;
+            int i = 0;
+            for (int t = pair; t < total_tiles; t += npairs, ++i) {
+                int mt, nt;
+                tile_coords(t, args, mt, nt);
+                int ok = 1;
+                if (lane == 0)
+                    ok = mbar_wait_bounded(tmem_full, i & 1, args.timeout_ns, s_abort, args.status);
+                ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+                if (!ok) break;
+                tc_fence_after();
+                uint32_t r[4][32];
+                const uint32_t tq = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + half * 64;
+                tmem_ld_32cols(tq, r[0]);
+                tmem_ld_32cols(tq + 32, r[1]);
+                tmem_ld_32cols(tq + 128, r[2]);
+                tmem_ld_32cols(tq + 160, r[3]);
+                tmem_ld_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(tmem_empty_leader);
+                const int m = mt * 256 + static_cast<int>(rank) * 128 + row;
+                if (m < args.M) {
+                    uint16_t* hrow = args.y + static_cast<int64_t>(m) * args.ldy;
+#pragma unroll
+                    for (int ch = 0; ch < 2; ++ch) {
+                        const int j0 = nt * (BN / 2) + half * 64 + ch * 32;
+                        uint32_t o[16];
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            const uint32_t h0 = silu_mul1(__fmul_rn(__uint_as_float(r[ch][2 * j]), al),
+                                                          __fmul_rn(__uint_as_float(r[2 + ch][2 * j]), al));
+                            const uint32_t h1 = silu_mul1(__fmul_rn(__uint_as_float(r[ch][2 * j + 1]), al),
+                                                          __fmul_rn(__uint_as_float(r[2 + ch][2 * j + 1]), al));
+                            mag = max(mag, max(h0 & 0x7FFFu, h1 & 0x7FFFu));
+                            o[j] = h0 | (h1 << 16);
+                        }
+#pragma unroll
+                        for (int u = 0; u < 4; ++u)
+                            st_global_v4_hint(hrow + j0 + 8 * u, o[4 * u], o[4 * u + 1], o[4 * u + 2],
+                                              o[4 * u + 3], pol_y);
+                    }
+                }
+            }
+            mag = __reduce_max_sync(0xFFFFFFFFu, mag);
+            if (lane == 0 && mag) atomicMax(&args.h_ws[0], mag << 16);
+        } else {
         constexpr int kHalf = BN / 2;
         constexpr int kChunks = kHalf / 32;
         const int q = warp & 3;
@@ -753,12 +816,28 @@ nvf4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a,
                 }
             }
         }
+        }
     }
 
     tc_fence_before();
     __syncthreads();
     cluster_sync();                                      // no CTA leaves while its peer may signal it
     tc_fence_after();
+    if constexpr (kSilu) {
+        // the last CTA to finish turns the max |h| into the global scale of h
+        if (threadIdx.x == 0) {
+            __threadfence();
+            const unsigned int tk = atomicAdd(&args.h_ws[1], 1u);
+            if (tk == gridDim.x - 1) {
+                __threadfence();
+                const unsigned int bits = atomicExch(&args.h_ws[0], 0u);
+                const float amax = __uint_as_float(bits);
+                *args.h_g = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 2688.0f);
+                if (args.h_amax) *args.h_amax = amax;
+                atomicExch(&args.h_ws[1], 0u);
+            }
+        }
+    }
     if (warp == 1) {
         __syncwarp();
         tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
@@ -880,11 +959,11 @@ nvfp4_status launch_gemm(const uint8_t* a_codes, const uint8_t* w_codes, GemmArg
     return cuda_status(cudaGetLastError());
 }
 
-template <int STAGES>
+template <int STAGES, bool kSilu = false>
 nvfp4_status launch_gemm_pair(const uint8_t* a_codes, const uint8_t* w_codes, GemmArgs& args,
                               const DeviceInfo& dev, cudaStream_t stream) {
     using Cf = PairCfg<STAGES>;
-    auto kern = nvf4_gemm_pair_kernel<STAGES>;
+    auto kern = nvf4_gemm_pair_kernel<STAGES, kSilu>;
     static bool attr_set[64] = {false};
     int devid = 0;
     if (cudaGetDevice(&devid) != cudaSuccess || devid < 0 || devid >= 64) return NVFP4_ERR_CUDA;
@@ -1057,10 +1136,67 @@ nvfp4_status gemm_impl(const uint8_t* a_codes, const uint8_t* a_sf, const float*
     return launch_gemm<128, 6, 2>(a_codes, w_codes, args, dev, cs);
 }
 
+// gate_up GEMM with the SiLU(gate) * up epilogue and the global scale of h.
+nvfp4_status gemm_silu_impl(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_g,
+                            const uint8_t* w_codes, const uint8_t* w_sf, const float* w_g, void* h,
+                            int64_t ldh, int64_t M, int64_t F, int64_t K, void* workspace,
+                            float* h_g, float* h_amax, void* stream) {
+    if (M < 0 || F <= 0 || K < 0 || !a_g || !w_g || !h_g || !workspace) return NVFP4_ERR_INVALID_ARG;
+    if (F % 128 != 0 || K % 32 != 0 || K < 32) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (M >= (int64_t(1) << 31) || 2 * F >= (int64_t(1) << 31) || K >= (int64_t(1) << 31))
+        return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (ldh < F || ldh % 8 != 0) return NVFP4_ERR_ALIGNMENT;
+    if (M <= 256) return NVFP4_ERR_UNSUPPORTED_SHAPE;      // the CTA-pair (prefill) kernel only
+    if (!a_codes || !a_sf || !w_codes || !w_sf || !h) return NVFP4_ERR_INVALID_ARG;
+    if (!aligned16(a_codes) || !aligned16(a_sf) || !aligned16(w_codes) || !aligned16(w_sf) ||
+        !aligned16(h) || !aligned16(workspace))
+        return NVFP4_ERR_ALIGNMENT;
+    DeviceInfo dev;
+    nvfp4_status st = require_sm100(&dev);
+    if (st != NVFP4_OK) return st;
+    int* status = device_status_ptr();
+    if (!status) return NVFP4_ERR_CUDA;
+    const int64_t N = 2 * F;
+    GemmArgs args = {};
+    args.a_sf = a_sf;
+    args.w_sf = w_sf;
+    args.a_g = a_g;
+    args.y = static_cast<uint16_t*>(h);
+    args.ldy = ldh;
+    args.M = static_cast<int>(M);
+    args.N = static_cast<int>(N);
+    args.K = static_cast<int>(K);
+    args.k_steps = static_cast<int>((K + 255) / 256);
+    args.atoms_per_rb = static_cast<int>((K + 63) / 64);
+    args.w_rowblocks = static_cast<int>(N / 128);
+    args.group_m = (M * (K / 2) <= (int64_t(48) << 20)) ? 1 << 30 : 16;
+    args.nseg = 1;
+    args.seg_end[0] = static_cast<int>(N);
+    args.seg_g[0] = w_g;
+    args.seg_kind[0] = NVFP4_ACT_NONE;
+    args.gate_lo = 0x7FFFFFFF;
+    args.timeout_ns = kTimeoutNs;
+    args.status = status;
+    args.h_ws = static_cast<unsigned int*>(workspace);
+    args.h_g = h_g;
+    args.h_amax = h_amax;
+    return launch_gemm_pair<5, true>(a_codes, w_codes, args, dev, as_stream(stream));
+}
+
 }  // namespace
 }  // namespace nvfp4
 
 using namespace nvfp4;
+
+extern "C" nvfp4_status nvfp4_gemm_silu_mul(const uint8_t* a_codes, const uint8_t* a_sf,
+                                            const float* a_g, const uint8_t* w_codes,
+                                            const uint8_t* w_sf, const float* w_g, void* h,
+                                            int64_t ldh, int64_t M, int64_t F, int64_t K,
+                                            void* workspace, float* h_g, float* h_amax,
+                                            void* stream) {
+    return gemm_silu_impl(a_codes, a_sf, a_g, w_codes, w_sf, w_g, h, ldh, M, F, K, workspace, h_g,
+                          h_amax, stream);
+}
 
 extern "C" nvfp4_status nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_g,
                                    const uint8_t* w_codes, const uint8_t* w_sf, const float* w_g,

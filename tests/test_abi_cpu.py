@@ -179,6 +179,18 @@ def test_fused_gemm_act_validates_activations(L):
     assert f(*args, segs, none, 2, FAKE, 128, 0, 64, NUL) == _lib.NVFP4_OK        # no table
 
 
+def test_gemm_silu_mul_rejects_bad_arguments(L):
+    f = L.nvfp4_gemm_silu_mul
+    a = (FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE)          # a_codes .. w_g, h
+    assert f(*a, 256, 256, 256, 256, FAKE, FAKE, NUL, NUL) == _lib.NVFP4_ERR_UNSUPPORTED_SHAPE  # M <= 256
+    assert f(*a, 256, 300, 200, 256, FAKE, FAKE, NUL, NUL) == _lib.NVFP4_ERR_UNSUPPORTED_SHAPE  # F % 128
+    assert f(*a, 256, 300, 256, 100, FAKE, FAKE, NUL, NUL) == _lib.NVFP4_ERR_UNSUPPORTED_SHAPE  # K % 32
+    assert f(*a, 128, 300, 256, 256, FAKE, FAKE, NUL, NUL) == _lib.NVFP4_ERR_ALIGNMENT          # ldh < F
+    assert f(*a, 256, 300, 256, 256, NUL, FAKE, NUL, NUL) == _lib.NVFP4_ERR_INVALID_ARG         # workspace
+    assert f(*a, 256, 300, 256, 256, FAKE, NUL, NUL, NUL) == _lib.NVFP4_ERR_INVALID_ARG         # h_g
+    assert f(*a, 256, 300, 256, 256, ODD, FAKE, NUL, NUL) == _lib.NVFP4_ERR_ALIGNMENT
+
+
 def test_debug_wait_rejects_bad_limits(L):
     assert L.nvfp4_debug_wait_timeout(0, NUL) == _lib.NVFP4_ERR_INVALID_ARG
     assert L.nvfp4_debug_wait_timeout(2_000_000_000, NUL) == _lib.NVFP4_ERR_INVALID_ARG
