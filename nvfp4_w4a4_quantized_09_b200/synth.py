@@ -18,6 +18,8 @@ max/RMS 63.5 and kurtosis ~1,564 -- evolve.pub review, Strengths, Table 2):
 * weights: N(0, sigma) per module, cast to BF16.
 * the tiny case: X ~ N(0, 1) with 1 % of entries times 50, W ~ N(0, 0.02),
   both rounded once to BF16.
+* Gated DeltaNet decay-gate parameters per head: A ~ U(1, 16), A_log = log A;
+  dt log-uniform in [1e-3, 1e-1], dt_bias its softplus preimage (FP32).
 """
 from __future__ import annotations
 
