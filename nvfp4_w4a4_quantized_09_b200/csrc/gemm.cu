@@ -69,19 +69,25 @@ struct GemmArgs {
     float* h_g;                                    // SiLU epilogue: fl32(amax(h) / 2688)
     float* h_amax;                                 // SiLU epilogue: amax(h) (may be null)
     int seg_kind[NVFP4_MAX_SEGMENTS];              // nvfp4_act_kind per segment
+    int seg_goff[NVFP4_MAX_SEGMENTS];              // decay gate: offset in the staged parameters
     const float* seg_p0[NVFP4_MAX_SEGMENTS];       // decay gate: A_log per column
     const float* seg_p1[NVFP4_MAX_SEGMENTS];       // decay gate: dt_bias per column
     uint64_t timeout_ns;
     int* status;
 };
 
+// Decay-gate parameters staged in shared memory: at most this many columns
+// over all decay-gate segments (the GDN projection has one per head).
+constexpr int kMaxGateCols = 256;
+
 // Per-segment epilogue data, copied to shared memory at kernel start.
 struct SegTable {
     float alpha[NVFP4_MAX_SEGMENTS];          // fl32(gA * gW[s])
     int end[NVFP4_MAX_SEGMENTS];              // one past the segment's last column
     int kind[NVFP4_MAX_SEGMENTS];             // nvfp4_act_kind
-    const float* p0[NVFP4_MAX_SEGMENTS];      // decay gate: A_log per column
-    const float* p1[NVFP4_MAX_SEGMENTS];      // decay gate: dt_bias per column
+    int goff[NVFP4_MAX_SEGMENTS];             // decay gate: first index in gp0/gp1
+    float gp0[kMaxGateCols];                  // decay gate: A_log per column
+    float gp1[kMaxGateCols];                  // decay gate: dt_bias per column
 };
 
 template <int BN>
@@ -141,20 +147,33 @@ __device__ __forceinline__ void fill_seg_table(SegTable& T, const GemmArgs& a, i
     T.alpha[t] = in ? __fmul_rn(*a.a_g, *a.seg_g[t]) : 0.0f;
     T.end[t] = in ? a.seg_end[t] : 0x7FFFFFFF;
     T.kind[t] = in ? a.seg_kind[t] : NVFP4_ACT_NONE;
-    T.p0[t] = in ? a.seg_p0[t] : nullptr;
-    T.p1[t] = in ? a.seg_p1[t] : nullptr;
+    T.goff[t] = in ? a.seg_goff[t] : 0;
+}
+
+// Stage the decay-gate parameters (all threads of the CTA; before a barrier).
+__device__ __forceinline__ void stage_gate_params(SegTable& T, const GemmArgs& a) {
+    if (!a.any_act) return;
+    for (int s = 0; s < a.nseg; ++s) {
+        if (a.seg_kind[s] != NVFP4_ACT_DECAY_GATE) continue;
+        const int start = s == 0 ? 0 : a.seg_end[s - 1];
+        const int n = a.seg_end[s] - start;
+        for (int c = threadIdx.x; c < n; c += blockDim.x) {
+            T.gp0[a.seg_goff[s] + c] = a.seg_p0[s][c];
+            T.gp1[a.seg_goff[s] + c] = a.seg_p1[s][c];
+        }
+    }
 }
 
 // Gated DeltaNet gate functions in FP32: the log-space decay gate
-// -exp(A_log) * softplus(v + dt_bias), softplus(z) = log(1 + e^z) written so
-// that neither branch overflows, and the sigmoid 1 / (1 + e^-v).
+// -exp(A_log) * softplus(v + dt_bias), softplus(z) = max(z, 0) + log(1 +
+// e^-|z|) (no branch, no overflow), and the sigmoid 1 / (1 + e^-v).
 __device__ __forceinline__ float gate_fn(float v, int kind, float a_log, float dt_bias) {
     if (kind == NVFP4_ACT_DECAY_GATE) {
         const float z = __fadd_rn(v, dt_bias);
-        const float sp = z > 0.0f ? __fadd_rn(z, log1pf(expf(-z))) : log1pf(expf(z));
+        const float sp = __fadd_rn(fmaxf(z, 0.0f), log1pf(expf(-fabsf(z))));
         return __fmul_rn(-expf(a_log), sp);
     }
-    if (kind == NVFP4_ACT_SIGMOID) return __fdiv_rn(1.0f, __fadd_rn(1.0f, expf(-v)));
+    if (kind == NVFP4_ACT_SIGMOID) return __frcp_rn(__fadd_rn(1.0f, expf(-v)));
     return v;
 }
 
@@ -170,10 +189,9 @@ __device__ __forceinline__ void apply_gates(float (&v)[CNT], int n0, int N, int 
         while (s < nseg - 1 && n >= T.end[s]) ++s;
         const int kind = T.kind[s];
         if (n < N && kind != NVFP4_ACT_NONE) {
-            const int c = n - (s == 0 ? 0 : T.end[s - 1]);
-            const float al = kind == NVFP4_ACT_DECAY_GATE ? T.p0[s][c] : 0.0f;
-            const float db = kind == NVFP4_ACT_DECAY_GATE ? T.p1[s][c] : 0.0f;
-            v[j] = gate_fn(v[j], kind, al, db);
+            const int g = T.goff[s] + n - (s == 0 ? 0 : T.end[s - 1]);
+            const bool decay = kind == NVFP4_ACT_DECAY_GATE;
+            v[j] = gate_fn(v[j], kind, decay ? T.gp0[g] : 0.0f, decay ? T.gp1[g] : 0.0f);
         }
     }
 }
@@ -223,6 +241,7 @@ nvf4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
     }
     if (threadIdx.x >= 64 && threadIdx.x < 64 + NVFP4_MAX_SEGMENTS)
         fill_seg_table(seg_tab, args, threadIdx.x - 64);
+    stage_gate_params(seg_tab, args);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -531,6 +550,7 @@ nvf4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a,
     }
     if (threadIdx.x >= 64 && threadIdx.x < 64 + NVFP4_MAX_SEGMENTS)
         fill_seg_table(seg_tab, args, threadIdx.x - 64);
+    stage_gate_params(seg_tab, args);
     tc_fence_before();
     __syncthreads();
     cluster_sync();                                      // barriers of both CTAs initialised
@@ -725,26 +745,56 @@ nvf4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a,
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive_cluster(tmem_empty_leader);
+                // every lane computes (the votes below need the whole warp);
+                // only rows inside M store and count toward the max
                 const int m = mt * 256 + static_cast<int>(rank) * 128 + row;
-                if (m < args.M) {
-                    uint16_t* hrow = args.y + static_cast<int64_t>(m) * args.ldy;
+                const bool row_ok = m < args.M;
+                {
+                    uint16_t* hrow = args.y + static_cast<int64_t>(row_ok ? m : 0) * args.ldy;
 #pragma unroll
                     for (int ch = 0; ch < 2; ++ch) {
                         const int j0 = nt * (BN / 2) + half * 64 + ch * 32;
-                        uint32_t o[16];
+                        // branch-free FP32 for every element (fast division: within
+                        // 2 ulp, far inside the BF16 result's rounding); the rare
+                        // g < -80, where e^-g overflows, is redone in FP64 after a
+                        // vote.  Eight outputs per 16-byte store keep few values live.
 #pragma unroll
-                        for (int j = 0; j < 16; ++j) {
-                            const uint32_t h0 = silu_mul1(__fmul_rn(__uint_as_float(r[ch][2 * j]), al),
-                                                          __fmul_rn(__uint_as_float(r[2 + ch][2 * j]), al));
-                            const uint32_t h1 = silu_mul1(__fmul_rn(__uint_as_float(r[ch][2 * j + 1]), al),
-                                                          __fmul_rn(__uint_as_float(r[2 + ch][2 * j + 1]), al));
-                            mag = max(mag, max(h0 & 0x7FFFu, h1 & 0x7FFFu));
-                            o[j] = h0 | (h1 << 16);
+                        for (int q8 = 0; q8 < 4; ++q8) {
+                            uint32_t o[4];
+                            bool rare = false;
+#pragma unroll
+                            for (int jj = 0; jj < 4; ++jj) {
+                                const int j = 4 * q8 + jj;
+                                const float g0 = __fmul_rn(__uint_as_float(r[ch][2 * j]), al);
+                                const float g1 = __fmul_rn(__uint_as_float(r[ch][2 * j + 1]), al);
+                                const float u0 = __fmul_rn(__uint_as_float(r[2 + ch][2 * j]), al);
+                                const float u1 = __fmul_rn(__uint_as_float(r[2 + ch][2 * j + 1]), al);
+                                rare |= (g0 < -80.0f) | (g1 < -80.0f);
+                                const float s0 = __fdividef(g0, __fadd_rn(1.0f, expf(-g0)));
+                                const float s1 = __fdividef(g1, __fadd_rn(1.0f, expf(-g1)));
+                                o[jj] = pack_bf16x2(__fmul_rn(s0, u0), __fmul_rn(s1, u1));
+                            }
+                            if (__any_sync(0xFFFFFFFFu, rare)) {
+#pragma unroll
+                                for (int jj = 0; jj < 4; ++jj) {
+                                    const int j = 4 * q8 + jj;
+                                    const float g0 = __fmul_rn(__uint_as_float(r[ch][2 * j]), al);
+                                    const float g1 = __fmul_rn(__uint_as_float(r[ch][2 * j + 1]), al);
+                                    if (g0 < -80.0f)
+                                        o[jj] = (o[jj] & 0xFFFF0000u) |
+                                                silu_mul1(g0, __fmul_rn(__uint_as_float(r[2 + ch][2 * j]), al));
+                                    if (g1 < -80.0f)
+                                        o[jj] = (o[jj] & 0xFFFFu) |
+                                                (silu_mul1(g1, __fmul_rn(__uint_as_float(r[2 + ch][2 * j + 1]), al)) << 16);
+                                }
+                            }
+                            if (row_ok) {
+#pragma unroll
+                                for (int jj = 0; jj < 4; ++jj)
+                                    mag = max(mag, max(o[jj] & 0x7FFFu, (o[jj] >> 16) & 0x7FFFu));
+                                st_global_v4_hint(hrow + j0 + 8 * q8, o[0], o[1], o[2], o[3], pol_y);
+                            }
                         }
-#pragma unroll
-                        for (int u = 0; u < 4; ++u)
-                            st_global_v4_hint(hrow + j0 + 8 * u, o[4 * u], o[4 * u + 1], o[4 * u + 2],
-                                              o[4 * u + 3], pol_y);
                     }
                 }
             }
@@ -1114,7 +1164,10 @@ nvfp4_status gemm_impl(const uint8_t* a_codes, const uint8_t* a_sf, const float*
     args.any_act = 0;
     args.gate_lo = 0x7FFFFFFF;
     args.gate_hi = 0;
+    int gate_cols = 0;
     for (int s = 0; s < nseg; ++s) {
+        args.seg_goff[s] = gate_cols;
+        if (acts && acts[s].kind == NVFP4_ACT_DECAY_GATE) gate_cols += static_cast<int>(segs[s].n_size);
         args.seg_end[s] = static_cast<int>(segs[s].n_offset + segs[s].n_size);
         args.seg_g[s] = segs[s].w_gscale;
         args.seg_kind[s] = acts ? acts[s].kind : NVFP4_ACT_NONE;
@@ -1126,6 +1179,7 @@ nvfp4_status gemm_impl(const uint8_t* a_codes, const uint8_t* a_sf, const float*
             args.gate_hi = std::max(args.gate_hi, static_cast<int>(segs[s].n_offset + segs[s].n_size));
         }
     }
+    if (gate_cols > kMaxGateCols) return NVFP4_ERR_UNSUPPORTED_SHAPE;
     args.timeout_ns = kTimeoutNs;
     args.status = status;
     cudaStream_t cs = as_stream(stream);

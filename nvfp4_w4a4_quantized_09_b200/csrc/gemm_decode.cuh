@@ -166,6 +166,7 @@ nvf4_gemm_decode_kernel(const __grid_constant__ CUtensorMap tmap_w,
     }
     if (threadIdx.x >= 64 && threadIdx.x < 64 + NVFP4_MAX_SEGMENTS)
         fill_seg_table(seg_tab, args, threadIdx.x - 64);
+    stage_gate_params(seg_tab, args);
     tc_fence_before();
     __syncthreads();
     // the peers' barriers are initialised before anyone arrives on them remotely
