@@ -135,7 +135,7 @@ __device__ __forceinline__ bool elect_one() {
     return pred != 0;
 }
 
-// Bounded wait by the whole warp: lane 0 polls, the verdict is broadcast.
+// Bounded wait by the whole warp: lane 0 polls, the outcome is broadcast.
 __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, uint64_t limit_ns,
                                                volatile int* abort, int* dev_status) {
     int ok = 1;
