@@ -74,3 +74,41 @@ def dequant(codes, sf):
 
 def host_bits(t: torch.Tensor) -> np.ndarray:
     return bf16_bits(t)
+
+
+def assert_gates_match(y_gpu_bits, y64, S, K, kind, a_log=None, dt_bias=None, label=""):
+    """Gate outputs of one segment against the oracle's gate functions on the
+    FP64 GEMM values y64 [rows, n]; S = |alpha| sum_k |a_k w_k| per element.
+    Bound (derived in tests/test_gpu_gates.py): L (e_v + 2^-24 |y + b|) +
+    (2^-7 + 2^-18) |r| + 2^-126 with e_v = 2^-23 |y64| + K 2^-22 S and L the
+    gate's Lipschitz constant (e^A_log for the decay gate, 1/4 for the sigmoid).
+    Returns the fraction equal to the oracle's BF16 value."""
+    ref_bits = oracle.gdn_gates(y64, kind, a_log, dt_bias)
+    ref = oracle.bf16_bits_to_f64(ref_bits)
+    e_v = 2.0 ** -23 * np.abs(y64) + K * 2.0 ** -22 * S
+    if kind == oracle.GATE_DECAY:
+        lip = np.exp(np.asarray(a_log, np.float64))[None, :]
+        zabs = np.abs(y64 + np.asarray(dt_bias, np.float64)[None, :])
+    else:
+        lip, zabs = 0.25, np.abs(y64)
+    bound = lip * (e_v + 2.0 ** -24 * zabs) + (2.0 ** -7 + 2.0 ** -18) * np.abs(ref) + 2.0 ** -126
+    err = np.abs(oracle.bf16_bits_to_f64(y_gpu_bits) - ref)
+    assert np.all(err <= bound), f"{label}: worst ratio {float((err / bound).max()):.3g}"
+    return float((y_gpu_bits == ref_bits).mean())
+
+
+def assert_silu_matches(h_gpu_bits, g64, u64, Sg, Su, K, label=""):
+    """h = SiLU(gate) * up against the oracle on the FP64 GEMM values.
+    Bound (derived in tests/test_gpu_mlp_fused.py): 1.1 e_g |u| + |SiLU(g)| e_u
+    + 1.1 e_g e_u + (2^-7 + 2^-18) |h_ref| + 2^-126.  Returns the fraction equal
+    to the oracle's BF16 value."""
+    ref_bits = oracle.silu_mul_f64(g64, u64)
+    ref = oracle.bf16_bits_to_f64(ref_bits)
+    e_g = 2.0 ** -23 * np.abs(g64) + K * 2.0 ** -22 * Sg
+    e_u = 2.0 ** -23 * np.abs(u64) + K * 2.0 ** -22 * Su
+    silu = np.abs(g64 / (1.0 + np.exp(-g64)))
+    bound = (1.1 * e_g * np.abs(u64) + silu * e_u + 1.1 * e_g * e_u +
+             (2.0 ** -7 + 2.0 ** -18) * np.abs(ref) + 2.0 ** -126)
+    err = np.abs(oracle.bf16_bits_to_f64(h_gpu_bits) - ref)
+    assert np.all(err <= bound), f"{label}: worst ratio {float((err / bound).max()):.3g}"
+    return float((h_gpu_bits == ref_bits).mean())

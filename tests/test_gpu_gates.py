@@ -21,7 +21,7 @@ import torch
 import oracle
 import nvfp4_w4a4_quantized_09_b200 as nv
 from nvfp4_w4a4_quantized_09_b200 import synth
-from parity_helpers import dequant, host_bits, oracle_quant
+from parity_helpers import assert_gates_match, dequant, host_bits, oracle_quant
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -76,7 +76,6 @@ def test_gate_epilogue_matches_oracle(M, layout):
     alpha = oracle.segment_alpha(ga, segs)
     y64 = oracle.gemm_f64(A, W, alpha)
     S = (np.abs(A) @ np.abs(W).T) * np.abs(alpha)[None, :]
-    yg = oracle.bf16_bits_to_f64(host_bits(y_act))
     yp = host_bits(y_plain)
     exact = total = 0
     for (off, n, _), (kind, _, _), (a_log, dt_bias) in zip(segs, acts, params):
@@ -84,19 +83,10 @@ def test_gate_epilogue_matches_oracle(M, layout):
         if kind == nv.ACT_NONE:
             assert np.array_equal(host_bits(y_act)[:, cols], yp[:, cols]), "identity segment changed"
             continue
-        ref_bits = oracle.gdn_gates(y64[:, cols], kind, a_log, dt_bias)
-        ref = oracle.bf16_bits_to_f64(ref_bits)
-        e_v = 2.0 ** -23 * np.abs(y64[:, cols]) + K * 2.0 ** -22 * S[:, cols]
-        if kind == nv.ACT_DECAY_GATE:
-            lip = np.exp(a_log.astype(np.float64))[None, :]
-            zabs = np.abs(y64[:, cols] + dt_bias.astype(np.float64)[None, :])
-        else:
-            lip, zabs = 0.25, np.abs(y64[:, cols])
-        bound = lip * (e_v + 2.0 ** -24 * zabs) + (2.0 ** -7 + 2.0 ** -18) * np.abs(ref) + 2.0 ** -126
-        err = np.abs(yg[:, cols] - ref)
-        assert np.all(err <= bound), (layout, M, kind, float((err / bound).max()))
-        exact += int((host_bits(y_act)[:, cols] == ref_bits).sum())
-        total += ref.size
+        frac = assert_gates_match(host_bits(y_act)[:, cols], y64[:, cols], S[:, cols], K, kind,
+                                  a_log, dt_bias, label=f"{layout} M={M} kind={kind}")
+        exact += int(round(frac * M * n))
+        total += M * n
     print(f"{layout} M={M}: {exact}/{total} gate outputs equal the oracle's BF16 exactly")
     assert exact >= 0.9 * total
 

@@ -18,7 +18,7 @@ import torch
 import oracle
 import nvfp4_w4a4_quantized_09_b200 as nv
 from nvfp4_w4a4_quantized_09_b200 import synth
-from parity_helpers import dequant, host_bits, np_f32, oracle_quant
+from parity_helpers import assert_silu_matches, dequant, host_bits, np_f32, oracle_quant
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -44,18 +44,8 @@ def test_gemm_silu_mul_matches_oracle(M, F, K):
     alpha = oracle.segment_alpha(ga, [(0, 2 * F, gw)])
     y64 = oracle.gemm_f64(A, W, alpha)
     S = (np.abs(A) @ np.abs(W).T) * np.abs(alpha)[None, :]
-    g64, u64 = y64[:, :F], y64[:, F:]
-    ref_bits = oracle.silu_mul_f64(g64, u64)
-    ref = oracle.bf16_bits_to_f64(ref_bits)
-    e_g = 2.0 ** -23 * np.abs(g64) + K * 2.0 ** -22 * S[:, :F]
-    e_u = 2.0 ** -23 * np.abs(u64) + K * 2.0 ** -22 * S[:, F:]
-    silu = np.abs(g64 / (1.0 + np.exp(-g64)))
-    bound = (1.1 * e_g * np.abs(u64) + silu * e_u + 1.1 * e_g * e_u +
-             (2.0 ** -7 + 2.0 ** -18) * np.abs(ref) + 2.0 ** -126)
-    got = oracle.bf16_bits_to_f64(host_bits(h))
-    err = np.abs(got - ref)
-    assert np.all(err <= bound), float((err / bound).max())
-    exact = float((host_bits(h) == ref_bits).mean())
+    exact = assert_silu_matches(host_bits(h), y64[:, :F], y64[:, F:], S[:, :F], S[:, F:], K,
+                                label=f"M={M} F={F} K={K}")
     print(f"M={M} F={F} K={K}: {exact:.4f} of h equal the oracle's BF16 exactly")
     assert exact > 0.9
 

@@ -1,15 +1,18 @@
-"""Sensitivity of the GEMM parity check, on the CPU: the comparison the GPU
-tests use accepts the oracle's own BF16 result and rejects results carrying
-a plausible kernel mistake -- a wrong module scale, swapped nibbles, a scale
-row taken from the neighbouring row, a dropped k-block, a transposed operand
-tile.  Every mistake is planted in oracle-side data (no GPU involved)."""
+"""Sensitivity of the parity checks, on the CPU: the comparisons the GPU tests
+use accept the oracle's own BF16 result and reject results carrying a
+plausible kernel mistake -- for the GEMM a wrong module scale, swapped
+nibbles, a scale row taken from the neighbouring row, a dropped k-block, a
+transposed operand tile; for the gate and SiLU epilogues a dropped parameter,
+a sign error, a swapped operand or a small scale error.  Every mistake is
+planted in oracle-side data (no GPU involved)."""
 import numpy as np
 import pytest
 import torch
 
 import oracle
 from nvfp4_w4a4_quantized_09_b200 import synth
-from parity_helpers import assert_gemm_matches, dequant, host_bits, oracle_quant
+from parity_helpers import (assert_gates_match, assert_gemm_matches, assert_silu_matches, dequant,
+                            host_bits, oracle_quant)
 
 M, N, K = 24, 40, 256
 
@@ -66,3 +69,56 @@ def test_rejects_a_transposed_tile(case):
     W = case["W"].copy()
     W[:16, :16] = W[:16, :16].T.copy()              # a 16 x 16 operand tile transposed
     _fails(oracle.bf16_from_double(oracle.gemm_f64(case["A"], W, case["alpha"])), case)
+
+
+# ---------------------------------------------------------------------------
+# the derived tolerances of the gate epilogue and the fused SiLU epilogue
+# ---------------------------------------------------------------------------
+@pytest.fixture(scope="module")
+def gate_case():
+    Mg, Ng, Kg = 32, 64, 512
+    x = synth.student_t_activations(Mg, Kg, seed=81)
+    w = synth.gaussian_weights(Ng, Kg, 0.05, seed=82)
+    ca, sa, ga = oracle_quant(host_bits(x))
+    cw, sw, gw = oracle_quant(host_bits(w))
+    A, W = dequant(ca, sa), dequant(cw, sw)
+    alpha = oracle.segment_alpha(ga, [(0, Ng, gw)])
+    y64 = oracle.gemm_f64(A, W, alpha)
+    S = (np.abs(A) @ np.abs(W).T) * np.abs(alpha)[None, :]
+    a_log, dt_bias = (t.numpy() for t in synth.gdn_gate_params(Ng, seed=83))
+    return dict(y64=y64, S=S, K=Kg, a_log=a_log, dt_bias=dt_bias)
+
+
+def test_gate_bound_accepts_the_oracle_and_rejects_mistakes(gate_case):
+    c = gate_case
+    for kind in (oracle.GATE_DECAY, oracle.GATE_SIGMOID):
+        ok = oracle.gdn_gates(c["y64"], kind, c["a_log"], c["dt_bias"])
+        assert assert_gates_match(ok, c["y64"], c["S"], c["K"], kind, c["a_log"], c["dt_bias"]) == 1.0
+    bad = [
+        # decay gate without dt_bias
+        (oracle.GATE_DECAY, oracle.gdn_gates(c["y64"], oracle.GATE_DECAY, c["a_log"],
+                                             np.zeros_like(c["dt_bias"]))),
+        # decay gate without the exp(A_log) factor
+        (oracle.GATE_DECAY, oracle.gdn_gates(c["y64"], oracle.GATE_DECAY, np.zeros_like(c["a_log"]),
+                                             c["dt_bias"])),
+        # sigmoid of the negated value
+        (oracle.GATE_SIGMOID, oracle.gdn_gates(-c["y64"], oracle.GATE_SIGMOID)),
+        # gate computed from a value with a 1 % scale error (a wrong alpha)
+        (oracle.GATE_SIGMOID, oracle.gdn_gates(1.01 * c["y64"], oracle.GATE_SIGMOID)),
+    ]
+    for kind, bits in bad:
+        with pytest.raises(AssertionError):
+            assert_gates_match(bits, c["y64"], c["S"], c["K"], kind, c["a_log"], c["dt_bias"])
+
+
+def test_silu_bound_accepts_the_oracle_and_rejects_mistakes(gate_case):
+    c = gate_case
+    g64, u64 = c["y64"][:, :32], c["y64"][:, 32:]
+    Sg, Su = c["S"][:, :32], c["S"][:, 32:]
+    ok = oracle.silu_mul_f64(g64, u64)
+    assert assert_silu_matches(ok, g64, u64, Sg, Su, c["K"]) == 1.0
+    for bits in (oracle.silu_mul_f64(u64, g64),            # gate and up swapped
+                 oracle.bf16_from_double(g64 * u64),        # the SiLU dropped
+                 oracle.silu_mul_f64(g64, 1.02 * u64)):     # a 2 % scale error on up
+        with pytest.raises(AssertionError):
+            assert_silu_matches(bits, g64, u64, Sg, Su, c["K"])
