@@ -920,16 +920,18 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
+// Looked up once (a thread-safe local static); nullptr when the driver has no
+// such entry point, which every tensor-map builder below reports as an error.
 EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    if (!fn) {
+    static const EncodeTiledFn fn = []() -> EncodeTiledFn {
         void* p = nullptr;
         cudaDriverEntryPointQueryResult q;
         if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
                 cudaSuccess &&
             q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-    }
+            return reinterpret_cast<EncodeTiledFn>(p);
+        return nullptr;
+    }();
     return fn;
 }
 
@@ -971,15 +973,17 @@ bool make_sf_map(CUtensorMap* m, const uint8_t* base, int64_t rowblocks, int64_t
 }  // namespace
 
 int* device_status_ptr() {
-    static int* cache[64] = {nullptr};
+    static int* cache[kMaxDevices] = {nullptr};
+    static PerDeviceOnce once;
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-    if (!cache[dev]) {
+    if (current_device(&dev) != NVFP4_OK) return nullptr;
+    const nvfp4_status st = once.run(dev, [&] {
         void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return nullptr;
+        if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess || !p) return NVFP4_ERR_CUDA;
         cache[dev] = static_cast<int*>(p);
-    }
-    return cache[dev];
+        return NVFP4_OK;
+    });
+    return st == NVFP4_OK ? cache[dev] : nullptr;
 }
 
 namespace {
@@ -989,15 +993,15 @@ nvfp4_status launch_gemm(const uint8_t* a_codes, const uint8_t* w_codes, GemmArg
                          const DeviceInfo& dev, cudaStream_t stream) {
     using Cf = Cfg<BN, STAGES, ACC>;
     auto kern = nvf4_gemm_kernel<BN, STAGES, ACC>;
-    static bool attr_set[64] = {false};
+    static PerDeviceOnce attr_once;
     int devid = 0;
-    if (cudaGetDevice(&devid) != cudaSuccess || devid < 0 || devid >= 64) return NVFP4_ERR_CUDA;
-    if (!attr_set[devid]) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::SMEM) !=
-            cudaSuccess)
-            return NVFP4_ERR_CUDA;
-        attr_set[devid] = true;
-    }
+    nvfp4_status st = current_device(&devid);
+    if (st != NVFP4_OK) return st;
+    st = attr_once.run(devid, [&] {
+        return cuda_status(
+            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::SMEM));
+    });
+    if (st != NVFP4_OK) return st;
     CUtensorMap ta, tb;
     if (!make_code_map(&ta, a_codes, args.M, args.K / 2, kBM)) return NVFP4_ERR_CUDA;
     if (!make_code_map(&tb, w_codes, args.N, args.K / 2, BN)) return NVFP4_ERR_CUDA;
@@ -1014,15 +1018,15 @@ nvfp4_status launch_gemm_pair(const uint8_t* a_codes, const uint8_t* w_codes, Ge
                               const DeviceInfo& dev, cudaStream_t stream) {
     using Cf = PairCfg<STAGES>;
     auto kern = nvf4_gemm_pair_kernel<STAGES, kSilu>;
-    static bool attr_set[64] = {false};
+    static PerDeviceOnce attr_once;
     int devid = 0;
-    if (cudaGetDevice(&devid) != cudaSuccess || devid < 0 || devid >= 64) return NVFP4_ERR_CUDA;
-    if (!attr_set[devid]) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::SMEM) !=
-            cudaSuccess)
-            return NVFP4_ERR_CUDA;
-        attr_set[devid] = true;
-    }
+    nvfp4_status st = current_device(&devid);
+    if (st != NVFP4_OK) return st;
+    st = attr_once.run(devid, [&] {
+        return cuda_status(
+            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::SMEM));
+    });
+    if (st != NVFP4_OK) return st;
     CUtensorMap ta, tb, tsa, tsb;
     const int64_t a_rb = (args.M + 127) / 128, w_rb = (args.N + 127) / 128;
     if (!make_code_map(&ta, a_codes, args.M, args.K / 2, 128)) return NVFP4_ERR_CUDA;
@@ -1056,19 +1060,21 @@ nvfp4_status launch_gemm_pair(const uint8_t* a_codes, const uint8_t* w_codes, Ge
 nvfp4_status launch_gemm_decode(const uint8_t* a_codes, const uint8_t* w_codes,
                                 GemmArgs& args, cudaStream_t stream) {
     auto kern = nvf4_gemm_decode_kernel;
-    static bool attr_set[64] = {false};
-    static int max_clusters[64][kDecMaxSplit + 1][9];   // [device][split][nt_tok / 16]
+    static PerDeviceOnce attr_once;
+    // resident clusters per [device][split][nt_tok / 16], 0 until measured
+    static std::atomic<int> max_clusters[kMaxDevices][kDecMaxSplit + 1][9];
     int devid = 0;
-    if (cudaGetDevice(&devid) != cudaSuccess || devid < 0 || devid >= 64) return NVFP4_ERR_CUDA;
-    if (!attr_set[devid]) {
+    nvfp4_status st = current_device(&devid);
+    if (st != NVFP4_OK) return st;
+    st = attr_once.run(devid, [&] {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(kDecStageBudget + 4096)) != cudaSuccess)
+                                 static_cast<int>(kDecStageBudget + 4096)) != cudaSuccess ||
+            cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100) !=
+                cudaSuccess)
             return NVFP4_ERR_CUDA;
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100) !=
-            cudaSuccess)
-            return NVFP4_ERR_CUDA;
-        attr_set[devid] = true;
-    }
+        return NVFP4_OK;
+    });
+    if (st != NVFP4_OK) return st;
     DecodeArgs d;
     d.g = args;
     d.nt_tok = ((args.M + 15) / 16) * 16;
@@ -1091,13 +1097,14 @@ nvfp4_status launch_gemm_decode(const uint8_t* a_codes, const uint8_t* w_codes,
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     // persistent: as many clusters as can be resident at once
-    int& slots = max_clusters[devid][d.split][d.nt_tok / 16];
+    // (racing threads may both measure; they store the same value)
+    std::atomic<int>& cached = max_clusters[devid][d.split][d.nt_tok / 16];
+    int slots = cached.load(std::memory_order_relaxed);
     if (slots <= 0) {
         cfg.gridDim = dim3(static_cast<unsigned>(d.split), 1, 1);
-        int n = 0;
-        if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0)
+        if (cudaOccupancyMaxActiveClusters(&slots, kern, &cfg) != cudaSuccess || slots <= 0)
             return NVFP4_ERR_CUDA;
-        slots = n;
+        cached.store(slots, std::memory_order_relaxed);
     }
     const int clusters = d.g.n_tiles < slots ? d.g.n_tiles : slots;
     cfg.gridDim = dim3(static_cast<unsigned>(clusters * d.split), 1, 1);

@@ -5,9 +5,44 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+#include <mutex>
+
 #include "nvfp4.h"
 
 namespace nvfp4 {
+
+// Device ordinals the per-device caches below can hold.
+constexpr int kMaxDevices = 64;
+
+// Ordinal of the calling thread's current device, or NVFP4_ERR_CUDA when it
+// cannot be read or lies beyond the caches.
+inline nvfp4_status current_device(int* dev) {
+    if (cudaGetDevice(dev) != cudaSuccess || *dev < 0 || *dev >= kMaxDevices) return NVFP4_ERR_CUDA;
+    return NVFP4_OK;
+}
+
+// One-time, per-device set-up that several host threads may reach at once
+// (cached device properties, symbol addresses, kernel attributes).  The first
+// caller runs `init` under a lock; a success is published with release order,
+// so a later caller that sees it (acquire) also sees everything `init` wrote.
+// A failed `init` is not recorded and runs again on the next call.
+class PerDeviceOnce {
+  public:
+    template <class F>
+    nvfp4_status run(int dev, F&& init) {
+        if (done_[dev].load(std::memory_order_acquire)) return NVFP4_OK;
+        std::lock_guard<std::mutex> lock(mu_);
+        if (done_[dev].load(std::memory_order_relaxed)) return NVFP4_OK;
+        const nvfp4_status st = init();
+        if (st == NVFP4_OK) done_[dev].store(true, std::memory_order_release);
+        return st;
+    }
+
+  private:
+    std::atomic<bool> done_[kMaxDevices] = {};
+    std::mutex mu_;
+};
 
 inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 

@@ -389,18 +389,21 @@ __global__ void __launch_bounds__(kThreads, 4) quantize_kernel(QuantParams p) {
 // host side
 // ---------------------------------------------------------------------------
 nvfp4_status current_device_info(DeviceInfo* info) {
-    static DeviceInfo cache[64];
+    static DeviceInfo cache[kMaxDevices];
+    static PerDeviceOnce once;
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return NVFP4_ERR_CUDA;
-    if (dev < 0 || dev >= 64) return NVFP4_ERR_CUDA;
-    if (cache[dev].sms == 0) {
+    nvfp4_status st = current_device(&dev);
+    if (st != NVFP4_OK) return st;
+    st = once.run(dev, [&] {
         DeviceInfo d;
         if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
             cudaDeviceGetAttribute(&d.major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
             cudaDeviceGetAttribute(&d.minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
             return NVFP4_ERR_CUDA;
         cache[dev] = d;
-    }
+        return NVFP4_OK;
+    });
+    if (st != NVFP4_OK) return st;
     *info = cache[dev];
     return NVFP4_OK;
 }
@@ -418,14 +421,18 @@ using namespace nvfp4;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[NVFP4_NOALLOC_SCRATCH_BYTES];
 
 static nvfp4_status noalloc_scratch_ptr(void** out) {
-    static void* cache[64] = {nullptr};
+    static void* cache[kMaxDevices] = {nullptr};
+    static PerDeviceOnce once;
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return NVFP4_ERR_CUDA;
-    if (!cache[dev]) {
+    nvfp4_status st = current_device(&dev);
+    if (st != NVFP4_OK) return st;
+    st = once.run(dev, [&] {
         void* p = nullptr;
         if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return NVFP4_ERR_CUDA;
         cache[dev] = p;
-    }
+        return NVFP4_OK;
+    });
+    if (st != NVFP4_OK) return st;
     *out = cache[dev];
     return NVFP4_OK;
 }
