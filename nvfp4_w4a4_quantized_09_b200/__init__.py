@@ -16,6 +16,7 @@ per-module global scales must be honoured (chatpaper.ai abstract).
 from __future__ import annotations
 
 import ctypes
+import functools
 from dataclasses import dataclass
 from typing import List, Optional, Sequence
 
@@ -46,25 +47,89 @@ def _stream(stream=None):
     return ctypes.c_void_p(s.cuda_stream)
 
 
+# ---------------------------------------------------------------------------
+# argument checks: the C ABI checks sizes, alignment and strides it is given,
+# but it cannot see how large a caller's buffer is.  Every buffer is checked
+# here for dtype, shape (or size) and device before the library is called.
+# ---------------------------------------------------------------------------
+def _check_bf16_matrix(x: torch.Tensor, name: str):
+    if not isinstance(x, torch.Tensor) or x.dtype != torch.bfloat16 or x.dim() != 2:
+        raise ValueError(f"{name} must be a 2-D bfloat16 tensor")
+    if x.stride(1) != 1:
+        raise ValueError(f"{name} must have unit stride along its last dimension")
+
+
+def _check_out_matrix(t: torch.Tensor, name: str, dtype: torch.dtype, rows: int, cols: int):
+    """A row-major output [rows, cols] with unit column stride; its row stride
+    may be wider than cols (the library checks its alignment)."""
+    if not isinstance(t, torch.Tensor) or t.dtype != dtype:
+        raise ValueError(f"{name} must be a {dtype} tensor")
+    if t.shape != (rows, cols):
+        raise ValueError(f"{name} must have shape ({rows}, {cols}), got {tuple(t.shape)}")
+    if cols > 0 and (t.stride(1) != 1 or (rows > 1 and t.stride(0) < cols)):
+        raise ValueError(f"{name} must be row-major with unit stride along its last dimension")
+
+
+def _check_packed(t: torch.Tensor, name: str, shape=None, min_bytes: Optional[int] = None):
+    """A contiguous uint8 buffer: packed codes of the given shape, or flat
+    scale bytes of at least min_bytes."""
+    if not isinstance(t, torch.Tensor) or t.dtype != torch.uint8 or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous uint8 tensor")
+    if shape is not None and t.shape != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if min_bytes is not None and t.numel() < min_bytes:
+        raise ValueError(f"{name} holds {t.numel()} bytes, {min_bytes} needed")
+
+
+def _check_f32(t: torch.Tensor, name: str, numel: int = 1):
+    if not isinstance(t, torch.Tensor) or t.dtype != torch.float32 or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous float32 tensor")
+    if t.numel() < numel:
+        raise ValueError(f"{name} must hold at least {numel} element(s), got {t.numel()}")
+
+
+def _check_quantized(q: "QuantizedTensor", name: str):
+    if q.cols % 2:
+        raise ValueError(f"{name}.cols must be even")
+    _check_packed(q.codes, f"{name}.codes", shape=(q.rows, q.cols // 2))
+    _check_packed(q.sf, f"{name}.sf", min_bytes=_sf_bytes_cached(q.rows, q.cols, q.layout))
+    _check_f32(q.g, f"{name}.g")
+
+
+def _check_devices(**tensors) -> torch.device:
+    """All tensors on the current CUDA device (the library launches on the
+    current device's stream); returns that device."""
+    dev = None
+    for name, t in tensors.items():
+        if t is None:
+            continue
+        if not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor")
+        if dev is None:
+            dev = t.device
+        elif t.device != dev:
+            raise ValueError(f"{name} is on {t.device}, the other operands on {dev}")
+    if dev is not None and dev.index != torch.cuda.current_device():
+        raise ValueError(f"operands are on {dev} but the current device is cuda:"
+                         f"{torch.cuda.current_device()}; call torch.cuda.set_device first")
+    return dev
+
+
 _workspaces = {}
 
 
-def _workspace(device: torch.device) -> torch.Tensor:
-    """Zero-initialised global-scale workspace, one per device (left zeroed by
-    every call).  Callers on several streams pass their own."""
+def _workspace(device: torch.device, stream=None) -> torch.Tensor:
+    """Zero-initialised global-scale workspace, one per (device, stream): each
+    call leaves it zeroed again, and calls on one stream run in order, so
+    calls on different streams never share one."""
     idx = device.index if device.index is not None else torch.cuda.current_device()
-    ws = _workspaces.get(idx)
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    key = (idx, s.cuda_stream)
+    ws = _workspaces.get(key)
     if ws is None:
         ws = torch.zeros(_lib.GLOBAL_SCALE_WORKSPACE_BYTES, dtype=torch.uint8, device=device)
-        _workspaces[idx] = ws
+        _workspaces[key] = ws
     return ws
-
-
-def _check_bf16_matrix(x: torch.Tensor, name: str):
-    if x.dtype != torch.bfloat16 or x.dim() != 2 or not x.is_cuda:
-        raise ValueError(f"{name} must be a 2-D bfloat16 CUDA tensor")
-    if x.stride(1) != 1:
-        raise ValueError(f"{name} must have unit stride along its last dimension")
 
 
 def sf_bytes(rows: int, cols: int, layout: int = SF_TCGEN05) -> int:
@@ -73,15 +138,26 @@ def sf_bytes(rows: int, cols: int, layout: int = SF_TCGEN05) -> int:
     return int(n.value)
 
 
+@functools.lru_cache(maxsize=1024)
+def _sf_bytes_cached(rows: int, cols: int, layout: int) -> int:
+    return sf_bytes(rows, cols, layout)
+
+
 def global_scale(x: torch.Tensor, g_out: Optional[torch.Tensor] = None,
                  amax_out: Optional[torch.Tensor] = None,
                  workspace: Optional[torch.Tensor] = None, stream=None):
     """(g, amax) as 1-element FP32 device tensors: g = amax / (6 * 448)."""
     _check_bf16_matrix(x, "x")
-    dev = x.device
+    if g_out is not None:
+        _check_f32(g_out, "g_out")
+    if amax_out is not None:
+        _check_f32(amax_out, "amax_out")
+    if workspace is not None:
+        _check_packed(workspace, "workspace", min_bytes=_lib.GLOBAL_SCALE_WORKSPACE_BYTES)
+    dev = _check_devices(x=x, g_out=g_out, amax_out=amax_out, workspace=workspace)
     g_out = torch.empty(1, dtype=torch.float32, device=dev) if g_out is None else g_out
     amax_out = torch.empty(1, dtype=torch.float32, device=dev) if amax_out is None else amax_out
-    ws = _workspace(dev) if workspace is None else workspace
+    ws = _workspace(dev, stream) if workspace is None else workspace
     rows, cols = x.shape
     _lib.check("nvfp4_global_scale", _lib.lib().nvfp4_global_scale(
         _ptr(x), rows, cols, x.stride(0), _ptr(g_out), _ptr(amax_out), _ptr(ws), _stream(stream)))
@@ -105,8 +181,13 @@ def quantize(x: torch.Tensor, g: torch.Tensor, layout: int = SF_TCGEN05,
              stream=None):
     """Codes and block scales of x under the global scale g (device tensor)."""
     _check_bf16_matrix(x, "x")
+    _check_f32(g, "g")
     rows, cols = x.shape
-    dev = x.device
+    if codes is not None:
+        _check_packed(codes, "codes", shape=(rows, cols // 2))
+    if sf is not None:
+        _check_packed(sf, "sf", min_bytes=_sf_bytes_cached(rows, cols, layout))
+    dev = _check_devices(x=x, g=g, codes=codes, sf=sf)
     if codes is None:
         codes = torch.empty(rows, cols // 2, dtype=torch.uint8, device=dev)
     if sf is None:
@@ -120,7 +201,13 @@ def quantize_into(x: torch.Tensor, g: torch.Tensor, codes: torch.Tensor, sf: tor
                   row_offset: int, total_rows: int, layout: int = SF_TCGEN05, stream=None):
     """Quantize x as rows [row_offset, row_offset + rows) of a larger tensor."""
     _check_bf16_matrix(x, "x")
+    _check_f32(g, "g")
     rows, cols = x.shape
+    if row_offset < 0 or row_offset + rows > total_rows:
+        raise ValueError(f"rows [{row_offset}, {row_offset + rows}) outside [0, {total_rows})")
+    _check_packed(codes, "codes", shape=(total_rows, cols // 2))
+    _check_packed(sf, "sf", min_bytes=_sf_bytes_cached(total_rows, cols, layout))
+    _check_devices(x=x, g=g, codes=codes, sf=sf)
     _lib.check("nvfp4_quantize_slice", _lib.lib().nvfp4_quantize_slice(
         _ptr(x), rows, cols, x.stride(0), _ptr(g), _ptr(codes), _ptr(sf), layout,
         row_offset, total_rows, _stream(stream)))
@@ -141,8 +228,14 @@ def gemm(a: QuantizedTensor, w: QuantizedTensor, y: Optional[torch.Tensor] = Non
     if a.cols != w.cols:
         raise ValueError("inner dimensions differ")
     M, K, N = a.rows, a.cols, w.rows
+    _check_quantized(a, "a")
+    _check_quantized(w, "w")
+    if y is not None:
+        _check_out_matrix(y, "y", torch.bfloat16, M, N)
+    dev = _check_devices(a_codes=a.codes, a_sf=a.sf, a_g=a.g, w_codes=w.codes, w_sf=w.sf, w_g=w.g,
+                         y=y)
     if y is None:
-        y = torch.empty(M, N, dtype=torch.bfloat16, device=a.codes.device)
+        y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
     _lib.check("nvfp4_gemm", _lib.lib().nvfp4_gemm(
         _ptr(a.codes), _ptr(a.sf), _ptr(a.g), _ptr(w.codes), _ptr(w.sf), _ptr(w.g),
         _ptr(y), y.stride(0), M, N, K, _stream(stream)))
@@ -165,6 +258,8 @@ class FusedWeight:
     def from_modules(cls, weights: Sequence[torch.Tensor], stream=None) -> "FusedWeight":
         if not 1 <= len(weights) <= MAX_SEGMENTS:
             raise ValueError(f"1..{MAX_SEGMENTS} modules")
+        for i, w in enumerate(weights):
+            _check_bf16_matrix(w, f"weights[{i}]")
         cols = weights[0].shape[1]
         total = sum(w.shape[0] for w in weights)
         dev = weights[0].device
@@ -201,12 +296,31 @@ def harmonize(w: "FusedWeight", layout: int = SF_TCGEN05, stream=None) -> Quanti
     """Checkpoint-side repair of the global-scale mismatch: a copy of the
     fused weight's block scales re-expressed against g_c = max_i g_i (codes
     shared, not copied), served afterwards by the single-scale GEMM."""
-    sf = w.sf.clone()
-    g_c = torch.empty(1, dtype=torch.float32, device=w.sf.device)
+    _check_packed(w.sf, "w.sf", min_bytes=_sf_bytes_cached(w.rows, w.cols, layout))
     segs = w.segments()
+    _check_segments(segs, w.rows)
+    dev = _check_devices(w_sf=w.sf, **{f"g[{i}]": g for i, (_, _, g) in enumerate(segs)})
+    sf = w.sf.clone()
+    g_c = torch.empty(1, dtype=torch.float32, device=dev)
     _lib.check("nvfp4_harmonize_scales", _lib.lib().nvfp4_harmonize_scales(
         _ptr(sf), w.cols, _segment_array(segs), len(segs), layout, _ptr(g_c), _stream(stream)))
     return QuantizedTensor(w.codes, sf, g_c, w.rows, w.cols, layout)
+
+
+def _check_segments(segments, n_total: Optional[int] = None):
+    """Segments [(n_offset, n_size, g)] tile [0, N) in order, each g a float32
+    scalar tensor; returns N."""
+    if not 1 <= len(segments) <= MAX_SEGMENTS:
+        raise ValueError(f"1..{MAX_SEGMENTS} segments")
+    off = 0
+    for i, (o, n, g) in enumerate(segments):
+        if int(o) != off or int(n) <= 0:
+            raise ValueError(f"segment {i} = [{int(o)}, {int(o) + int(n)}) does not continue at {off}")
+        _check_f32(g, f"segments[{i}] global scale")
+        off += int(n)
+    if n_total is not None and off != n_total:
+        raise ValueError(f"segments cover {off} rows, the weight has {n_total}")
+    return off
 
 
 ACT_NONE, ACT_DECAY_GATE, ACT_SIGMOID = _lib.ACT_NONE, _lib.ACT_DECAY_GATE, _lib.ACT_SIGMOID
@@ -223,18 +337,34 @@ def fused_gemm(a: QuantizedTensor, w_codes: torch.Tensor, w_sf: torch.Tensor,
     if a.layout != SF_TCGEN05:
         raise ValueError("the GEMM reads block scales in the tensor-core layout")
     nseg = len(segments)
-    arr = _segment_array(segments)
-    N = sum(int(s[1]) for s in segments)
+    if acts is not None and len(acts) != nseg:
+        raise ValueError("one activation entry per segment")
+    N = _check_segments(segments)
     M, K = a.rows, a.cols
+    _check_quantized(a, "a")
+    _check_packed(w_codes, "w_codes", shape=(N, K // 2))
+    _check_packed(w_sf, "w_sf", min_bytes=_sf_bytes_cached(N, K, SF_TCGEN05))
+    if y is not None:
+        _check_out_matrix(y, "y", torch.bfloat16, M, N)
+    params = {}
+    if acts is not None:
+        for i, ((_, n, _), (kind, a_log, dt_bias)) in enumerate(zip(segments, acts)):
+            if int(kind) == ACT_DECAY_GATE:
+                if a_log is None or dt_bias is None:
+                    raise ValueError(f"segment {i}: the decay gate needs a_log and dt_bias")
+                _check_f32(a_log, f"acts[{i}].a_log", int(n))
+                _check_f32(dt_bias, f"acts[{i}].dt_bias", int(n))
+                params[f"acts[{i}].a_log"], params[f"acts[{i}].dt_bias"] = a_log, dt_bias
+    dev = _check_devices(a_codes=a.codes, a_sf=a.sf, a_g=a.g, w_codes=w_codes, w_sf=w_sf, y=y,
+                         **{f"segments[{i}] g": g for i, (_, _, g) in enumerate(segments)}, **params)
+    arr = _segment_array(segments)
     if y is None:
-        y = torch.empty(M, N, dtype=torch.bfloat16, device=a.codes.device)
+        y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
     if acts is None:
         _lib.check("nvfp4_fused_gemm", _lib.lib().nvfp4_fused_gemm(
             _ptr(a.codes), _ptr(a.sf), _ptr(a.g), _ptr(w_codes), _ptr(w_sf), arr, nseg,
             _ptr(y), y.stride(0), M, K, _stream(stream)))
         return y
-    if len(acts) != nseg:
-        raise ValueError("one activation entry per segment")
     act_arr = (_lib.SegmentAct * max(nseg, 1))()
     for i, (kind, a_log, dt_bias) in enumerate(acts):
         act_arr[i].kind = int(kind)
@@ -260,9 +390,14 @@ def silu_mul(gate_up: torch.Tensor, h: Optional[torch.Tensor] = None, stream=Non
     """h = SiLU(gate_up[:, :f]) * gate_up[:, f:] in BF16 (the MLP intermediate)."""
     _check_bf16_matrix(gate_up, "gate_up")
     rows, two_f = gate_up.shape
+    if two_f % 2:
+        raise ValueError("gate_up must have an even number of columns")
     f = two_f // 2
+    if h is not None:
+        _check_out_matrix(h, "h", torch.bfloat16, rows, f)
+    dev = _check_devices(gate_up=gate_up, h=h)
     if h is None:
-        h = torch.empty(rows, f, dtype=torch.bfloat16, device=gate_up.device)
+        h = torch.empty(rows, f, dtype=torch.bfloat16, device=dev)
     _lib.check("nvfp4_silu_mul", _lib.lib().nvfp4_silu_mul(
         _ptr(gate_up), rows, f, gate_up.stride(0), _ptr(h), h.stride(0), _stream(stream)))
     return h
@@ -288,16 +423,25 @@ def gemm_silu_mul(a: QuantizedTensor, w_interleaved: QuantizedTensor,
     for its requantization.  Returns (h, g_h, amax_h)."""
     if a.layout != SF_TCGEN05 or w_interleaved.layout != SF_TCGEN05:
         raise ValueError("the GEMM reads block scales in the tensor-core layout")
+    if a.cols != w_interleaved.cols:
+        raise ValueError("inner dimensions differ")
+    if w_interleaved.rows % 2:
+        raise ValueError("the gate_up weight must have 2F rows")
     M, K, F = a.rows, a.cols, w_interleaved.rows // 2
-    dev = a.codes.device
+    _check_quantized(a, "a")
+    _check_quantized(w_interleaved, "w_interleaved")
+    if h is not None:
+        _check_out_matrix(h, "h", torch.bfloat16, M, F)
+    dev = _check_devices(a_codes=a.codes, a_sf=a.sf, a_g=a.g, w_codes=w_interleaved.codes,
+                         w_sf=w_interleaved.sf, w_g=w_interleaved.g, h=h)
     if h is None:
         h = torch.empty(M, F, dtype=torch.bfloat16, device=dev)
     g_h = torch.empty(1, dtype=torch.float32, device=dev)
     amax_h = torch.empty(1, dtype=torch.float32, device=dev)
     _lib.check("nvfp4_gemm_silu_mul", _lib.lib().nvfp4_gemm_silu_mul(
         _ptr(a.codes), _ptr(a.sf), _ptr(a.g), _ptr(w_interleaved.codes), _ptr(w_interleaved.sf),
-        _ptr(w_interleaved.g), _ptr(h), h.stride(0), M, F, K, _ptr(_workspace(dev)), _ptr(g_h),
-        _ptr(amax_h), _stream(stream)))
+        _ptr(w_interleaved.g), _ptr(h), h.stride(0), M, F, K, _ptr(_workspace(dev, stream)),
+        _ptr(g_h), _ptr(amax_h), _stream(stream)))
     return h, g_h, amax_h
 
 
@@ -322,9 +466,13 @@ def kv_quantize(x: torch.Tensor, scale: torch.Tensor, out: Optional[torch.Tensor
                 stream=None) -> torch.Tensor:
     """Signed E4M3 bytes of x / scale (RNE, saturating at 448) as uint8 [rows, cols]."""
     _check_bf16_matrix(x, "x")
+    _check_f32(scale, "scale")
     rows, cols = x.shape
+    if out is not None:
+        _check_out_matrix(out, "out", torch.uint8, rows, cols)
+    dev = _check_devices(x=x, scale=scale, out=out)
     if out is None:
-        out = torch.empty(rows, cols, dtype=torch.uint8, device=x.device)
+        out = torch.empty(rows, cols, dtype=torch.uint8, device=dev)
     _lib.check("nvfp4_kv_quantize_e4m3", _lib.lib().nvfp4_kv_quantize_e4m3(
         _ptr(x), rows, cols, x.stride(0), _ptr(scale), _ptr(out), out.stride(0), _stream(stream)))
     return out
