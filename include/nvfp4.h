@@ -135,7 +135,8 @@ nvfp4_status nvfp4_global_scale_noalloc(const void* x, int64_t rows, int64_t col
 
 /* Bytes of the scale buffer for a [rows, cols] tensor in `layout`:
  * LINEAR rows * cols/16; TCGEN05 roundup(rows,128) * roundup(cols/16,4).
- * cols must be a multiple of 16. */
+ * cols must be a multiple of 16, and rows and cols below 2^31
+ * (NVFP4_ERR_UNSUPPORTED_SHAPE otherwise). */
 nvfp4_status nvfp4_sf_bytes(int64_t rows, int64_t cols, nvfp4_sf_layout layout,
                             size_t* bytes);
 

@@ -1134,12 +1134,14 @@ nvfp4_status gemm_impl(const uint8_t* a_codes, const uint8_t* a_sf, const float*
     for (int s = 0; s < nseg; ++s) {
         if (segs[s].n_offset != N || segs[s].n_size <= 0 || !segs[s].w_gscale)
             return NVFP4_ERR_INVALID_ARG;
-        N += segs[s].n_size;
+        if (segs[s].n_size >= (int64_t(1) << 31)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+        N += segs[s].n_size;   // at most 16 terms below 2^31: no overflow
     }
     if (K % 32 != 0 || K < 32) return NVFP4_ERR_UNSUPPORTED_SHAPE;
     if (M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31) || K >= (int64_t(1) << 31))
         return NVFP4_ERR_UNSUPPORTED_SHAPE;
     if (ldy < N || ldy % 8 != 0) return NVFP4_ERR_ALIGNMENT;
+    if (extent_too_large(M, ldy, 2)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
     if (M == 0) return NVFP4_OK;
     if (!a_codes || !a_sf || !w_codes || !w_sf || !y) return NVFP4_ERR_INVALID_ARG;
     if (!aligned16(a_codes) || !aligned16(a_sf) || !aligned16(w_codes) || !aligned16(w_sf) ||
@@ -1204,9 +1206,10 @@ nvfp4_status gemm_silu_impl(const uint8_t* a_codes, const uint8_t* a_sf, const f
                             float* h_g, float* h_amax, void* stream) {
     if (M < 0 || F <= 0 || K < 0 || !a_g || !w_g || !h_g || !workspace) return NVFP4_ERR_INVALID_ARG;
     if (F % 128 != 0 || K % 32 != 0 || K < 32) return NVFP4_ERR_UNSUPPORTED_SHAPE;
-    if (M >= (int64_t(1) << 31) || 2 * F >= (int64_t(1) << 31) || K >= (int64_t(1) << 31))
+    if (M >= (int64_t(1) << 31) || F >= (int64_t(1) << 30) || K >= (int64_t(1) << 31))
         return NVFP4_ERR_UNSUPPORTED_SHAPE;
     if (ldh < F || ldh % 8 != 0) return NVFP4_ERR_ALIGNMENT;
+    if (extent_too_large(M, ldh, 2)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
     if (M <= 256) return NVFP4_ERR_UNSUPPORTED_SHAPE;      // the CTA-pair (prefill) kernel only
     if (!a_codes || !a_sf || !w_codes || !w_sf || !h) return NVFP4_ERR_INVALID_ARG;
     if (!aligned16(a_codes) || !aligned16(a_sf) || !aligned16(w_codes) || !aligned16(w_sf) ||

@@ -50,6 +50,16 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 
 inline nvfp4_status cuda_status(cudaError_t e) { return e == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA; }
 
+// True when `rows` rows `ld` elements apart, of elem_bytes each, would span
+// more than 2^48 bytes -- more than any device address space.  Checked before
+// any stride or size arithmetic on caller values (rows, ld >= 0), so that
+// none of it can overflow int64.
+inline bool extent_too_large(int64_t rows, int64_t ld, int64_t elem_bytes) {
+    constexpr int64_t kMaxBytes = int64_t(1) << 48;
+    if (rows <= 0 || ld <= 0) return false;
+    return ld > kMaxBytes / elem_bytes || rows > kMaxBytes / (ld * elem_bytes);
+}
+
 // Multiprocessor count and compute capability of the current device, cached
 // per device ordinal.
 struct DeviceInfo {

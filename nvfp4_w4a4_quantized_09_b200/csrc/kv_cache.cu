@@ -161,6 +161,8 @@ extern "C" nvfp4_status nvfp4_kv_quantize_e4m3(const void* x, int64_t rows, int6
     if (cols % 8 != 0 || ld % 8 != 0 || ldo % 8 != 0) return NVFP4_ERR_ALIGNMENT;
     if (rows == 0 || cols == 0) return NVFP4_OK;
     if (!x || !out || ld < cols || ldo < cols) return NVFP4_ERR_INVALID_ARG;
+    if (extent_too_large(rows, ld, 2) || extent_too_large(rows, ldo, 1))
+        return NVFP4_ERR_UNSUPPORTED_SHAPE;
     if (!aligned16(x) || (reinterpret_cast<uintptr_t>(out) & 7u) != 0) return NVFP4_ERR_ALIGNMENT;
     if (cols / 8 >= (int64_t(1) << 31)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
     DeviceInfo dev;

@@ -63,7 +63,9 @@ extern "C" nvfp4_status nvfp4_silu_mul(const void* gate_up, int64_t rows, int64_
     if (f % 8 != 0 || ld % 8 != 0 || ldh % 8 != 0) return NVFP4_ERR_ALIGNMENT;
     if (rows == 0 || f == 0) return NVFP4_OK;
     if (!gate_up || !h) return NVFP4_ERR_INVALID_ARG;
-    if (ld < 2 * f || ldh < f) return NVFP4_ERR_INVALID_ARG;
+    if (extent_too_large(rows, ld, 2) || extent_too_large(rows, ldh, 2))
+        return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (f > ld / 2 || ldh < f) return NVFP4_ERR_INVALID_ARG;   // ld >= 2f, ld even
     if (!aligned16(gate_up) || !aligned16(h)) return NVFP4_ERR_ALIGNMENT;
     DeviceInfo dev;
     nvfp4_status st = current_device_info(&dev);

@@ -456,7 +456,9 @@ extern "C" nvfp4_status nvfp4_global_scale_noalloc(const void* x, int64_t rows, 
 extern "C" nvfp4_status nvfp4_sf_bytes(int64_t rows, int64_t cols, nvfp4_sf_layout layout,
                                        size_t* bytes) {
     if (!bytes || rows < 0 || cols < 0) return NVFP4_ERR_INVALID_ARG;
-    if (cols % 16 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    // both below 2^31, so the padded product below cannot overflow
+    if (cols % 16 != 0 || rows >= (int64_t(1) << 31) || cols >= (int64_t(1) << 31))
+        return NVFP4_ERR_UNSUPPORTED_SHAPE;
     const int64_t sfcols = cols / 16;
     if (layout == NVFP4_SF_LINEAR) {
         *bytes = static_cast<size_t>(rows * sfcols);
@@ -475,6 +477,7 @@ extern "C" nvfp4_status nvfp4_global_scale(const void* x, int64_t rows, int64_t 
     if (rows > 0 && cols > 0 && !x) return NVFP4_ERR_INVALID_ARG;
     if (cols % 8 != 0 || ld % 8 != 0) return NVFP4_ERR_ALIGNMENT;
     if (rows > 0 && ld < cols) return NVFP4_ERR_INVALID_ARG;
+    if (extent_too_large(rows, ld, 2)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
     if ((x && !aligned16(x)) || !aligned16(workspace)) return NVFP4_ERR_ALIGNMENT;
     DeviceInfo dev;
     nvfp4_status st = current_device_info(&dev);
@@ -497,7 +500,10 @@ nvfp4_status quantize_impl(const void* x, int64_t rows, int64_t cols, int64_t ld
                            int64_t row_offset, int64_t total_rows, void* stream) {
     if (rows < 0 || cols < 0 || !g || row_offset < 0 || total_rows < 0)
         return NVFP4_ERR_INVALID_ARG;
-    if (row_offset + rows > total_rows) return NVFP4_ERR_INVALID_ARG;
+    if (row_offset > total_rows || rows > total_rows - row_offset) return NVFP4_ERR_INVALID_ARG;
+    // bounds that keep every size product below inside int64
+    if (cols >= (int64_t(1) << 31) || total_rows >= (int64_t(1) << 40) || extent_too_large(rows, ld, 2))
+        return NVFP4_ERR_UNSUPPORTED_SHAPE;
     if (layout != NVFP4_SF_LINEAR && layout != NVFP4_SF_TCGEN05) return NVFP4_ERR_INVALID_ARG;
     if (cols % 32 != 0 || ld % 8 != 0) return NVFP4_ERR_ALIGNMENT;
     const bool last = (row_offset + rows == total_rows);

@@ -55,6 +55,10 @@ def test_sf_bytes(L):
     assert L.nvfp4_sf_bytes(10, 24, _lib.SF_LINEAR, ctypes.byref(n)) == _lib.NVFP4_ERR_UNSUPPORTED_SHAPE
     assert L.nvfp4_sf_bytes(-1, 32, _lib.SF_LINEAR, ctypes.byref(n)) == _lib.NVFP4_ERR_INVALID_ARG
     assert L.nvfp4_sf_bytes(1, 32, 7, ctypes.byref(n)) == _lib.NVFP4_ERR_INVALID_ARG
+    # sizes whose byte count would overflow are refused, not wrapped
+    assert L.nvfp4_sf_bytes(1 << 31, 32, _lib.SF_LINEAR, ctypes.byref(n)) == _lib.NVFP4_ERR_UNSUPPORTED_SHAPE
+    assert L.nvfp4_sf_bytes(1 << 40, 1 << 40, _lib.SF_TCGEN05, ctypes.byref(n)) == \
+        _lib.NVFP4_ERR_UNSUPPORTED_SHAPE
 
 
 FAKE = ctypes.c_void_p(0x10000)      # 16-byte aligned, never dereferenced
@@ -123,6 +127,9 @@ def test_fused_gemm_validates_segment_table(L):
     assert f(*args, noscale, 2, FAKE, 128, 4, 64, NUL) == _lib.NVFP4_ERR_INVALID_ARG
     assert f(*args, good, 2, FAKE, 120, 4, 64, NUL) == _lib.NVFP4_ERR_ALIGNMENT        # ldy < N
     assert f(*args, good, 2, FAKE, 128, 0, 64, NUL) == _lib.NVFP4_OK                   # M = 0
+    # segment sizes whose sum would overflow int64 are refused one by one
+    huge = seg_array([(0, 1 << 62, 0x10000), (1 << 62, 1 << 62, 0x10010)])
+    assert f(*args, huge, 2, FAKE, 1 << 62, 4, 64, NUL) == _lib.NVFP4_ERR_UNSUPPORTED_SHAPE
 
 
 def test_harmonize_rejects_bad_arguments(L):
@@ -138,6 +145,8 @@ def test_harmonize_rejects_bad_arguments(L):
     assert f(FAKE, 64, gap, 2, LIN, FAKE, NUL) == _lib.NVFP4_ERR_INVALID_ARG   # not contiguous
     noscale = seg_array([(0, 64, 0x10000), (64, 64, 0)])
     assert f(FAKE, 64, noscale, 2, LIN, FAKE, NUL) == _lib.NVFP4_ERR_INVALID_ARG
+    huge = seg_array([(0, 1 << 62, 0x10000), (1 << 62, 1 << 62, 0x10010)])
+    assert f(FAKE, 64, huge, 2, LIN, FAKE, NUL) == _lib.NVFP4_ERR_UNSUPPORTED_SHAPE
     assert f(FAKE, 24, good, 2, T, FAKE, NUL) == _lib.NVFP4_ERR_UNSUPPORTED_SHAPE   # K % 16
     assert f(FAKE, 0, good, 2, T, FAKE, NUL) == _lib.NVFP4_ERR_UNSUPPORTED_SHAPE
     assert f(ctypes.c_void_p(0x10008), 64, good, 2, T, FAKE, NUL) == _lib.NVFP4_ERR_ALIGNMENT
@@ -189,6 +198,37 @@ def test_gemm_silu_mul_rejects_bad_arguments(L):
     assert f(*a, 256, 300, 256, 256, NUL, FAKE, NUL, NUL) == _lib.NVFP4_ERR_INVALID_ARG         # workspace
     assert f(*a, 256, 300, 256, 256, FAKE, NUL, NUL, NUL) == _lib.NVFP4_ERR_INVALID_ARG         # h_g
     assert f(*a, 256, 300, 256, 256, ODD, FAKE, NUL, NUL) == _lib.NVFP4_ERR_ALIGNMENT
+
+
+def test_silu_mul_rejects_bad_arguments(L):
+    s = L.nvfp4_silu_mul
+    assert s(FAKE, -1, 64, 128, FAKE, 64, NUL) == _lib.NVFP4_ERR_INVALID_ARG
+    assert s(FAKE, 4, 60, 128, FAKE, 64, NUL) == _lib.NVFP4_ERR_ALIGNMENT      # f % 8
+    assert s(FAKE, 4, 64, 120, FAKE, 64, NUL) == _lib.NVFP4_ERR_INVALID_ARG    # ld < 2f
+    assert s(FAKE, 4, 64, 128, FAKE, 56, NUL) == _lib.NVFP4_ERR_INVALID_ARG    # ldh < f
+    assert s(NUL, 4, 64, 128, FAKE, 64, NUL) == _lib.NVFP4_ERR_INVALID_ARG
+    assert s(ODD, 4, 64, 128, FAKE, 64, NUL) == _lib.NVFP4_ERR_ALIGNMENT
+    assert s(FAKE, 0, 64, 128, FAKE, 64, NUL) == _lib.NVFP4_OK                 # nothing to do
+
+
+def test_extents_that_would_overflow_are_refused(L):
+    # sizes and strides whose byte products exceed any address space are
+    # refused before any size arithmetic, instead of wrapping around
+    big, wide = 1 << 30, 1 << 20
+    assert L.nvfp4_global_scale(FAKE, big, 64, wide, FAKE, NUL, FAKE, NUL) == \
+        _lib.NVFP4_ERR_UNSUPPORTED_SHAPE
+    assert L.nvfp4_quantize(FAKE, big, 64, wide, FAKE, FAKE, FAKE, 1, NUL) == \
+        _lib.NVFP4_ERR_UNSUPPORTED_SHAPE
+    assert L.nvfp4_quantize_slice(FAKE, 4, 64, 64, FAKE, FAKE, FAKE, 1, 1 << 62, 1 << 62, NUL) == \
+        _lib.NVFP4_ERR_INVALID_ARG                                              # offset + rows wraps
+    assert L.nvfp4_kv_quantize_e4m3(FAKE, big, 64, wide, FAKE, FAKE, 64, NUL) == \
+        _lib.NVFP4_ERR_UNSUPPORTED_SHAPE
+    assert L.nvfp4_silu_mul(FAKE, big, 64, wide, FAKE, 64, NUL) == _lib.NVFP4_ERR_UNSUPPORTED_SHAPE
+    assert L.nvfp4_silu_mul(FAKE, 1, 1 << 62, 128, FAKE, 64, NUL) == _lib.NVFP4_ERR_INVALID_ARG
+    ok = (FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE)
+    assert L.nvfp4_gemm(*ok, wide, big, 128, 64, NUL) == _lib.NVFP4_ERR_UNSUPPORTED_SHAPE
+    assert L.nvfp4_gemm_silu_mul(*ok, 1 << 62, 300, 1 << 62, 256, FAKE, FAKE, NUL, NUL) == \
+        _lib.NVFP4_ERR_UNSUPPORTED_SHAPE
 
 
 def test_debug_wait_rejects_bad_limits(L):
