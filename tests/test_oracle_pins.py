@@ -261,6 +261,49 @@ def test_block_scale_tracks_absmax_over_6():
     assert np.all(np.abs(dec[~normal] - target[~normal]) <= 2.0 ** -10 * (1 + 1e-6))
 
 
+# (block absmax, global scale as float32 bits): inputs near an E4M3 rounding
+# midpoint where fl32(fl32(ab / 6) / g) and the one-division alternative
+# fl32(ab / fl32(6 g)) round to different scale codes, in both directions
+BLOCK_SCALE_ORDER_CASES = [
+    (1.0078125, 0x3EA1E1E1), (1.0625, 0x3EAAAAAA), (1.0390625, 0x3EA6E6E6),
+    (1.1640625, 0x3EBAFAFA), (1.1640625, 0x3E3AFAFA), (1.3828125, 0x3E5E1E1D),
+    (1.328125, 0x3E1DAE61), (1.4375, 0x3E2AAAAB), (1.0546875, 0x3D555556),
+    (1.109375, 0x3D606523),
+]
+
+
+def test_block_scale_is_two_float32_divisions():
+    # the block scale takes the fixed sequence fl32(fl32(ab / 6) / g), then
+    # E4M3 RNE: evaluated here with numpy's IEEE float32 division and torch's
+    # float8_e4m3fn cast, on inputs where the order of the operations decides
+    # the code (the alternative order must give another code, or the case
+    # would prove nothing)
+    for ab, gbits in BLOCK_SCALE_ORDER_CASES:
+        g = np.array([gbits], np.uint32).view(np.float32)[0]
+        spec = f32(f32(f32(ab) / f32(6.0)) / g)
+        alt = f32(f32(ab) / f32(f32(6.0) * g))
+        e4 = [int(torch.tensor([v]).to(torch.float8_e4m3fn).view(torch.uint8)[0]) for v in (spec, alt)]
+        assert e4[0] != e4[1], (ab, hex(gbits))
+        x = np.zeros((1, 16), np.float32)
+        x[0, 0], x[0, 5] = ab, -ab / 2
+        _, sf = oracle.quantize(bf16_bits_of(x), float(g))
+        assert int(sf[0, 0]) == e4[0], (ab, hex(gbits))
+
+
+def test_element_code_is_a_true_division_at_ties():
+    # g = 1 and block absmax 11.25 give s8 = E4M3(1.875) = 0x3F and d = 1.875.
+    # 2.34375, 4.6875 and 9.375 are exactly 1.25 d, 2.5 d and 5 d: E2M1 ties
+    # that go to the even code (1.0, 2.0, 4.0).  1/1.875 is not a float32, so
+    # a reciprocal multiply would land just above each tie and round up.
+    x = np.zeros((1, 16), np.float32)
+    x[0, :6] = [11.25, 2.34375, 4.6875, 9.375, -2.34375, -4.6875]
+    codes, sf = oracle.quantize(bf16_bits_of(x), 1.0)
+    assert int(sf[0, 0]) == 0x3F
+    nib = [(int(b) >> (4 * h)) & 15 for b in codes[0] for h in (0, 1)]
+    assert nib[:6] == [0x7, 0x2, 0x4, 0x6, 0xA, 0xC]
+    assert nib[6:] == [0] * 10
+
+
 def test_dequantization_error_bound():
     # |x - xhat| <= half the E2M1 spacing at |x/d| times d (plus the FP32
     # rounding of x/d), or the clip error when |x/d| > 6.
@@ -542,6 +585,15 @@ def test_kv_quantize_golden(golden_dir):
         xv, sv, expect = line.split()[:3]
         got = oracle.kv_quantize(_bf16([[float(xv)]]), float(sv))[0, 0]
         assert got == int(expect, 16), line
+
+
+def test_kv_code_is_a_true_division_at_ties():
+    # s = 1.75: 2.734375, 3.171875 and 5.46875 are exactly 1.5625 s, 1.8125 s
+    # and 3.125 s, E4M3 ties that go to the even code (1.5 = 0x3C,
+    # 1.75 = 0x3E, 3.0 = 0x44); 1/1.75 is not a float32, so a reciprocal
+    # multiply would land just above each tie and round up to the odd code
+    got = oracle.kv_quantize(_bf16([[2.734375, 3.171875, 5.46875, -2.734375]]), 1.75)[0]
+    assert [int(v) for v in got] == [0x3C, 0x3E, 0x44, 0xBC]
 
 
 @pytest.mark.parametrize("s", [1.0, 0.37, 3.1e-3, 41.0])
