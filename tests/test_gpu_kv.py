@@ -35,6 +35,18 @@ def test_kv_every_bf16_value_bitexact(s):
     assert np.array_equal(np_u8(out), oracle.kv_quantize(host_bits(x), np.float32(s)))
 
 
+def test_kv_exact_ties_behind_an_inexact_reciprocal():
+    # s = 1.75: the quotients 1.5625, 1.8125 and 3.125 are exact E4M3 ties and
+    # 1/1.75 is not a float32; the even codes must come out
+    x = torch.tensor([[2.734375, 3.171875, 5.46875, -2.734375, 0, 0, 0, 0]],
+                     dtype=torch.bfloat16, device=DEV)
+    out = nv.kv_quantize(x, torch.tensor([1.75], dtype=torch.float32, device=DEV))
+    torch.cuda.synchronize()
+    want = oracle.kv_quantize(host_bits(x), np.float32(1.75))
+    assert [int(v) for v in want[0, :4]] == [0x3C, 0x3E, 0x44, 0xBC]
+    assert np.array_equal(np_u8(out), want)
+
+
 @pytest.mark.parametrize("rows,cols,ld,ldo", [(1, 8, 8, 8), (33, 136, 152, 144), (257, 1024, 1024, 1032),
                                                (4096, 2048, 2048, 2048)])
 def test_kv_shapes_calibrated_bitexact(rows, cols, ld, ldo):

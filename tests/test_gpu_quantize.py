@@ -104,6 +104,34 @@ def test_edge_values_under_given_global_scale(g):
     check_quant_bitexact(x, nv.SF_LINEAR, g_host=g)
 
 
+# (block absmax, global scale as float32 bits) next to an E4M3 midpoint, where
+# the order of the two float32 divisions of the block scale decides the code
+SCALE_ORDER_CASES = [
+    (1.0078125, 0x3EA1E1E1), (1.0625, 0x3EAAAAAA), (1.1640625, 0x3E3AFAFA),
+    (1.328125, 0x3E1DAE61), (1.4375, 0x3E2AAAAB), (1.0546875, 0x3D555556),
+]
+
+
+def test_exact_ties_behind_an_inexact_reciprocal():
+    # d = 1.875 (g = 1, block absmax 11.25): the quotients 1.25, 2.5 and 5 are
+    # exact E2M1 ties, and 1/1.875 is not a float32 -- the kernel's encoder
+    # must reach the even code exactly as a true division does
+    x = np.zeros((2, 32), np.float32)
+    x[0, :6] = [11.25, 2.34375, 4.6875, 9.375, -2.34375, -4.6875]
+    x[1, 16:22] = [-11.25, 4.6875, 2.34375, -9.375, 9.375, 2.34375]
+    xt = torch.from_numpy(x).to(torch.bfloat16).to(DEV)
+    check_quant_bitexact(xt, nv.SF_TCGEN05, g_host=1.0)
+    check_quant_bitexact(xt, nv.SF_LINEAR, g_host=1.0)
+
+
+@pytest.mark.parametrize("ab,gbits", SCALE_ORDER_CASES)
+def test_block_scale_division_order(ab, gbits):
+    g = float(np.array([gbits], np.uint32).view(np.float32)[0])
+    x = np.zeros((1, 32), np.float32)
+    x[0, 0], x[0, 7], x[0, 16] = ab, -ab / 2, -ab
+    check_quant_bitexact(torch.from_numpy(x).to(torch.bfloat16).to(DEV), nv.SF_LINEAR, g_host=g)
+
+
 def test_every_bf16_value_through_the_encoder():
     # all finite non-negative BF16 patterns and their negatives, 16 to a block,
     # under a few global scales: exercises every E2M1 rounding decision
