@@ -1068,7 +1068,7 @@ nvfp4_status launch_gemm_decode(const uint8_t* a_codes, const uint8_t* w_codes,
     if (st != NVFP4_OK) return st;
     st = attr_once.run(devid, [&] {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(kDecStageBudget + 4096)) != cudaSuccess ||
+                                 static_cast<int>(kDecSmemAttr)) != cudaSuccess ||
             cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100) !=
                 cudaSuccess)
             return NVFP4_ERR_CUDA;

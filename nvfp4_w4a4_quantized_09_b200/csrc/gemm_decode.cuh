@@ -45,6 +45,9 @@ constexpr int kDecMaxParts = 4;
 constexpr int kDecHeld = 2;           // reduced outputs a reducer holds before its stores
 constexpr uint32_t kDecStageBudget = 210 * 1024;   // ring + partial buffers
 constexpr uint32_t kDecMinSmem = 116 * 1024;       // > half an SM: one CTA per SM
+constexpr uint32_t kDecSmemAttr = kDecStageBudget + 4096;   // dynamic shared memory granted
+static_assert(2 * kDecMinSmem > 228 * 1024,
+              "two decode CTAs could share an SM (and its 512 TMEM columns)");
 
 struct DecodeArgs {
     GemmArgs g;
@@ -59,16 +62,16 @@ struct DecLayout {
     uint32_t off_w, off_x, off_sfw, off_sfx, off_part, off_bar, off_seg, off_misc, bytes;
 };
 
-__host__ __device__ inline uint32_t dec_stage_bytes(int nt_tok) {
+__host__ __device__ constexpr uint32_t dec_stage_bytes(int nt_tok) {
     return kBM * kBKBytes + nt_tok * kBKBytes + 2 * kAtomsPerStep * kAtom;
 }
 
-__host__ __device__ inline uint32_t dec_part_bytes(int nt_tok) {
+__host__ __device__ constexpr uint32_t dec_part_bytes(int nt_tok) {
     return static_cast<uint32_t>(nt_tok) * kBM * 4;
 }
 
-__host__ __device__ inline DecLayout dec_layout(int nt_tok, int stages, int nparts) {
-    DecLayout L;
+__host__ __device__ constexpr DecLayout dec_layout(int nt_tok, int stages, int nparts) {
+    DecLayout L{};
     L.off_w = 0;
     L.off_x = L.off_w + stages * kBM * kBKBytes;
     L.off_sfw = L.off_x + stages * nt_tok * kBKBytes;
@@ -85,7 +88,7 @@ __host__ __device__ inline DecLayout dec_layout(int nt_tok, int stages, int npar
 }
 
 // Accumulators, partial buffers and ring depth for a token width.
-__host__ __device__ inline void dec_config(int nt_tok, int* stages, int* nparts, int* nacc) {
+__host__ __device__ constexpr void dec_config(int nt_tok, int* stages, int* nparts, int* nacc) {
     const int np = nt_tok <= 32 ? 4 : (nt_tok <= 64 ? 2 : 1);
     int st = static_cast<int>((kDecStageBudget - np * dec_part_bytes(nt_tok)) / dec_stage_bytes(nt_tok));
     st = st > kDecMaxStages ? kDecMaxStages : st;
@@ -93,6 +96,31 @@ __host__ __device__ inline void dec_config(int nt_tok, int* stages, int* nparts,
     *nparts = np;
     *nacc = nt_tok <= 64 ? 4 : 2;
 }
+
+// Every configuration the launcher can pick (token widths 16..128) fits the
+// hardware: ring and partial buffers within the shared memory the kernel is
+// granted (and the 227 KB a CTA may have), 2..8 stages, the scale slots of
+// all stages within the 512 TMEM columns, each accumulator's NT columns
+// within its share of columns 0..255, and the operand tiles on the 1024-byte
+// boundaries their 128-byte swizzle needs (scales and partials on 16 bytes,
+// barriers on 8, the segment table and the two status words, all read as
+// 4-byte scalars, on 4).
+constexpr bool dec_configs_fit() {
+    for (int nt = 16; nt <= 128; nt += 16) {
+        int st = 0, np = 0, na = 0;
+        dec_config(nt, &st, &np, &na);
+        const DecLayout L = dec_layout(nt, st, np);
+        if (L.bytes > kDecSmemAttr || L.bytes > 227 * 1024) return false;
+        if (st < 2 || st > kDecMaxStages || np < 1 || np > kDecMaxParts || na < 1 || na > kDecMaxAcc)
+            return false;
+        if (kDecSfCol + st * kDecSfSlot > kDecTmemCols || nt > 256 / na) return false;
+        if (L.off_x % 1024 != 0 || L.off_sfw % 16 != 0 || L.off_sfx % 16 != 0 ||
+            L.off_part % 16 != 0 || L.off_bar % 8 != 0 || L.off_seg % 4 != 0 || L.off_misc % 4 != 0)
+            return false;
+    }
+    return true;
+}
+static_assert(dec_configs_fit(), "a decode configuration exceeds a hardware limit");
 
 __device__ __forceinline__ uint32_t make_idesc_dec(int nt_tok) {
     return (1u << 7) | (1u << 10) | (static_cast<uint32_t>(nt_tok >> 3) << 17) |
