@@ -121,6 +121,9 @@ struct Cfg {
                                    : COLS_USED <= 128 ? 128 : COLS_USED <= 256 ? 256 : 512;
     static_assert(COLS_USED <= 512, "tensor memory overflow");
     static_assert(SMEM <= 232448, "shared memory overflow");
+    // a CTA that takes more than half the TMEM must also take more than half
+    // the shared memory, so that no second CTA on its SM waits in the allocator
+    static_assert(TMEM_COLS <= 256 || SMEM > 228 * 1024 / 2, "two CTAs per SM would share TMEM");
     static_assert(BN % 128 == 0 && BN <= 256, "BN must be 128 or 256");
 };
 
@@ -487,6 +490,7 @@ struct PairCfg {
     static constexpr int TMEM_COLS = 512;
     static_assert(BN + STAGES * SF_STRIDE <= TMEM_COLS, "tensor memory overflow");
     static_assert(SMEM <= 232448, "shared memory overflow");
+    static_assert(SMEM > 228 * 1024 / 2, "two CTAs per SM would share TMEM");
 };
 
 // kind::mxf4nvf4 descriptor for the pair MMA: M = 256, N = 256.
