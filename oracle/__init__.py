@@ -87,6 +87,8 @@ def _L():
         lib.oracle_e4m3_encode_array.argtypes = [P, I64, P]
         lib.oracle_bf16_from_double_array.argtypes = [P, I64, P]
         lib.oracle_num_threads.restype = ctypes.c_int
+        lib.oracle_set_num_threads.argtypes = [ctypes.c_int]
+        lib.oracle_set_num_threads.restype = None
         lib.oracle_silu_mul.argtypes = [P, I64, I64, I64, P]
         lib.oracle_silu_mul.restype = None
         lib.oracle_harmonize_scales.argtypes = [P, I64, I64, P, P, ctypes.c_int, P]
@@ -315,3 +317,9 @@ def silu_mul_f64(gate64: np.ndarray, up64: np.ndarray) -> np.ndarray:
 
 def num_threads() -> int:
     return int(_L().oracle_num_threads())
+
+
+def set_num_threads(n: int) -> None:
+    """Threads the oracle's parallel loops use from now on (timing only: each
+    output is computed by one thread in k order, so results do not change)."""
+    _L().oracle_set_num_threads(int(n))

@@ -316,6 +316,18 @@ void oracle_bf16_from_double_array(const double* x, int64_t n, uint16_t* out)
     for (int64_t i = 0; i < n; ++i) out[i] = oracle_bf16_from_double(x[i]);
 }
 
+/* Threads the parallel loops above use from now on (n >= 1); lets a caller
+ * time the oracle on one core as well as on all of them.  No arithmetic
+ * depends on it: each output is computed by one thread in k order. */
+void oracle_set_num_threads(int n)
+{
+#ifdef _OPENMP
+    if (n >= 1) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}
+
 int oracle_num_threads(void)
 {
 #ifdef _OPENMP
