@@ -51,6 +51,8 @@ def test_tiny_config_full():
     (130, 136, 96),      # K % 64 == 32, ragged everything
     (512, 1024, 1024),   # several full tiles each way
     (257, 264, 5120),    # long K
+    (300, 136, 160),     # large-M configuration, K % 64 == 32 (half an MMA in the last step)
+    (513, 392, 2080),    # large-M, K % 256 == 32, one row into a third 256-row tile
     (1, 128, 256),
     (7, 40, 64),
 ])
