@@ -23,6 +23,14 @@
  *   - Argument checks happen on the host before anything is enqueued; a
  *     failing check returns an error status and enqueues nothing.  A CUDA
  *     launch error returns NVFP4_ERR_CUDA.  No C++ exception crosses the ABI.
+ *     Sizes are bounded before any arithmetic on them: a strided buffer that
+ *     would span more than 2^48 bytes, and M, N, K or a segment at or above
+ *     2^31, give NVFP4_ERR_UNSUPPORTED_SHAPE.  The library cannot see how
+ *     large a buffer is: each entry point states the bytes it reads and
+ *     writes, and the caller provides at least that many.
+ *   - Every entry point may be called from several host threads; the
+ *     per-device state the library caches (device properties, symbol
+ *     addresses, kernel attributes) is set up once under a lock.
  *   - BF16 tensors are row-major with a row stride `ld` in elements.
  *   - Packed codes: two E2M1 codes per byte, element 2j in the low nibble of
  *     byte j (sign in bit 3 of each nibble); a [rows, cols] tensor occupies
