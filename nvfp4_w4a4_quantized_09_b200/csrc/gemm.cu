@@ -8,7 +8,19 @@
 // W4A4 on every linear layer and the fused-module global-scale repair
 // (chatpaper.ai abstract); native NVFP4 execution (evolve.pub FAQ).
 //
-// Design (sm_100a, one CTA per SM, persistent):
+// Three kernels, chosen by M alone (so a fused GEMM and its per-module GEMMs
+// accumulate every output identically):
+//   M <= 128         nvf4_gemm_decode_kernel (gemm_decode.cuh): operands
+//                    swapped, K split over a cluster, persistent.
+//   128 < M <= 256   nvf4_gemm_kernel<128, 6, 2>: one CTA per 128 x 128 tile,
+//                    described below.
+//   M > 256          nvf4_gemm_pair_kernel<5, kSilu>: a CTA pair per 256 x 256
+//                    tile (cta_group::2), described above its definition.
+// Epilogue variants: the gate functions of the Gated DeltaNet projection on
+// chosen segments (any kernel, `apply_gates`), and SiLU(gate) * up with the
+// global scale of h for the MLP's gate_up GEMM (pair kernel, kSilu = true).
+//
+// Design of the one-CTA kernel (sm_100a, one CTA per SM, persistent):
 //   warp 0      TMA producer: A/B code tiles by tiled TMA (128-byte swizzle),
 //               their scale atoms by 1-D bulk copies (the scales are stored
 //               in the tensor-core layout, so one k-step of a 128-row block
