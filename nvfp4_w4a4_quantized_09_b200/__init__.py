@@ -30,6 +30,7 @@ __all__ = [
     "ACT_NONE", "ACT_DECAY_GATE", "ACT_SIGMOID",
     "global_scale", "sf_bytes", "quantize", "quantize_into", "quantize_tensor",
     "gemm", "fused_gemm", "FusedWeight", "linear", "silu_mul", "mlp", "interleave_gate_up", "gemm_silu_mul", "harmonize", "kv_scale", "kv_quantize", "last_device_status",
+    "save_quantized", "load_quantized",
     "debug_wait_timeout", "library_path",
 ]
 
@@ -476,6 +477,62 @@ def kv_quantize(x: torch.Tensor, scale: torch.Tensor, out: Optional[torch.Tensor
     _lib.check("nvfp4_kv_quantize_e4m3", _lib.lib().nvfp4_kv_quantize_e4m3(
         _ptr(x), rows, cols, x.stride(0), _ptr(scale), _ptr(out), out.stride(0), _stream(stream)))
     return out
+
+
+# ---------------------------------------------------------------------------
+# the quantized weight format on disk: quantize (and harmonise) once offline,
+# serve many times.  One torch file holding plain CPU tensors and integers
+# (loadable with weights_only=True): packed codes, scale bytes in their
+# layout, one FP32 global scale per module and the module row counts.
+# ---------------------------------------------------------------------------
+_FORMAT = "nvfp4-w4a4"
+_FORMAT_VERSION = 1
+
+
+def save_quantized(path: str, w) -> None:
+    """Write a QuantizedTensor or FusedWeight (device or host tensors) to path."""
+    if isinstance(w, FusedWeight):
+        kind, sizes, gs, layout = "fused", list(w.sizes), list(w.g_list), SF_TCGEN05
+    elif isinstance(w, QuantizedTensor):
+        kind, sizes, gs, layout = "single", [w.rows], [w.g], w.layout
+    else:
+        raise TypeError("save_quantized takes a QuantizedTensor or a FusedWeight")
+    g = torch.cat([t.detach().reshape(-1)[:1].to("cpu", torch.float32) for t in gs])
+    torch.save({"format": _FORMAT, "version": _FORMAT_VERSION, "kind": kind,
+                "rows": int(sum(sizes)), "cols": int(w.cols), "layout": int(layout),
+                "sizes": [int(n) for n in sizes],
+                "codes": w.codes.detach().to("cpu").contiguous(),
+                "sf": w.sf.detach().to("cpu").contiguous(), "g": g}, path)
+
+
+def load_quantized(path: str, device="cuda"):
+    """Read what save_quantized wrote, onto `device`; every field is checked
+    against the others (shapes, scale bytes for the layout, one scale per
+    module) before anything is returned."""
+    d = torch.load(path, map_location="cpu", weights_only=True)
+    if not isinstance(d, dict) or d.get("format") != _FORMAT or d.get("version") != _FORMAT_VERSION:
+        raise ValueError(f"{path}: not an {_FORMAT} v{_FORMAT_VERSION} file")
+    rows, cols, layout, sizes = d["rows"], d["cols"], d["layout"], d["sizes"]
+    if layout not in (SF_LINEAR, SF_TCGEN05) or cols % 32 or sum(sizes) != rows or \
+            any(n <= 0 for n in sizes) or d["kind"] not in ("single", "fused"):
+        raise ValueError(f"{path}: inconsistent header")
+    _check_packed(d["codes"], "codes", shape=(rows, cols // 2))
+    _check_packed(d["sf"], "sf", min_bytes=_sf_bytes_cached(rows, cols, layout))
+    if d["sf"].numel() != _sf_bytes_cached(rows, cols, layout):
+        raise ValueError(f"{path}: {d['sf'].numel()} scale bytes for a [{rows}, {cols}] weight")
+    _check_f32(d["g"], "g", len(sizes))
+    if d["g"].numel() != len(sizes) or not bool(torch.isfinite(d["g"]).all()) or \
+            not bool((d["g"] > 0).all()):
+        raise ValueError(f"{path}: one positive finite global scale per module expected")
+    codes, sf = d["codes"].to(device), d["sf"].to(device)
+    g = [d["g"][i:i + 1].clone().to(device) for i in range(len(sizes))]
+    if d["kind"] == "fused":
+        if layout != SF_TCGEN05:
+            raise ValueError(f"{path}: a fused weight is stored in the tensor-core layout")
+        return FusedWeight(codes, sf, g, sizes, cols)
+    if len(sizes) != 1:
+        raise ValueError(f"{path}: a single tensor has one module")
+    return QuantizedTensor(codes, sf, g[0], rows, cols, layout)
 
 
 def last_device_status(stream=None) -> int:
