@@ -36,6 +36,7 @@ __all__ = [
 
 
 def library_path() -> str:
+    """Path of the CUDA library the binding loads (built in-tree)."""
     return _lib.LIB_PATH
 
 
@@ -134,6 +135,8 @@ def _workspace(device: torch.device, stream=None) -> torch.Tensor:
 
 
 def sf_bytes(rows: int, cols: int, layout: int = SF_TCGEN05) -> int:
+    """Bytes of the block-scale buffer of a [rows, cols] tensor in `layout`
+    (the tensor-core layout pads rows to 128 and scale columns to 4)."""
     n = ctypes.c_size_t(0)
     _lib.check("nvfp4_sf_bytes", _lib.lib().nvfp4_sf_bytes(rows, cols, layout, ctypes.byref(n)))
     return int(n.value)
@@ -541,5 +544,9 @@ def last_device_status(stream=None) -> int:
 
 
 def debug_wait_timeout(limit_ns: int, stream=None) -> None:
+    """Launch a one-thread kernel whose bounded wait on a barrier nothing
+    arrives on gives up after limit_ns: the device status then reads 5
+    (timeout) through last_device_status(), with the context still usable.
+    Exercises the failure path of every kernel's waits without a fault."""
     _lib.check("nvfp4_debug_wait_timeout",
                _lib.lib().nvfp4_debug_wait_timeout(int(limit_ns), _stream(stream)))
