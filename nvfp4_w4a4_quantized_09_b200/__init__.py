@@ -544,9 +544,10 @@ def last_device_status(stream=None) -> int:
 
 
 def debug_wait_timeout(limit_ns: int, stream=None) -> None:
-    """Launch a one-thread kernel whose bounded wait on a barrier nothing
-    arrives on gives up after limit_ns: the device status then reads 5
-    (timeout) through last_device_status(), with the context still usable.
-    Exercises the failure path of every kernel's waits without a fault."""
+    """Launch one warp whose first thread waits on a barrier that nothing
+    arrives on.  The bounded wait gives up after limit_ns, so the device
+    status then reads 5 (timeout) through last_device_status() and the
+    context stays usable: the failure path of every kernel's waits,
+    exercised without a fault."""
     _lib.check("nvfp4_debug_wait_timeout",
                _lib.lib().nvfp4_debug_wait_timeout(int(limit_ns), _stream(stream)))
