@@ -61,7 +61,10 @@ double oracle_e2m1_value(int code)
 
 /* Unsigned E4M3 ("E4M3FN" without the sign): exponent bias 7, subnormals
  * k * 2^-9, largest finite 448 (code 0x7E); 0x7F is NaN and is never
- * produced by the encoder.  Bit 7 (the sign) is always 0 for block scales. */
+ * produced by the encoder.  Bit 7 (the sign) is always 0 for block scales.
+ * Source: the E4M3 block scale named on the evolve.pub review (Scope &
+ * Claims) and the thevalue.engineering page; the bit fields are those of the
+ * public 8-bit floating-point (E4M3FN) definition, which the pages assume. */
 double oracle_e4m3_value(int code)
 {
     int e = (code >> 3) & 15;
@@ -74,7 +77,9 @@ double oracle_e4m3_value(int code)
 }
 
 /* E2M1 round-to-nearest-even with saturation: the code whose value is nearest
- * to t; on a tie the even code (mantissa bit 0) wins.  Magnitudes beyond 6
+ * to t; on a tie the even code (mantissa bit 0) wins.  The pages name the
+ * format but not the rounding; RNE with saturation is the public NVFP4
+ * conversion and the plainest reading.  Magnitudes beyond 6
  * (infinity included) saturate to 6.  The sign bit is taken from t
  * itself, so a negative t that rounds to magnitude 0 gives code 0x8. */
 int oracle_e2m1_encode(float t)
@@ -95,7 +100,8 @@ int oracle_e2m1_encode(float t)
 
 /* Unsigned E4M3 round-to-nearest-even with saturation to 448: nearest over the
  * 127 finite non-negative codes 0x00..0x7E, tie to the even code.  s must be
- * >= 0 (block scales are magnitudes). */
+ * >= 0 (block scales are magnitudes).  As for E2M1, the rounding is the
+ * public conversion's (the pages give the format only). */
 int oracle_e4m3_encode(float s)
 {
     double a = (double)s;
@@ -122,7 +128,10 @@ static float bf16_to_float(uint16_t b)
 }
 
 /* double -> BF16 with ONE round-to-nearest-even step (no detour through
- * binary32, which would round twice).  BF16: 8 significant bits, exponent
+ * binary32, which would round twice).  The pages measure the quantized model
+ * against BF16 and note that public recipes keep the gate projections in
+ * BF16 (evolve.pub review, Scope & Claims); they do not state the GEMM's
+ * output type, and a BF16 output rounded once is the plainest reading.  BF16: 8 significant bits, exponent
  * range of binary32, subnormal spacing 2^-133.  Overflow gives +-inf. */
 uint16_t oracle_bf16_from_double(double x)
 {
@@ -254,7 +263,9 @@ void oracle_sf_to_tcgen05(const uint8_t* sf_linear, int64_t rows, int64_t sfcols
 /* ---------------------------------------------------------------------- */
 
 /* xq[r, k] = E2M1(code) * E4M3(s8 of the block), WITHOUT the global scale,
- * in FP64 (exact: a 2-bit by 4-bit significand product). */
+ * in FP64 (exact: a 2-bit by 4-bit significand product) -- the value an
+ * NVFP4 element stands for, E2M1 times its block's E4M3 scale (evolve.pub
+ * review, Scope & Claims). */
 void oracle_dequantize_noglobal(const uint8_t* codes, const uint8_t* sf_linear,
                                 int64_t rows, int64_t cols, double* out)
 {
