@@ -4,8 +4,10 @@
  * The layer follows the pages on "Why Gated DeltaNet Survives 4-Bit
  * Quantization: NVFP4 W4A4 for the Recurrent Half of a Hybrid 27B LLM":
  *   - every linear layer runs with 4-bit weights AND activations (chatpaper.ai
- *     abstract: "NVFP4 W4A4 on all 496 linear layers");
- *   - NVFP4 = E2M1 values with one E4M3 scale per 16-element block
+ *     abstract: the paper quantizes every one of its model's 496 linear
+ *     layers this way);
+ *   - NVFP4 = 4-bit E2M1 elements, each group of 16 consecutive elements
+ *     sharing one E4M3 scale
  *     (evolve.pub review, Scope & Claims; thevalue.engineering, second section);
  *   - the GEMM runs natively on NVFP4-capable hardware (evolve.pub FAQ);
  *   - modules fused into one GEMM keep their own global scales, which is the
@@ -158,8 +160,8 @@ nvfp4_status nvfp4_sf_bytes(int64_t rows, int64_t cols, nvfp4_sf_layout layout,
  * `layout`) are written completely, padding included.
  * Requirements: cols % 32 == 0, ld % 8 == 0, ld >= cols; x, codes, sf 16-byte
  * aligned.  rows == 0 enqueues nothing.
- * Source: evolve.pub review, Scope & Claims (E2M1 values, E4M3 scale per
- * 16-element block); thevalue.engineering, second section. */
+ * Source: evolve.pub review, Scope & Claims (the element and scale formats
+ * and the 16-element grouping); thevalue.engineering, second section. */
 nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t ld,
                             const float* g, uint8_t* codes, uint8_t* sf,
                             nvfp4_sf_layout layout, void* stream);
@@ -210,8 +212,9 @@ nvfp4_status nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float
  *   NVFP4_MAX_SEGMENTS.  w_codes/w_sf hold the concatenated [N, K] weight,
  *   each module quantized with its own global scale.
  * Requirements as nvfp4_gemm.
- * Source: chatpaper.ai abstract ("kernels that fuse those modules into one
- * GEMM"); evolve.pub Key claims, fourth bullet. */
+ * Source: chatpaper.ai abstract (serving modules calibrated one by one
+ * through a single fused GEMM is where the mismatch arises); evolve.pub Key
+ * claims, fourth bullet. */
 nvfp4_status nvfp4_fused_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_g,
                               const uint8_t* w_codes, const uint8_t* w_sf,
                               const nvfp4_segment* segs, int nseg,
@@ -230,9 +233,9 @@ nvfp4_status nvfp4_fused_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const
  * Errors: as nvfp4_fused_gemm; NVFP4_ERR_INVALID_ARG for an unknown kind or a
  * missing parameter array.
  * Source: evolve.pub, Key claims under review, second bullet, and Report
- * preview, Table 3 (log-space softplus/exponential and sigmoid gate
- * parameterizations); the formulas are the Gated DeltaNet reading -- the
- * pages give none. */
+ * preview, Table 3 (the decay gate, kept in log space through a softplus and an
+ * exponential, and the sigmoid write strength); the formulas are the Gated
+ * DeltaNet reading -- the pages give none. */
 nvfp4_status nvfp4_fused_gemm_act(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_g,
                                   const uint8_t* w_codes, const uint8_t* w_sf,
                                   const nvfp4_segment* segs, const nvfp4_segment_act* acts,

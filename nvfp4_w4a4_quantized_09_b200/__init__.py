@@ -8,8 +8,8 @@ kernels.  There is no CPU or PyTorch fallback: if ``libnvfp4.so`` is missing,
 the first call raises.
 
 Method: the pages on "Why Gated DeltaNet Survives 4-Bit Quantization: NVFP4
-W4A4 for the Recurrent Half of a Hybrid 27B LLM" -- NVFP4 (E2M1 values, E4M3
-scale per 16-element block) on weights and activations of every linear layer
+W4A4 for the Recurrent Half of a Hybrid 27B LLM" -- NVFP4 (4-bit E2M1 elements,
+16 of them sharing one E4M3 scale) on weights and activations of every linear layer
 (evolve.pub review, Scope & Claims), served by fused multi-module GEMMs whose
 per-module global scales must be honoured (chatpaper.ai abstract).
 """

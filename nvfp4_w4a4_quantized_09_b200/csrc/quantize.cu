@@ -3,8 +3,8 @@
 //   nvfp4_quantize:     16-element block scales (UE4M3) and packed E2M1 codes,
 //                       scales written straight into the tensor-core layout.
 // Format: evolve.pub review of "Why Gated DeltaNet Survives 4-Bit
-// Quantization", Scope & Claims (E2M1 values, E4M3 scale per 16-element
-// block); per-module global scales: chatpaper.ai abstract.
+// Quantization", Scope & Claims (the E2M1 element format, with one E4M3
+// scale for every 16 elements); per-module global scales: chatpaper.ai abstract.
 #include <cuda_runtime.h>
 #include <stdint.h>
 

@@ -10,10 +10,10 @@
  * Sources (the web pages on "Why Gated DeltaNet Survives 4-Bit Quantization:
  * NVFP4 W4A4 for the Recurrent Half of a Hybrid 27B LLM"):
  *   - evolve.pub review, "Report preview / Scope & Claims": NVFP4 W4A4 means
- *     E2M1 values with one E4M3 scale per 16-element block, applied to both
- *     weights and activations of every linear layer.
+ *     4-bit E2M1 elements, each run of 16 sharing one E4M3 scale, on both the
+ *     weights and the activations of every linear layer.
  *   - thevalue.engineering news page, second section: the same format
- *     (4-bit E2M1 values, an E4M3 scale per 16-element block) for native
+ *     (E2M1 elements grouped by 16 under an E4M3 scale) for native
  *     execution.
  *   - chatpaper.ai abstract: per-module-calibrated checkpoints served by
  *     kernels that fuse several modules into one GEMM suffer a global-scale
@@ -161,9 +161,10 @@ uint16_t oracle_bf16_from_double(double x)
  * being the largest magnitude an E2M1 value times an E4M3 scale can hold.
  * An all-zero tensor gets g = 1 so that later divisions stay finite.
  * Source: the per-module global scale implied by the chatpaper.ai abstract
- * ("per-module-calibrated NVFP4 checkpoints", "global-scale mismatch") and
- * the evolve.pub review (Key claims, fourth bullet); the absmax reading is
- * the plainest one for a dynamic activation scale. */
+ * (checkpoints whose modules were calibrated one by one, and the mismatch of
+ * global scales when such modules are fused) and the evolve.pub review (Key
+ * claims, fourth bullet); the absmax reading is the plainest one for a
+ * dynamic activation scale. */
 float oracle_global_scale(const uint16_t* x, int64_t rows, int64_t cols,
                           int64_t ld, float* amax_out)
 {
@@ -192,8 +193,9 @@ float oracle_global_scale(const uint16_t* x, int64_t rows, int64_t cols,
  * Codes are packed two per byte, element 2j in the low nibble of byte j:
  * codes[r * (cols/2) + j].  Scales go to sf_linear[r * (cols/16) + b].
  * cols must be a multiple of 16.
- * Source: evolve.pub review (Scope & Claims: E2M1 values, E4M3 scale per
- * 16-element block); thevalue.engineering page (same format). */
+ * Source: evolve.pub review (Scope & Claims: the E2M1 element format and
+ * its E4M3 scale shared by 16 elements); thevalue.engineering page (same
+ * format). */
 void oracle_quantize(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld,
                      float g, uint8_t* codes, uint8_t* sf_linear)
 {
@@ -283,7 +285,7 @@ void oracle_dequantize_noglobal(const uint8_t* codes, const uint8_t* sf_linear,
  * alpha[n] = gA * gW[seg(n)] (an FP64 product of the two FP32 scales).
  * Only the rows listed in row_ids (n_rows of them) are computed; out is
  * [n_rows, N].  Source: W4A4 GEMM of the chatpaper.ai abstract and the
- * evolve.pub FAQ ("running natively on NVFP4-capable hardware"); the
+ * evolve.pub FAQ (the model runs natively on hardware with NVFP4 support); the
  * per-column alpha is the per-module global scale of the fused-GEMM repair
  * (chatpaper.ai abstract; evolve.pub Key claims, fourth bullet). */
 void oracle_gemm_f64(const double* A, const double* W, const double* alpha,
@@ -452,9 +454,10 @@ void oracle_kv_quantize(const uint16_t* x, int64_t rows, int64_t cols, int64_t l
 
 /* The fused GDN input projection carries the two gate projections: a (one
  * column per head) feeds the log-space decay gate and b feeds the sigmoid
- * write strength; the pages credit these "log-space softplus/exponential and
- * sigmoid parameterizations" with compressing ~11 % GEMM error to ~2 % output
- * error (evolve.pub, Key claims under review, second bullet; Report preview,
+ * write strength; the pages credit these two gate functions (a decay kept in
+ * log space through a softplus and an exponential, and a sigmoid) with
+ * shrinking a GEMM error of about 11 % to an output error of about 2 %
+ * (evolve.pub, Key claims under review, second bullet; Report preview,
  * Table 3).  They give no formula; the plain reading is the Gated DeltaNet
  * parameterisation:
  *   decay (kind 1): g    = -exp(A_log[c]) * softplus(y + dt_bias[c]),
