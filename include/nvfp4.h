@@ -288,7 +288,8 @@ nvfp4_status nvfp4_gemm_silu_mul(const uint8_t* a_codes, const uint8_t* a_sf, co
  *            nvfp4_fused_gemm; the w_gscale pointers are device FP32.
  *   g_common (device) receives g_c.
  * Errors: NVFP4_ERR_INVALID_ARG (null pointer, bad segment table, bad
- * layout), NVFP4_ERR_UNSUPPORTED_SHAPE (K), NVFP4_ERR_ALIGNMENT, CUDA errors.
+ * layout), NVFP4_ERR_UNSUPPORTED_SHAPE (K, or a segment or N at 2^31 or
+ * more), NVFP4_ERR_ALIGNMENT, CUDA errors.
  * Asynchronous on `stream`.
  * Source: chatpaper.ai abstract (per-module-calibrated checkpoints, fused
  * multi-module kernels, the global-scale mismatch and its repair); the choice
@@ -311,7 +312,8 @@ nvfp4_status nvfp4_harmonize_scales(uint8_t* w_sf, int64_t K, const nvfp4_segmen
  *   scale  (device) FP32 per-tensor scale, positive and finite.
  *   out    (device) bytes [rows, cols], row stride ldo bytes; 8-byte aligned.
  * Requirements: cols, ld, ldo multiples of 8; ld >= cols, ldo >= cols.
- * Errors: NVFP4_ERR_INVALID_ARG, NVFP4_ERR_ALIGNMENT, CUDA errors.  Both calls
+ * Errors: NVFP4_ERR_INVALID_ARG, NVFP4_ERR_ALIGNMENT, NVFP4_ERR_UNSUPPORTED_SHAPE
+ * (the size bounds of the conventions above), CUDA errors.  Both calls
  * are asynchronous on `stream`.
  * Source: evolve.pub, Key claims under review (calibrated per-tensor FP8
  * KV-cache scales); the formula is a reading -- the pages give none. */
