@@ -286,9 +286,10 @@ nvfp4_status nvfp4_gemm_silu_mul(const uint8_t* a_codes, const uint8_t* a_sf, co
  *   K        multiple of 16 (so cols/16 scales per row).
  *   segs     (host, nseg entries, copied during the call): as for
  *            nvfp4_fused_gemm; the w_gscale pointers are device FP32.
- *   g_common (device) receives g_c.
+ *   g_common (device) receives g_c; it must not be one of the segments'
+ *            scales (it is written while the kernel still reads them).
  * Errors: NVFP4_ERR_INVALID_ARG (null pointer, bad segment table, bad
- * layout), NVFP4_ERR_UNSUPPORTED_SHAPE (K, or a segment or N at 2^31 or
+ * layout, g_common equal to a segment's scale pointer), NVFP4_ERR_UNSUPPORTED_SHAPE (K, or a segment or N at 2^31 or
  * more), NVFP4_ERR_ALIGNMENT, CUDA errors.
  * Asynchronous on `stream`.
  * Source: chatpaper.ai abstract (per-module-calibrated checkpoints, fused

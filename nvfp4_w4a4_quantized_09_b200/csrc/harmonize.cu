@@ -118,6 +118,8 @@ extern "C" nvfp4_status nvfp4_harmonize_scales(uint8_t* w_sf, int64_t K, const n
         if (segs[s].n_offset != N || segs[s].n_size <= 0 || !segs[s].w_gscale)
             return NVFP4_ERR_INVALID_ARG;
         if (segs[s].n_size >= (int64_t(1) << 31)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+        // g_common is written while other CTAs still read the module scales
+        if (segs[s].w_gscale == g_common) return NVFP4_ERR_INVALID_ARG;
         N += segs[s].n_size;   // at most 16 terms below 2^31: no overflow
     }
     if (K <= 0 || K % 16 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;

@@ -134,7 +134,7 @@ def test_fused_gemm_validates_segment_table(L):
 
 def test_harmonize_rejects_bad_arguments(L):
     f = L.nvfp4_harmonize_scales
-    good = seg_array([(0, 64, 0x10000), (64, 64, 0x10010)])
+    good = seg_array([(0, 64, 0x20000), (64, 64, 0x20010)])   # scales apart from FAKE
     T, LIN = _lib.SF_TCGEN05, _lib.SF_LINEAR
     assert f(NUL, 64, good, 2, T, FAKE, NUL) == _lib.NVFP4_ERR_INVALID_ARG     # no scales
     assert f(FAKE, 64, good, 2, T, NUL, NUL) == _lib.NVFP4_ERR_INVALID_ARG     # no g_common
@@ -147,6 +147,8 @@ def test_harmonize_rejects_bad_arguments(L):
     assert f(FAKE, 64, noscale, 2, LIN, FAKE, NUL) == _lib.NVFP4_ERR_INVALID_ARG
     huge = seg_array([(0, 1 << 62, 0x10000), (1 << 62, 1 << 62, 0x10010)])
     assert f(FAKE, 64, huge, 2, LIN, FAKE, NUL) == _lib.NVFP4_ERR_UNSUPPORTED_SHAPE
+    # g_common may not alias a module scale the kernel is still reading
+    assert f(FAKE, 64, good, 2, LIN, ctypes.c_void_p(0x20010), NUL) == _lib.NVFP4_ERR_INVALID_ARG
     assert f(FAKE, 24, good, 2, T, FAKE, NUL) == _lib.NVFP4_ERR_UNSUPPORTED_SHAPE   # K % 16
     assert f(FAKE, 0, good, 2, T, FAKE, NUL) == _lib.NVFP4_ERR_UNSUPPORTED_SHAPE
     assert f(ctypes.c_void_p(0x10008), 64, good, 2, T, FAKE, NUL) == _lib.NVFP4_ERR_ALIGNMENT
