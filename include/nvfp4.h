@@ -108,7 +108,8 @@ typedef struct {
  * g_out (device, 1 float) receives g; amax_out (device, 1 float) receives
  * amax, or may be NULL.  workspace (device, NVFP4_GLOBAL_SCALE_WORKSPACE_BYTES,
  * 16-byte aligned) must be zero before the first call; every call leaves it
- * zero again.  Calls that share a workspace must not overlap in time.
+ * zero again.  Calls that share a workspace must not overlap in time, and
+ * g_out / amax_out must lie outside it (NVFP4_ERR_INVALID_ARG otherwise).
  * Requirements: cols % 8 == 0, ld % 8 == 0, ld >= cols, x 16-byte aligned.
  * rows == 0 or cols == 0 yields amax = 0, g = 1.
  * Source: the per-module global scale behind the fused-GEMM repair
@@ -256,7 +257,8 @@ nvfp4_status nvfp4_fused_gemm_act(const uint8_t* a_codes, const uint8_t* a_sf, c
  *     quantizing changes neither the rows' codes nor the global scale.
  *   h: device BF16 [M, F], row stride ldh elements.
  *   workspace: as nvfp4_global_scale (NVFP4_GLOBAL_SCALE_WORKSPACE_BYTES,
- *     zero-initialised, left zeroed); h_g, h_amax: device FP32.
+ *     zero-initialised, left zeroed); h_g, h_amax: device FP32, outside
+ *     the workspace (NVFP4_ERR_INVALID_ARG otherwise).
  * Requirements: M > 256 (the CTA-pair prefill kernel; smaller batches use
  * nvfp4_gemm + nvfp4_silu_mul), F a multiple of 128, K as nvfp4_gemm,
  * ldh >= F and a multiple of 8, pointers 16-byte aligned.

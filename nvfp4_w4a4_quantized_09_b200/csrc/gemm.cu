@@ -1231,6 +1231,10 @@ nvfp4_status gemm_silu_impl(const uint8_t* a_codes, const uint8_t* a_sf, const f
     if (!aligned16(a_codes) || !aligned16(a_sf) || !aligned16(w_codes) || !aligned16(w_sf) ||
         !aligned16(h) || !aligned16(workspace))
         return NVFP4_ERR_ALIGNMENT;
+    // the last CTA writes the scale of h and then clears the workspace
+    if (overlaps(h_g, 4, workspace, NVFP4_GLOBAL_SCALE_WORKSPACE_BYTES) ||
+        overlaps(h_amax, 4, workspace, NVFP4_GLOBAL_SCALE_WORKSPACE_BYTES))
+        return NVFP4_ERR_INVALID_ARG;
     DeviceInfo dev;
     nvfp4_status st = require_sm100(&dev);
     if (st != NVFP4_OK) return st;

@@ -50,6 +50,13 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 
 inline nvfp4_status cuda_status(cudaError_t e) { return e == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA; }
 
+// True when [p, p + pn) and [q, q + qn) share a byte (either may be null).
+inline bool overlaps(const void* p, size_t pn, const void* q, size_t qn) {
+    if (!p || !q) return false;
+    const uintptr_t a = reinterpret_cast<uintptr_t>(p), b = reinterpret_cast<uintptr_t>(q);
+    return a < b + qn && b < a + pn;
+}
+
 // True when `rows` rows `ld` elements apart, of elem_bytes each, would span
 // more than 2^48 bytes -- more than any device address space.  Checked before
 // any stride or size arithmetic on caller values (rows, ld >= 0), so that

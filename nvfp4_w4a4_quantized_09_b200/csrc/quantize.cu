@@ -479,6 +479,10 @@ extern "C" nvfp4_status nvfp4_global_scale(const void* x, int64_t rows, int64_t 
     if (rows > 0 && ld < cols) return NVFP4_ERR_INVALID_ARG;
     if (extent_too_large(rows, ld, 2)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
     if ((x && !aligned16(x)) || !aligned16(workspace)) return NVFP4_ERR_ALIGNMENT;
+    // the last CTA writes the results and then clears the workspace
+    if (overlaps(g_out, 4, workspace, NVFP4_GLOBAL_SCALE_WORKSPACE_BYTES) ||
+        overlaps(amax_out, 4, workspace, NVFP4_GLOBAL_SCALE_WORKSPACE_BYTES))
+        return NVFP4_ERR_INVALID_ARG;
     DeviceInfo dev;
     nvfp4_status st = current_device_info(&dev);
     if (st != NVFP4_OK) return st;

@@ -92,6 +92,10 @@ def test_global_scale_rejects_bad_arguments(L):
     assert gs(FAKE, 4, 60, 64, FAKE, NUL, FAKE, NUL) == _lib.NVFP4_ERR_ALIGNMENT
     assert gs(ODD, 4, 64, 64, FAKE, NUL, FAKE, NUL) == _lib.NVFP4_ERR_ALIGNMENT
     assert gs(FAKE, 4, 64, 64, FAKE, NUL, ODD, NUL) == _lib.NVFP4_ERR_ALIGNMENT
+    # results inside the workspace the kernel clears at the end are refused
+    WS = ctypes.c_void_p(0x40000)
+    assert gs(FAKE, 4, 64, 64, ctypes.c_void_p(0x40000 + 200), NUL, WS, NUL) == _lib.NVFP4_ERR_INVALID_ARG
+    assert gs(FAKE, 4, 64, 64, FAKE, ctypes.c_void_p(0x40000 - 2), WS, NUL) == _lib.NVFP4_ERR_INVALID_ARG
 
 
 def test_gemm_rejects_bad_arguments(L):
@@ -200,6 +204,9 @@ def test_gemm_silu_mul_rejects_bad_arguments(L):
     assert f(*a, 256, 300, 256, 256, NUL, FAKE, NUL, NUL) == _lib.NVFP4_ERR_INVALID_ARG         # workspace
     assert f(*a, 256, 300, 256, 256, FAKE, NUL, NUL, NUL) == _lib.NVFP4_ERR_INVALID_ARG         # h_g
     assert f(*a, 256, 300, 256, 256, ODD, FAKE, NUL, NUL) == _lib.NVFP4_ERR_ALIGNMENT
+    WS = ctypes.c_void_p(0x40000)
+    assert f(*a, 256, 300, 256, 256, WS, ctypes.c_void_p(0x40000 + 252), NUL, NUL) == \
+        _lib.NVFP4_ERR_INVALID_ARG                                  # h_g inside the workspace
 
 
 def test_silu_mul_rejects_bad_arguments(L):
