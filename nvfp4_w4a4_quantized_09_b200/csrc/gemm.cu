@@ -1163,6 +1163,18 @@ nvfp4_status gemm_impl(const uint8_t* a_codes, const uint8_t* a_sf, const float*
     if (!aligned16(a_codes) || !aligned16(a_sf) || !aligned16(w_codes) || !aligned16(w_sf) ||
         !aligned16(y))
         return NVFP4_ERR_ALIGNMENT;
+    // the epilogues read the scales and gate parameters while other CTAs write y
+    {
+        const size_t ybytes = extent_bytes(M, ldy, N, 2);
+        if (overlaps(a_g, 4, y, ybytes)) return NVFP4_ERR_INVALID_ARG;
+        for (int s = 0; s < nseg; ++s) {
+            const size_t pb = static_cast<size_t>(segs[s].n_size) * 4;
+            if (overlaps(segs[s].w_gscale, 4, y, ybytes) ||
+                (acts && overlaps(acts[s].a_log, pb, y, ybytes)) ||
+                (acts && overlaps(acts[s].dt_bias, pb, y, ybytes)))
+                return NVFP4_ERR_INVALID_ARG;
+        }
+    }
     DeviceInfo dev;
     nvfp4_status st = require_sm100(&dev);
     if (st != NVFP4_OK) return st;
@@ -1231,9 +1243,12 @@ nvfp4_status gemm_silu_impl(const uint8_t* a_codes, const uint8_t* a_sf, const f
     if (!aligned16(a_codes) || !aligned16(a_sf) || !aligned16(w_codes) || !aligned16(w_sf) ||
         !aligned16(h) || !aligned16(workspace))
         return NVFP4_ERR_ALIGNMENT;
-    // the last CTA writes the scale of h and then clears the workspace
+    // the last CTA writes the scale of h and then clears the workspace; the
+    // epilogues read the input scales while other CTAs write h
+    const size_t hbytes = extent_bytes(M, ldh, F, 2);
     if (overlaps(h_g, 4, workspace, NVFP4_GLOBAL_SCALE_WORKSPACE_BYTES) ||
-        overlaps(h_amax, 4, workspace, NVFP4_GLOBAL_SCALE_WORKSPACE_BYTES))
+        overlaps(h_amax, 4, workspace, NVFP4_GLOBAL_SCALE_WORKSPACE_BYTES) ||
+        overlaps(a_g, 4, h, hbytes) || overlaps(w_g, 4, h, hbytes))
         return NVFP4_ERR_INVALID_ARG;
     DeviceInfo dev;
     nvfp4_status st = require_sm100(&dev);

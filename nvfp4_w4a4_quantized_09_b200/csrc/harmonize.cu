@@ -128,6 +128,10 @@ extern "C" nvfp4_status nvfp4_harmonize_scales(uint8_t* w_sf, int64_t K, const n
     size_t nbytes = 0;
     nvfp4_status st = nvfp4_sf_bytes(N, K, layout, &nbytes);
     if (st != NVFP4_OK) return st;
+    // the module scales are read, and g_common written, while w_sf is rewritten
+    if (overlaps(g_common, 4, w_sf, nbytes)) return NVFP4_ERR_INVALID_ARG;
+    for (int s = 0; s < nseg; ++s)
+        if (overlaps(segs[s].w_gscale, 4, w_sf, nbytes)) return NVFP4_ERR_INVALID_ARG;
     DeviceInfo dev;
     st = require_sm100(&dev);
     if (st != NVFP4_OK) return st;

@@ -57,6 +57,14 @@ inline bool overlaps(const void* p, size_t pn, const void* q, size_t qn) {
     return a < b + qn && b < a + pn;
 }
 
+// Bytes spanned by a row-major [rows, cols] matrix with row stride ld, all
+// counted in elements of elem_bytes (0 when empty).  Callers have bounded
+// rows and ld with extent_too_large first.
+inline size_t extent_bytes(int64_t rows, int64_t ld, int64_t cols, int64_t elem_bytes) {
+    if (rows <= 0 || cols <= 0) return 0;
+    return static_cast<size_t>(((rows - 1) * ld + cols) * elem_bytes);
+}
+
 // True when `rows` rows `ld` elements apart, of elem_bytes each, would span
 // more than 2^48 bytes -- more than any device address space.  Checked before
 // any stride or size arithmetic on caller values (rows, ld >= 0), so that

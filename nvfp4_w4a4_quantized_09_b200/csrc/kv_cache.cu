@@ -164,6 +164,8 @@ extern "C" nvfp4_status nvfp4_kv_quantize_e4m3(const void* x, int64_t rows, int6
     if (extent_too_large(rows, ld, 2) || extent_too_large(rows, ldo, 1))
         return NVFP4_ERR_UNSUPPORTED_SHAPE;
     if (!aligned16(x) || (reinterpret_cast<uintptr_t>(out) & 7u) != 0) return NVFP4_ERR_ALIGNMENT;
+    // every CTA reads *scale while others write out
+    if (overlaps(scale, 4, out, extent_bytes(rows, ldo, cols, 1))) return NVFP4_ERR_INVALID_ARG;
     if (cols / 8 >= (int64_t(1) << 31)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
     DeviceInfo dev;
     const nvfp4_status st = current_device_info(&dev);

@@ -479,9 +479,12 @@ extern "C" nvfp4_status nvfp4_global_scale(const void* x, int64_t rows, int64_t 
     if (rows > 0 && ld < cols) return NVFP4_ERR_INVALID_ARG;
     if (extent_too_large(rows, ld, 2)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
     if ((x && !aligned16(x)) || !aligned16(workspace)) return NVFP4_ERR_ALIGNMENT;
-    // the last CTA writes the results and then clears the workspace
+    // the last CTA writes the results and then clears the workspace, while
+    // other CTAs may still read x
+    const size_t xbytes = extent_bytes(rows, ld, cols, 2);
     if (overlaps(g_out, 4, workspace, NVFP4_GLOBAL_SCALE_WORKSPACE_BYTES) ||
-        overlaps(amax_out, 4, workspace, NVFP4_GLOBAL_SCALE_WORKSPACE_BYTES))
+        overlaps(amax_out, 4, workspace, NVFP4_GLOBAL_SCALE_WORKSPACE_BYTES) ||
+        overlaps(g_out, 4, x, xbytes) || overlaps(amax_out, 4, x, xbytes))
         return NVFP4_ERR_INVALID_ARG;
     DeviceInfo dev;
     nvfp4_status st = current_device_info(&dev);
@@ -517,6 +520,13 @@ nvfp4_status quantize_impl(const void* x, int64_t rows, int64_t cols, int64_t ld
     if (!codes || !sf || (rows > 0 && !x)) return NVFP4_ERR_INVALID_ARG;
     if (rows > 0 && ld < cols) return NVFP4_ERR_INVALID_ARG;
     if ((x && !aligned16(x)) || !aligned16(codes) || !aligned16(sf)) return NVFP4_ERR_ALIGNMENT;
+    // every CTA reads *g while others write codes and scales
+    size_t sf_total = 0;
+    const nvfp4_status sfst = nvfp4_sf_bytes(total_rows, cols, layout, &sf_total);
+    if (sfst != NVFP4_OK) return sfst;
+    if (overlaps(g, 4, codes, static_cast<size_t>(total_rows) * static_cast<size_t>(cols / 2)) ||
+        overlaps(g, 4, sf, sf_total))
+        return NVFP4_ERR_INVALID_ARG;
     QuantParams p;
     p.x = static_cast<const uint8_t*>(x);
     p.ld_bytes = ld * 2;

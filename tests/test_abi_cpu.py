@@ -250,3 +250,40 @@ def test_python_api_refuses_cpu_tensors():
     import nvfp4_w4a4_quantized_09_b200 as nv
     with pytest.raises(ValueError):
         nv.quantize_tensor(torch.zeros(4, 64, dtype=torch.bfloat16))
+
+
+def test_scalars_aliasing_an_output_are_refused(L):
+    # a kernel reads these scalars while other CTAs write the output, so a
+    # scalar inside the output's bytes is refused on the host (fake pointers,
+    # never dereferenced)
+    P = ctypes.c_void_p
+    OUT, OUT2 = 0x50000, 0x60000
+    # quantize: g inside the codes, or inside the scale bytes
+    assert L.nvfp4_quantize(FAKE, 4, 64, 64, P(OUT + 16), P(OUT), P(OUT2), 1, NUL) == _lib.NVFP4_ERR_INVALID_ARG
+    assert L.nvfp4_quantize(FAKE, 4, 64, 64, P(OUT2 + 256), P(OUT), P(OUT2), 1, NUL) == _lib.NVFP4_ERR_INVALID_ARG
+    # global scale: g_out inside x
+    assert L.nvfp4_global_scale(P(OUT), 4, 64, 64, P(OUT + 256), NUL, FAKE, NUL) == _lib.NVFP4_ERR_INVALID_ARG
+    # GEMM: the activation's scale inside y (4 x 128 BF16 = 1 KB)
+    g = L.nvfp4_gemm
+    assert g(FAKE, FAKE, P(OUT + 1000), FAKE, FAKE, FAKE, P(OUT), 128, 4, 128, 64, NUL) == _lib.NVFP4_ERR_INVALID_ARG
+    # fused GEMM: a module's scale inside y; a gate parameter array reaching into y
+    f = L.nvfp4_fused_gemm
+    segs = seg_array([(0, 64, 0x20000), (64, 64, OUT + 512)])
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, segs, 2, P(OUT), 128, 4, 64, NUL) == _lib.NVFP4_ERR_INVALID_ARG
+    fa = L.nvfp4_fused_gemm_act
+    segs = seg_array([(0, 64, 0x20000), (64, 64, 0x20010)])
+    acts = (_lib.SegmentAct * 2)()
+    acts[1].kind, acts[1].a_log, acts[1].dt_bias = _lib.ACT_DECAY_GATE, OUT - 200, 0x30000   # 256 B: ends in y
+    assert fa(FAKE, FAKE, FAKE, FAKE, FAKE, segs, acts, 2, P(OUT), 128, 4, 64, NUL) == _lib.NVFP4_ERR_INVALID_ARG
+    # SiLU GEMM: an input scale inside h
+    s = L.nvfp4_gemm_silu_mul
+    assert s(FAKE, FAKE, P(OUT + 64), FAKE, FAKE, FAKE, P(OUT), 256, 300, 256, 256, P(0x40000),
+             P(0x48000), NUL, NUL) == _lib.NVFP4_ERR_INVALID_ARG
+    # KV cache: the scale inside the output bytes
+    assert L.nvfp4_kv_quantize_e4m3(FAKE, 4, 8, 8, P(OUT + 8), P(OUT), 8, NUL) == _lib.NVFP4_ERR_INVALID_ARG
+    # harmonisation: a module scale, or g_common, inside the scale bytes being rewritten
+    h = L.nvfp4_harmonize_scales
+    segs = seg_array([(0, 64, 0x20000), (64, 64, OUT + 100)])
+    assert h(P(OUT), 64, segs, 2, _lib.SF_LINEAR, P(0x30000), NUL) == _lib.NVFP4_ERR_INVALID_ARG
+    segs = seg_array([(0, 64, 0x20000), (64, 64, 0x20010)])
+    assert h(P(OUT), 64, segs, 2, _lib.SF_LINEAR, P(OUT + 400), NUL) == _lib.NVFP4_ERR_INVALID_ARG

@@ -1,8 +1,10 @@
-"""The library's once-per-device set-up helper (csrc/host_common.h), compiled
-with the host C++ compiler and driven from many threads: every device's
-set-up runs exactly once however many threads race for it, what the set-up
-wrote is visible to every caller that returns, and a failed set-up is retried
-rather than cached."""
+"""Host helpers of the library (csrc/host_common.h), compiled with the host
+C++ compiler.  The once-per-device set-up, driven from many threads: every
+device's set-up runs exactly once however many threads race for it, what the
+set-up wrote is visible to every caller that returns, and a failed set-up is
+retried rather than cached.  The size and overlap checks the entry points run
+before any launch: half-open byte ranges, strided extents, and the 2^48-byte
+bound at its edge and far beyond it."""
 import os
 import shutil
 import subprocess
@@ -77,3 +79,41 @@ def test_per_device_once_under_contention(tmp_path):
     out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
     assert out.returncode == 0, out.stdout + out.stderr
     assert out.stdout.strip() == "ok"
+
+
+HELPERS = r"""
+#include "host_common.h"
+#include <cstdio>
+
+using namespace nvfp4;
+
+int main() {
+    char buf[64];
+    // half-open byte ranges: touching is not overlapping
+    if (!overlaps(buf, 4, buf + 3, 4) || !overlaps(buf + 3, 4, buf, 4)) return 1;
+    if (overlaps(buf, 4, buf + 4, 4) || overlaps(buf + 4, 4, buf, 4)) return 2;
+    if (!overlaps(buf + 10, 4, buf, 64) || overlaps(nullptr, 4, buf, 64)) return 3;
+    // bytes of a strided matrix: (rows - 1) * ld + cols elements
+    if (extent_bytes(4, 64, 32, 2) != (3 * 64 + 32) * 2) return 4;
+    if (extent_bytes(0, 64, 32, 2) != 0 || extent_bytes(4, 64, 0, 2) != 0) return 5;
+    // 2^48-byte bound, checked without overflow even for huge operands
+    if (extent_too_large(1, int64_t(1) << 47, 2)) return 6;           // exactly 2^48 bytes
+    if (!extent_too_large(2, int64_t(1) << 47, 2)) return 7;
+    if (!extent_too_large(int64_t(1) << 62, int64_t(1) << 62, 8)) return 8;
+    if (extent_too_large(0, int64_t(1) << 62, 2) || extent_too_large(32768, 34816, 2)) return 9;
+    std::printf("ok\n");
+    return 0;
+}
+"""
+
+
+@pytest.mark.skipif(shutil.which("g++") is None or not os.path.exists(CUDA_INCLUDE),
+                    reason="needs g++ and the CUDA headers")
+def test_size_and_overlap_helpers(tmp_path):
+    src = tmp_path / "helpers.cpp"
+    exe = tmp_path / "helpers"
+    src.write_text(HELPERS)
+    subprocess.check_call(["g++", "-std=c++17", "-O2", "-I", CSRC, "-I", INCLUDE,
+                           "-I", CUDA_INCLUDE, "-o", str(exe), str(src)])
+    out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert out.returncode == 0 and out.stdout.strip() == "ok", (out.returncode, out.stdout, out.stderr)
