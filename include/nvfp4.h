@@ -139,8 +139,8 @@ nvfp4_status nvfp4_global_scale(const void* x, int64_t rows, int64_t cols, int64
  * first call before any stream capture.  All calls on a device share the one
  * array, which keeps the last call's contents: calls that overlap on the GPU
  * (different streams, no ordering between them) race and may return a wrong
- * g; serialize them.  Arguments, results and requirements as
- * nvfp4_global_scale, without `workspace`. */
+ * g; serialize them.  Arguments, results, requirements and errors as
+ * nvfp4_global_scale, without `workspace`.  Source: as nvfp4_global_scale. */
 nvfp4_status nvfp4_global_scale_noalloc(const void* x, int64_t rows, int64_t cols, int64_t ld,
                                         float* g_out, float* amax_out, void* stream);
 
@@ -161,6 +161,9 @@ nvfp4_status nvfp4_sf_bytes(int64_t rows, int64_t cols, nvfp4_sf_layout layout,
  * `layout`) are written completely, padding included.
  * Requirements: cols % 32 == 0, ld % 8 == 0, ld >= cols; x, codes, sf 16-byte
  * aligned.  rows == 0 enqueues nothing.
+ * Errors: NVFP4_ERR_INVALID_ARG (null pointer, negative size, ld < cols, bad
+ * layout, g inside codes or sf), NVFP4_ERR_ALIGNMENT (cols, ld or a pointer),
+ * NVFP4_ERR_UNSUPPORTED_SHAPE (the size bounds), CUDA errors.
  * Source: evolve.pub review, Scope & Claims (the element and scale formats
  * and the 16-element grouping); thevalue.engineering, second section. */
 nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t ld,
@@ -174,8 +177,8 @@ nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t l
  * cols, layout) scale bytes); only this slice's rows are written, plus, when
  * row_offset + rows == total_rows, the tensor-core layout's padding rows.
  * Calls for different slices of one tensor may run in any order.
- * Requirements as nvfp4_quantize; 0 <= row_offset, row_offset + rows <=
- * total_rows.
+ * Requirements and errors as nvfp4_quantize; 0 <= row_offset, row_offset +
+ * rows <= total_rows (NVFP4_ERR_INVALID_ARG otherwise).
  * Source: per-module global scales of a fused GEMM (chatpaper.ai abstract;
  * evolve.pub Key claims, fourth bullet). */
 nvfp4_status nvfp4_quantize_slice(const void* x, int64_t rows, int64_t cols, int64_t ld,
@@ -194,6 +197,11 @@ nvfp4_status nvfp4_quantize_slice(const void* x, int64_t rows, int64_t cols, int
  * nvfp4_quantize like activations.  No bias.
  * Requirements: K % 32 == 0, K >= 32; ldy >= N, ldy % 8 == 0; all pointers
  * 16-byte aligned.  M == 0 or N == 0 enqueues nothing.
+ * Errors: NVFP4_ERR_INVALID_ARG (null pointer, negative size, a scale inside
+ * y), NVFP4_ERR_ALIGNMENT (ldy or a pointer), NVFP4_ERR_UNSUPPORTED_SHAPE (K,
+ * the size bounds), NVFP4_ERR_DEVICE (not sm_100), CUDA errors.  A bounded
+ * wait that gives up inside the kernel is reported later by
+ * nvfp4_last_device_status as NVFP4_ERR_TIMEOUT.
  * Source: chatpaper.ai abstract (W4A4 on every linear layer); evolve.pub FAQ
  * (native NVFP4 execution). */
 nvfp4_status nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_g,
@@ -212,7 +220,9 @@ nvfp4_status nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float
  *   starting at 0, n_size > 0; N = sum of n_size.  1 <= nseg <=
  *   NVFP4_MAX_SEGMENTS.  w_codes/w_sf hold the concatenated [N, K] weight,
  *   each module quantized with its own global scale.
- * Requirements as nvfp4_gemm.
+ * Requirements as nvfp4_gemm.  Errors as nvfp4_gemm, and NVFP4_ERR_INVALID_ARG
+ * for a segment table that is not contiguous from 0 or has more than
+ * NVFP4_MAX_SEGMENTS entries.
  * Source: chatpaper.ai abstract (serving modules calibrated one by one
  * through a single fused GEMM is where the mismatch arises); evolve.pub Key
  * claims, fourth bullet. */
@@ -330,7 +340,10 @@ nvfp4_status nvfp4_kv_quantize_e4m3(const void* x, int64_t rows, int64_t cols, i
  * evaluated in FP32 (expf, IEEE division); h is BF16 [rows, f], row stride
  * ldh (device).  Within one BF16 ulp of the value rounded once from exact
  * arithmetic.  Requirements: f, ld, ldh multiples of 8; ld >= 2f, ldh >= f;
- * pointers 16-byte aligned.
+ * pointers 16-byte aligned.  rows == 0 or f == 0 enqueues nothing.
+ * Errors: NVFP4_ERR_INVALID_ARG (null pointer, negative size, ld < 2f,
+ * ldh < f), NVFP4_ERR_ALIGNMENT (f, ld, ldh or a pointer),
+ * NVFP4_ERR_UNSUPPORTED_SHAPE (the size bounds), CUDA errors.
  * Source: W4A4 on every linear layer, the MLP down projection included
  * (chatpaper.ai abstract); the SiLU-gated MLP is the plain reading of the
  * 27B hybrid's MLP block, which the pages do not describe. */

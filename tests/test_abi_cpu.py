@@ -32,6 +32,26 @@ def test_header_declares_the_path():
         assert required in names
 
 
+UTILITIES = {"nvfp4_sf_bytes", "nvfp4_last_device_status", "nvfp4_debug_wait_timeout",
+             "nvfp4_status_string", "nvfp4_version"}
+
+
+def test_every_computational_entry_documents_its_source_and_errors():
+    # each declaration of the path is preceded by a comment that cites the
+    # passage it follows and states its errors (utilities have no passage)
+    src = open(HEADER).read()
+    found = set()
+    for m in re.finditer(r"/\*((?:(?!\*/).)*)\*/\s*\n(?:nvfp4_status|const char\*|int)\s+(nvfp4_[a-z0-9_]+)\(",
+                         src, re.S):
+        comment, name = m.group(1), m.group(2)
+        found.add(name)
+        if name in UTILITIES:
+            continue
+        assert "Source" in comment, f"{name}: no source passage"
+        assert "Errors" in comment or "errors" in comment, f"{name}: no error behaviour"
+    assert set(declared_functions()) - found <= {"nvfp4_kv_quantize_e4m3"}   # shares the KV block
+
+
 def test_library_exports_every_declared_symbol(L):
     for name in declared_functions():
         assert hasattr(L, name), name
