@@ -112,6 +112,10 @@ typedef struct {
  * g_out / amax_out must lie outside it (NVFP4_ERR_INVALID_ARG otherwise).
  * Requirements: cols % 8 == 0, ld % 8 == 0, ld >= cols, x 16-byte aligned.
  * rows == 0 or cols == 0 yields amax = 0, g = 1.
+ * Errors: NVFP4_ERR_INVALID_ARG (null g_out or workspace, negative size,
+ * ld < cols, a result inside the workspace or inside x), NVFP4_ERR_ALIGNMENT
+ * (cols, ld, x or workspace), NVFP4_ERR_UNSUPPORTED_SHAPE (the size bounds),
+ * CUDA errors.
  * Source: the per-module global scale behind the fused-GEMM repair
  * (chatpaper.ai abstract); absmax is the dynamic reading of it. */
 nvfp4_status nvfp4_global_scale(const void* x, int64_t rows, int64_t cols, int64_t ld,
