@@ -338,6 +338,37 @@ nvfp4_status nvfp4_kv_scale_from_amax(const float* amax, float* scale, void* str
 nvfp4_status nvfp4_kv_quantize_e4m3(const void* x, int64_t rows, int64_t cols, int64_t ld,
                                     const float* scale, uint8_t* out, int64_t ldo, void* stream);
 
+/* The whole W4A4 linear layer from host buffers, on one stream: the BF16
+ * activation x_host [M, K] is copied into x_dev, its global scale (a_g,
+ * a_amax) and NVFP4 codes (a_codes, a_sf in the tensor-core layout)
+ * computed, the fused GEMM run against the pre-quantized weight (w_codes,
+ * w_sf, segs exactly as nvfp4_fused_gemm), and y_dev [M, N] (row stride N)
+ * copied back to y_host -- nvfp4_global_scale, nvfp4_quantize and
+ * nvfp4_fused_gemm between two cudaMemcpyAsync calls.
+ *   x_host (host) BF16 [M, K], contiguous; y_host (host) BF16 [M, N],
+ *            contiguous.  Page-locked memory makes the copies asynchronous;
+ *            pageable memory works but the copies then block the caller.
+ *   x_dev (device, M * K * 2 bytes), a_codes (device, M * K/2 bytes), a_sf
+ *            (device, nvfp4_sf_bytes(M, K, NVFP4_SF_TCGEN05) bytes), a_g,
+ *            a_amax (device FP32; a_amax may be NULL), workspace (device, as
+ *            nvfp4_global_scale), y_dev (device, M * N * 2 bytes): scratch
+ *            the caller owns; the call allocates nothing.
+ * Every check of the three composed calls is made before anything is
+ * enqueued, so a refused call enqueues nothing.  Requirements: K % 32 == 0,
+ * N % 8 == 0, device pointers 16-byte aligned, no scalar inside an output
+ * and x_dev apart from y_dev.
+ * Errors: NVFP4_ERR_INVALID_ARG, NVFP4_ERR_ALIGNMENT,
+ * NVFP4_ERR_UNSUPPORTED_SHAPE, NVFP4_ERR_DEVICE, as the composed calls;
+ * NVFP4_ERR_CUDA when a copy or a launch fails.  M == 0 enqueues nothing.
+ * Source: the pages' serving path, W4A4 on every linear layer with
+ * per-module global scales in the fused GEMM (chatpaper.ai abstract;
+ * evolve.pub review, Scope & Claims). */
+nvfp4_status nvfp4_fused_linear_host(const void* x_host, int64_t M, int64_t K,
+                                     const uint8_t* w_codes, const uint8_t* w_sf,
+                                     const nvfp4_segment* segs, int nseg, void* y_host,
+                                     void* x_dev, uint8_t* a_codes, uint8_t* a_sf, float* a_g,
+                                     float* a_amax, void* workspace, void* y_dev, void* stream);
+
 /* MLP intermediate for the W4A4 down projection: h[r, c] = BF16_RNE(
  * fl32(SiLU(gate) * up)) with gate = gate_up[r, c], up = gate_up[r, f + c]
  * (BF16, row stride ld elements, device) and SiLU(v) = v / (1 + e^-v)

@@ -30,7 +30,7 @@ __all__ = [
     "ACT_NONE", "ACT_DECAY_GATE", "ACT_SIGMOID",
     "global_scale", "sf_bytes", "quantize", "quantize_into", "quantize_tensor",
     "gemm", "fused_gemm", "FusedWeight", "linear", "silu_mul", "mlp", "interleave_gate_up", "gemm_silu_mul", "harmonize", "kv_scale", "kv_quantize", "last_device_status",
-    "save_quantized", "load_quantized",
+    "save_quantized", "load_quantized", "linear_host", "HostLinearScratch",
     "debug_wait_timeout", "library_path",
 ]
 
@@ -388,6 +388,67 @@ def linear(x: torch.Tensor, w, y: Optional[torch.Tensor] = None, stream=None) ->
     if isinstance(w, FusedWeight):
         return fused_gemm(a, w.codes, w.sf, w.segments(), y, stream)
     return gemm(a, w, y, stream)
+
+
+class HostLinearScratch:
+    """Device scratch of linear_host for one (M, K, N): the activation copy,
+    its codes, scales, global scale and amax, the global-scale workspace and
+    the output before its copy back.  Reuse it across calls of that shape on
+    one stream (its workspace is left zeroed by every call)."""
+
+    def __init__(self, M: int, K: int, N: int, device):
+        self.shape = (int(M), int(K), int(N))
+        self.x = torch.empty(M, K, dtype=torch.bfloat16, device=device)
+        self.codes = torch.empty(M, K // 2, dtype=torch.uint8, device=device)
+        self.sf = torch.empty(sf_bytes(M, K), dtype=torch.uint8, device=device)
+        self.g = torch.empty(1, dtype=torch.float32, device=device)
+        self.amax = torch.empty(1, dtype=torch.float32, device=device)
+        self.workspace = torch.zeros(_lib.GLOBAL_SCALE_WORKSPACE_BYTES, dtype=torch.uint8, device=device)
+        self.y = torch.empty(M, N, dtype=torch.bfloat16, device=device)
+
+
+def linear_host(x_host: torch.Tensor, w, y_host: Optional[torch.Tensor] = None,
+                scratch: Optional[HostLinearScratch] = None, stream=None) -> torch.Tensor:
+    """The W4A4 linear layer from a host BF16 activation [M, K] to a host BF16
+    output [M, N] through one C-ABI call (nvfp4_fused_linear_host): copy in,
+    global scale, quantization, fused GEMM against the pre-quantized weight
+    (FusedWeight or QuantizedTensor), copy out.  The copies are asynchronous
+    when the host tensors are page-locked: synchronize `stream` before
+    reading y_host."""
+    if not isinstance(x_host, torch.Tensor) or x_host.dtype != torch.bfloat16 or x_host.dim() != 2 \
+            or x_host.is_cuda or not x_host.is_contiguous():
+        raise ValueError("x_host must be a contiguous 2-D bfloat16 host tensor")
+    if isinstance(w, FusedWeight):
+        segments = w.segments()
+    elif isinstance(w, QuantizedTensor):
+        if w.layout != SF_TCGEN05:
+            raise ValueError("the GEMM reads block scales in the tensor-core layout")
+        segments = [(0, w.rows, w.g)]
+    else:
+        raise TypeError("w must be a FusedWeight or a QuantizedTensor")
+    M, K = x_host.shape
+    if K != w.cols:
+        raise ValueError(f"x_host has {K} columns, the weight {w.cols}")
+    N = _check_segments(segments, w.rows)
+    _check_packed(w.codes, "w.codes", shape=(N, K // 2))
+    _check_packed(w.sf, "w.sf", min_bytes=_sf_bytes_cached(N, K, SF_TCGEN05))
+    if y_host is None:
+        y_host = torch.empty(M, N, dtype=torch.bfloat16, pin_memory=True)
+    elif (not isinstance(y_host, torch.Tensor) or y_host.dtype != torch.bfloat16 or y_host.is_cuda
+          or y_host.shape != (M, N) or not y_host.is_contiguous()):
+        raise ValueError(f"y_host must be a contiguous bfloat16 host tensor of shape ({M}, {N})")
+    if scratch is None:
+        scratch = HostLinearScratch(M, K, N, w.codes.device)
+    elif scratch.shape != (M, K, N):
+        raise ValueError(f"scratch is for {scratch.shape}, the call needs {(M, K, N)}")
+    _check_devices(w_codes=w.codes, w_sf=w.sf, x=scratch.x, codes=scratch.codes, sf=scratch.sf,
+                   g=scratch.g, workspace=scratch.workspace, y=scratch.y,
+                   **{f"segments[{i}] g": g for i, (_, _, g) in enumerate(segments)})
+    _lib.check("nvfp4_fused_linear_host", _lib.lib().nvfp4_fused_linear_host(
+        _ptr(x_host), M, K, _ptr(w.codes), _ptr(w.sf), _segment_array(segments), len(segments),
+        _ptr(y_host), _ptr(scratch.x), _ptr(scratch.codes), _ptr(scratch.sf), _ptr(scratch.g),
+        _ptr(scratch.amax), _ptr(scratch.workspace), _ptr(scratch.y), _stream(stream)))
+    return y_host
 
 
 def silu_mul(gate_up: torch.Tensor, h: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:

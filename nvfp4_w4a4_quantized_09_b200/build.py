@@ -18,7 +18,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libnvfp4.so")
-SOURCES = ["quantize.cu", "gemm.cu", "mlp.cu", "harmonize.cu", "kv_cache.cu"]
+SOURCES = ["quantize.cu", "gemm.cu", "mlp.cu", "harmonize.cu", "kv_cache.cu", "linear_host.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

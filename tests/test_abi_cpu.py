@@ -307,3 +307,24 @@ def test_scalars_aliasing_an_output_are_refused(L):
     assert h(P(OUT), 64, segs, 2, _lib.SF_LINEAR, P(0x30000), NUL) == _lib.NVFP4_ERR_INVALID_ARG
     segs = seg_array([(0, 64, 0x20000), (64, 64, 0x20010)])
     assert h(P(OUT), 64, segs, 2, _lib.SF_LINEAR, P(OUT + 400), NUL) == _lib.NVFP4_ERR_INVALID_ARG
+
+
+def test_fused_linear_host_rejects_bad_arguments_before_enqueuing(L):
+    f = L.nvfp4_fused_linear_host
+    P = ctypes.c_void_p
+    segs = seg_array([(0, 64, 0x20000), (64, 64, 0x20010)])
+    scratch = (P(0x100000), P(0x200000), P(0x300000), P(0x400000), P(0x410000), P(0x420000),
+               P(0x500000))                                  # x_dev .. y_dev
+    H = P(0x900000)                                          # host buffers (never touched)
+    assert f(H, 4, 48, FAKE, FAKE, segs, 2, H, *scratch, NUL) == _lib.NVFP4_ERR_UNSUPPORTED_SHAPE  # K % 32
+    odd = seg_array([(0, 64, 0x20000), (64, 60, 0x20010)])
+    assert f(H, 4, 64, FAKE, FAKE, odd, 2, H, *scratch, NUL) == _lib.NVFP4_ERR_ALIGNMENT         # N % 8
+    gap = seg_array([(0, 64, 0x20000), (72, 64, 0x20010)])
+    assert f(H, 4, 64, FAKE, FAKE, gap, 2, H, *scratch, NUL) == _lib.NVFP4_ERR_INVALID_ARG
+    assert f(NUL, 4, 64, FAKE, FAKE, segs, 2, H, *scratch, NUL) == _lib.NVFP4_ERR_INVALID_ARG       # no x_host
+    assert f(H, 4, 64, FAKE, FAKE, segs, 2, H, ODD, *scratch[1:], NUL) == _lib.NVFP4_ERR_ALIGNMENT
+    same = (P(0x100000),) + scratch[1:6] + (P(0x100000),)   # y_dev on top of x_dev
+    assert f(H, 4, 64, FAKE, FAKE, segs, 2, H, *same, NUL) == _lib.NVFP4_ERR_INVALID_ARG
+    g_in_codes = scratch[:3] + (P(0x200010),) + scratch[4:]  # a_g inside a_codes
+    assert f(H, 4, 64, FAKE, FAKE, segs, 2, H, *g_in_codes, NUL) == _lib.NVFP4_ERR_INVALID_ARG
+    assert f(H, 0, 64, FAKE, FAKE, segs, 2, H, *scratch, NUL) == _lib.NVFP4_OK                     # M = 0

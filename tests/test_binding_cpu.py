@@ -157,3 +157,21 @@ def test_well_formed_host_tensors_stop_at_the_device_check():
                       torch.zeros(512, dtype=torch.uint8), [(0, 32, G), (32, 16, G)])
     with pytest.raises(ValueError, match="must be a CUDA tensor"):
         nv.quantize(X, G)
+
+
+def test_linear_host_checks_its_arguments_before_the_library():
+    w = _q(48, 64)
+    with pytest.raises(ValueError, match="x_host must be a contiguous 2-D bfloat16 host tensor"):
+        nv.linear_host(torch.zeros(8, 64, dtype=torch.float32), w)
+    with pytest.raises(ValueError, match="x_host must be"):
+        nv.linear_host(torch.zeros(64, 8, dtype=torch.bfloat16).t(), w)
+    with pytest.raises(TypeError):
+        nv.linear_host(X, torch.zeros(4))
+    with pytest.raises(ValueError, match="x_host has 64 columns, the weight 96"):
+        nv.linear_host(X, _q(48, 96))
+    with pytest.raises(ValueError, match=r"y_host must be a contiguous bfloat16 host tensor of shape \(8, 48\)"):
+        nv.linear_host(X, w, torch.zeros(8, 40, dtype=torch.bfloat16))
+    scratch = nv.HostLinearScratch.__new__(nv.HostLinearScratch)
+    scratch.shape = (8, 64, 40)
+    with pytest.raises(ValueError, match=r"scratch is for \(8, 64, 40\)"):
+        nv.linear_host(X, w, torch.zeros(8, 48, dtype=torch.bfloat16), scratch=scratch)
