@@ -21,6 +21,7 @@ import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 SRC = os.path.join(ROOT, "oracle", "nvfp4_oracle.c")
+PY_SRC = os.path.join(ROOT, "oracle", "__init__.py")
 
 # (name, text in the oracle, replacement, which occurrence (0 = first))
 MUTANTS = [
@@ -90,6 +91,24 @@ MUTANTS = [
 ]
 
 
+# the same for the oracle's Python wrapper (argument marshalling and the
+# per-column alpha); every one stays inside the buffers it touches
+PY_MUTANTS = [
+    ("alpha without the weight scale", "alpha[int(off):int(off) + int(size)] = float(np.float32(g_a)) * float(np.float32(gw))",
+     "alpha[int(off):int(off) + int(size)] = float(np.float32(g_a))"),
+    ("alpha with the weight scale squared", "alpha[int(off):int(off) + int(size)] = float(np.float32(g_a)) * float(np.float32(gw))",
+     "alpha[int(off):int(off) + int(size)] = float(np.float32(gw)) * float(np.float32(gw))"),
+    ("harmonisation rows from the offsets", "seg_rows = np.array([int(s[1]) for s in segments], np.int64)",
+     "seg_rows = np.array([int(s[0]) for s in segments], np.int64)"),
+    ("SiLU row stride f", "_L().oracle_silu_mul(_ptr(gu), rows, f, two_f, _ptr(h))",
+     "_L().oracle_silu_mul(_ptr(gu), rows, f, f, _ptr(h))"),
+    ("gate parameters swapped", "_ptr(y), rows, ncols, ncols, _ptr(al), _ptr(db), int(kind)",
+     "_ptr(y), rows, ncols, ncols, _ptr(db), _ptr(al), int(kind)"),
+    ("quantizer row stride halved", "_L().oracle_quantize(_ptr(x), rows, cols, cols, ctypes.c_float(float(g)),",
+     "_L().oracle_quantize(_ptr(x), rows, cols, cols // 2, ctypes.c_float(float(g)),"),
+]
+
+
 def _apply(src: str, old: str, new: str, nth: int) -> str:
     """src with the nth occurrence of `old` in code (comments skipped, so a
     mistake is never planted where the compiler ignores it) replaced."""
@@ -102,12 +121,13 @@ def _apply(src: str, old: str, new: str, nth: int) -> str:
     return src[:pos] + new + src[pos + len(old):]
 
 
-def _tree(base: str, c_source: str) -> str:
+def _tree(base: str, c_source: str, py_source: str) -> str:
     """A minimal copy in which `import oracle` and the pins resolve to the
     planted oracle: oracle/ (wrapper + C source), tests/ (conftest, pins,
     golden files)."""
     os.makedirs(os.path.join(base, "oracle"))
-    shutil.copy(os.path.join(ROOT, "oracle", "__init__.py"), os.path.join(base, "oracle"))
+    with open(os.path.join(base, "oracle", "__init__.py"), "w") as f:
+        f.write(py_source)
     with open(os.path.join(base, "oracle", "nvfp4_oracle.c"), "w") as f:
         f.write(c_source)
     os.makedirs(os.path.join(base, "tests"))
@@ -128,12 +148,16 @@ def _run_pins(base: str) -> subprocess.CompletedProcess:
 @pytest.mark.skipif(shutil.which("gcc") is None, reason="needs gcc for the C oracle")
 def test_every_planted_mistake_fails_a_pin(tmp_path):
     src = open(SRC).read()
+    py = open(PY_SRC).read()
     planted = []
     for i, (name, old, new, nth) in enumerate(MUTANTS):
         mutated = _apply(src, old, new, nth)
         assert mutated, f"mutant '{name}' no longer applies to the oracle source"
-        planted.append((name, _tree(str(tmp_path / f"m{i:02d}"), mutated)))
-    control = _tree(str(tmp_path / "control"), src)
+        planted.append((name, _tree(str(tmp_path / f"m{i:02d}"), mutated, py)))
+    for i, (name, old, new) in enumerate(PY_MUTANTS):
+        assert py.count(old) == 1, f"mutant '{name}' no longer applies to the oracle wrapper"
+        planted.append((name, _tree(str(tmp_path / f"p{i:02d}"), src, py.replace(old, new))))
+    control = _tree(str(tmp_path / "control"), src, py)
 
     with ThreadPoolExecutor(max_workers=max(1, min(8, os.cpu_count() or 1))) as pool:
         ctrl = pool.submit(_run_pins, control)
