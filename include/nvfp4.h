@@ -16,7 +16,9 @@
  *
  * Conventions shared by every entry point:
  *   - Pointers marked (device) are CUDA device pointers on the current device;
- *     (host) pointers are read during the call only.  The caller allocates and
+ *     (host) pointers are read during the call only -- except the activation
+ *     and output of nvfp4_fused_linear_host, which its stream's copies use
+ *     until they complete.  The caller allocates and
  *     owns every buffer; the library allocates no device memory.
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *     stream).  Work is enqueued asynchronously; nothing synchronizes except
@@ -346,8 +348,10 @@ nvfp4_status nvfp4_kv_quantize_e4m3(const void* x, int64_t rows, int64_t cols, i
  * copied back to y_host -- nvfp4_global_scale, nvfp4_quantize and
  * nvfp4_fused_gemm between two cudaMemcpyAsync calls.
  *   x_host (host) BF16 [M, K], contiguous; y_host (host) BF16 [M, N],
- *            contiguous.  Page-locked memory makes the copies asynchronous;
- *            pageable memory works but the copies then block the caller.
+ *            contiguous.  Page-locked memory makes the copies asynchronous:
+ *            keep both buffers alive, x_host unchanged and y_host unread
+ *            until the stream has passed the copies (synchronize it).
+ *            Pageable memory works, but the copies then block the caller.
  *   x_dev (device, M * K * 2 bytes), a_codes (device, M * K/2 bytes), a_sf
  *            (device, nvfp4_sf_bytes(M, K, NVFP4_SF_TCGEN05) bytes), a_g,
  *            a_amax (device FP32; a_amax may be NULL), workspace (device, as
