@@ -1,8 +1,9 @@
 """Parity at the full workload sizes, in the launch configuration the
 benchmark times: the quantizer on the whole [32768, 5120] activation
 (bit-exact), the fused GDN input projection at 8192 x 24704 x 5120 (codes and
-scales bit-exact everywhere, GEMM on sampled rows against the oracle, fused ==
-per-module bit for bit), and the decode-shaped sweep."""
+scales bit-exact everywhere, GEMM on 256 seeded rows against the oracle, fused ==
+per-module bit for bit), the decode-shaped sweep (every row), and the 32K MLP
+(64 seeded rows through every stage)."""
 import numpy as np
 import pytest
 import torch
@@ -61,7 +62,7 @@ def test_fused_gdn_prefill_full_size():
     assert np.array_equal(np_u8(fw.sf), oracle.sf_to_tcgen05(sw))
     xb = host_bits(x)
     ga, _ = oracle.global_scale(xb)
-    rows = sample_rows(8192, 14, 0)
+    rows = sample_rows(8192, 254, 0)                     # 256 rows with the first and last
     ca, sa = oracle.quantize(xb[rows], ga)
     assert np.array_equal(np_u8(a.codes)[rows], ca)
     # GEMM on sampled rows against the FP64 oracle
@@ -112,7 +113,7 @@ def test_decode_sweep(which, M):
     torch.cuda.synchronize()
     xb = host_bits(x)
     ga, _ = oracle.global_scale(xb)
-    rows = sample_rows(M, 6, M)
+    rows = sample_rows(M, M, M)                          # every row (M <= 128)
     ca, sa = oracle.quantize(xb[rows], ga)
     A = dequant(ca, sa)
     alpha = oracle.segment_alpha(ga, segs)
@@ -135,7 +136,7 @@ def test_mlp_32k_prefill_sampled():
     hq = nv.quantize_tensor(h)
     y = nv.gemm(hq, wq_dn)
     torch.cuda.synchronize()
-    rows = sample_rows(M, 6, 7)
+    rows = sample_rows(M, 62, 7)
     rid = torch.from_numpy(rows).to(DEV)
     xb = host_bits(x)
     ga, _ = oracle.global_scale(xb)
