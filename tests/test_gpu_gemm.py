@@ -8,8 +8,7 @@ import torch
 import oracle
 import nvfp4_w4a4_quantized_09_b200 as nv
 from nvfp4_w4a4_quantized_09_b200 import synth
-from parity_helpers import (assert_gemm_matches, dequant, host_bits, np_f32, np_u8,
-                            oracle_quant)
+from parity_helpers import assert_gemm_matches, dequant, host_bits, np_f32, oracle_quant
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"

@@ -7,7 +7,6 @@ a sign error, a swapped operand or a small scale error.  Every mistake is
 planted in oracle-side data (no GPU involved)."""
 import numpy as np
 import pytest
-import torch
 
 import oracle
 from nvfp4_w4a4_quantized_09_b200 import synth
