@@ -107,11 +107,6 @@ def gdn_gate_params(heads: int, seed: int = 40, device="cpu"):
     return (torch.log(a).to(torch.float32).to(device), dt_bias.to(torch.float32).to(device))
 
 
-def random_bf16(rows: int, cols: int, seed: int, scale: float = 1.0, device="cpu"):
-    """Plain N(0, scale) BF16 matrix for small parity cases."""
-    return gaussian_weights(rows, cols, scale, seed, device)
-
-
 def bf16_bits(t: torch.Tensor):
     """Host numpy uint16 view of a BF16 tensor's bit patterns (for the oracle)."""
     import numpy as np

@@ -14,14 +14,6 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
 
-def gpu_quant(x, g=None, layout=nv.SF_TCGEN05):
-    if g is None:
-        g, amax = nv.global_scale(x)
-    codes, sf = nv.quantize(x, g, layout)
-    torch.cuda.synchronize()
-    return codes, sf, g
-
-
 def check_quant_bitexact(x, layout=nv.SF_TCGEN05, g_host=None):
     bits = host_bits(x)
     if g_host is None:
