@@ -118,10 +118,12 @@ def _c(a, dtype):
 # --------------------------------------------------------------------------
 
 def e2m1_value(code: int) -> float:
+    """Value of a 4-bit E2M1 code (bit 3 the sign) -- oracle_e2m1_value."""
     return _L().oracle_e2m1_value(int(code))
 
 
 def e4m3_value(code: int) -> float:
+    """Value of an E4M3 byte (NaN for 0x7F/0xFF) -- oracle_e4m3_value."""
     return _L().oracle_e4m3_value(int(code))
 
 
@@ -150,6 +152,7 @@ def bf16_from_double(x) -> np.ndarray:
 
 
 def bf16_bits_to_f64(b) -> np.ndarray:
+    """Exact FP64 values of BF16 bit patterns (uint16)."""
     b = _c(b, np.uint16)
     return (b.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
 
@@ -180,6 +183,8 @@ def quantize(x_bf16: np.ndarray, g: float):
 
 
 def sf_offset_tcgen05(r: int, c: int, sfcols_padded: int) -> int:
+    """Byte offset of scale (row r, 16-block column c) in the tensor-core
+    layout with sfcols_padded scale columns -- oracle_sf_offset_tcgen05."""
     return _L().oracle_sf_offset_tcgen05(r, c, sfcols_padded)
 
 
@@ -195,6 +200,8 @@ def sf_to_tcgen05(sf_linear: np.ndarray) -> np.ndarray:
 
 
 def dequantize_noglobal(codes: np.ndarray, sf_linear: np.ndarray) -> np.ndarray:
+    """FP64 [rows, cols] of E2M1(code) x E4M3(block scale), without the
+    global scale (exact) -- oracle_dequantize_noglobal."""
     codes = _c(codes, np.uint8)
     sf = _c(sf_linear, np.uint8)
     rows = codes.shape[0]
@@ -316,6 +323,7 @@ def silu_mul_f64(gate64: np.ndarray, up64: np.ndarray) -> np.ndarray:
 
 
 def num_threads() -> int:
+    """Threads the oracle's parallel loops use."""
     return int(_L().oracle_num_threads())
 
 
