@@ -1158,6 +1158,9 @@ nvfp4_status gemm_impl(const uint8_t* a_codes, const uint8_t* a_sf, const float*
         return NVFP4_ERR_UNSUPPORTED_SHAPE;
     if (ldy < N || ldy % 8 != 0) return NVFP4_ERR_ALIGNMENT;
     if (extent_too_large(M, ldy, 2)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    // tile indices are 32-bit in the kernels (128 x 128 tiles at the finest),
+    // and a persistent CTA adds the grid size to its index
+    if (((M + 127) / 128) * ((N + 127) / 128) >= (int64_t(1) << 30)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
     if (M == 0) return NVFP4_OK;
     if (!a_codes || !a_sf || !w_codes || !w_sf || !y) return NVFP4_ERR_INVALID_ARG;
     if (!aligned16(a_codes) || !aligned16(a_sf) || !aligned16(w_codes) || !aligned16(w_sf) ||
@@ -1238,6 +1241,7 @@ nvfp4_status gemm_silu_impl(const uint8_t* a_codes, const uint8_t* a_sf, const f
         return NVFP4_ERR_UNSUPPORTED_SHAPE;
     if (ldh < F || ldh % 8 != 0) return NVFP4_ERR_ALIGNMENT;
     if (extent_too_large(M, ldh, 2)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (((M + 255) / 256) * ((2 * F + 255) / 256) >= (int64_t(1) << 30)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
     if (M <= 256) return NVFP4_ERR_UNSUPPORTED_SHAPE;      // the CTA-pair (prefill) kernel only
     if (!a_codes || !a_sf || !w_codes || !w_sf || !h) return NVFP4_ERR_INVALID_ARG;
     if (!aligned16(a_codes) || !aligned16(a_sf) || !aligned16(w_codes) || !aligned16(w_sf) ||

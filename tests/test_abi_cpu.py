@@ -256,6 +256,9 @@ def test_extents_that_would_overflow_are_refused(L):
     assert L.nvfp4_silu_mul(FAKE, 1, 1 << 62, 128, FAKE, 64, NUL) == _lib.NVFP4_ERR_INVALID_ARG
     ok = (FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE)
     assert L.nvfp4_gemm(*ok, wide, big, 128, 64, NUL) == _lib.NVFP4_ERR_UNSUPPORTED_SHAPE
+    # 2^30 tiles of 128 x 128 or more: beyond the kernels' 32-bit tile indices
+    # (an output of 2^47 bytes, under the extent bound, so this check decides)
+    assert L.nvfp4_gemm(*ok, 1 << 23, 1 << 23, 1 << 23, 64, NUL) == _lib.NVFP4_ERR_UNSUPPORTED_SHAPE
     assert L.nvfp4_gemm_silu_mul(*ok, 1 << 62, 300, 1 << 62, 256, FAKE, FAKE, NUL, NUL) == \
         _lib.NVFP4_ERR_UNSUPPORTED_SHAPE
 
