@@ -420,6 +420,20 @@ using namespace nvfp4;
 // ---------------------------------------------------------------------------
 static __device__ __align__(256) unsigned char g_noalloc_scratch[NVFP4_NOALLOC_SCRATCH_BYTES];
 
+// Checks of nvfp4_global_scale's arguments other than the workspace, in the
+// order the entry points report them; shared with the no-alloc variant so
+// that it too refuses a call before enqueuing anything.
+static nvfp4_status global_scale_args(const void* x, int64_t rows, int64_t cols, int64_t ld,
+                                      const float* g_out) {
+    if (!g_out || rows < 0 || cols < 0) return NVFP4_ERR_INVALID_ARG;
+    if (rows > 0 && cols > 0 && !x) return NVFP4_ERR_INVALID_ARG;
+    if (cols % 8 != 0 || ld % 8 != 0) return NVFP4_ERR_ALIGNMENT;
+    if (rows > 0 && ld < cols) return NVFP4_ERR_INVALID_ARG;
+    if (extent_too_large(rows, ld, 2)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (x && !aligned16(x)) return NVFP4_ERR_ALIGNMENT;
+    return NVFP4_OK;
+}
+
 static nvfp4_status noalloc_scratch_ptr(void** out) {
     static void* cache[kMaxDevices] = {nullptr};
     static PerDeviceOnce once;
@@ -443,9 +457,13 @@ extern "C" nvfp4_status nvfp4_global_scale_noalloc(const void* x, int64_t rows, 
     static_assert(sizeof(GlobalScaleWorkspace) <= NVFP4_NOALLOC_SCRATCH_BYTES,
                   "scratch array too small for the global-scale workspace");
     if (sizeof(GlobalScaleWorkspace) > NVFP4_NOALLOC_SCRATCH_BYTES) return NVFP4_ERR_UNSUPPORTED_SHAPE;
-    if (!g_out || rows < 0 || cols < 0) return NVFP4_ERR_INVALID_ARG;
+    // refuse before the memset below is enqueued
+    nvfp4_status st = global_scale_args(x, rows, cols, ld, g_out);
+    if (st != NVFP4_OK) return st;
+    const size_t xbytes = extent_bytes(rows, ld, cols, 2);
+    if (overlaps(g_out, 4, x, xbytes) || overlaps(amax_out, 4, x, xbytes)) return NVFP4_ERR_INVALID_ARG;
     void* ws = nullptr;
-    nvfp4_status st = noalloc_scratch_ptr(&ws);
+    st = noalloc_scratch_ptr(&ws);
     if (st != NVFP4_OK) return st;
     // the workspace must start at zero: clear it on the stream (no allocation)
     if (cudaMemsetAsync(ws, 0, sizeof(GlobalScaleWorkspace), as_stream(stream)) != cudaSuccess)
@@ -473,12 +491,10 @@ extern "C" nvfp4_status nvfp4_sf_bytes(int64_t rows, int64_t cols, nvfp4_sf_layo
 extern "C" nvfp4_status nvfp4_global_scale(const void* x, int64_t rows, int64_t cols, int64_t ld,
                                            float* g_out, float* amax_out, void* workspace,
                                            void* stream) {
-    if (!g_out || !workspace || rows < 0 || cols < 0) return NVFP4_ERR_INVALID_ARG;
-    if (rows > 0 && cols > 0 && !x) return NVFP4_ERR_INVALID_ARG;
-    if (cols % 8 != 0 || ld % 8 != 0) return NVFP4_ERR_ALIGNMENT;
-    if (rows > 0 && ld < cols) return NVFP4_ERR_INVALID_ARG;
-    if (extent_too_large(rows, ld, 2)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
-    if ((x && !aligned16(x)) || !aligned16(workspace)) return NVFP4_ERR_ALIGNMENT;
+    if (!workspace) return NVFP4_ERR_INVALID_ARG;
+    nvfp4_status st = global_scale_args(x, rows, cols, ld, g_out);
+    if (st != NVFP4_OK) return st;
+    if (!aligned16(workspace)) return NVFP4_ERR_ALIGNMENT;
     // the last CTA writes the results and then clears the workspace, while
     // other CTAs may still read x
     const size_t xbytes = extent_bytes(rows, ld, cols, 2);
@@ -487,7 +503,7 @@ extern "C" nvfp4_status nvfp4_global_scale(const void* x, int64_t rows, int64_t 
         overlaps(g_out, 4, x, xbytes) || overlaps(amax_out, 4, x, xbytes))
         return NVFP4_ERR_INVALID_ARG;
     DeviceInfo dev;
-    nvfp4_status st = current_device_info(&dev);
+    st = current_device_info(&dev);
     if (st != NVFP4_OK) return st;
     const int64_t eff_rows = (cols == 0) ? 0 : rows;
     int64_t warps = eff_rows < 1 ? 1 : eff_rows;

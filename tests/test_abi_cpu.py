@@ -118,6 +118,21 @@ def test_global_scale_rejects_bad_arguments(L):
     assert gs(FAKE, 4, 64, 64, FAKE, ctypes.c_void_p(0x40000 - 2), WS, NUL) == _lib.NVFP4_ERR_INVALID_ARG
 
 
+def test_global_scale_noalloc_refuses_before_enqueuing(L):
+    # the no-alloc form clears its scratch with a memset on the stream; every
+    # refusal must come before that (no CUDA call is made for these)
+    gs = L.nvfp4_global_scale_noalloc
+    P = ctypes.c_void_p
+    assert gs(FAKE, 4, 64, 64, NUL, NUL, NUL) == _lib.NVFP4_ERR_INVALID_ARG          # g_out
+    assert gs(NUL, 4, 64, 64, FAKE, NUL, NUL) == _lib.NVFP4_ERR_INVALID_ARG          # x
+    assert gs(FAKE, 4, 60, 64, FAKE, NUL, NUL) == _lib.NVFP4_ERR_ALIGNMENT           # cols % 8
+    assert gs(FAKE, 4, 64, 60, FAKE, NUL, NUL) == _lib.NVFP4_ERR_ALIGNMENT           # ld % 8
+    assert gs(FAKE, 4, 64, 56, FAKE, NUL, NUL) == _lib.NVFP4_ERR_INVALID_ARG         # ld < cols
+    assert gs(ODD, 4, 64, 64, P(0x30000), NUL, NUL) == _lib.NVFP4_ERR_ALIGNMENT      # x alignment
+    assert gs(P(0x50000), 4, 64, 64, P(0x50000 + 100), NUL, NUL) == _lib.NVFP4_ERR_INVALID_ARG   # g in x
+    assert gs(FAKE, 1 << 30, 64, 1 << 20, FAKE, NUL, NUL) == _lib.NVFP4_ERR_UNSUPPORTED_SHAPE
+
+
 def test_gemm_rejects_bad_arguments(L):
     g = L.nvfp4_gemm
     ok = (FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE)
