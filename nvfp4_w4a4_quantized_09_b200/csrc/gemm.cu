@@ -1172,9 +1172,11 @@ nvfp4_status gemm_impl(const uint8_t* a_codes, const uint8_t* a_sf, const float*
         if (overlaps(a_g, 4, y, ybytes)) return NVFP4_ERR_INVALID_ARG;
         for (int s = 0; s < nseg; ++s) {
             const size_t pb = static_cast<size_t>(segs[s].n_size) * 4;
+            // the parameter arrays are read only for a decay gate (unused otherwise)
+            const bool decay = acts && acts[s].kind == NVFP4_ACT_DECAY_GATE;
             if (overlaps(segs[s].w_gscale, 4, y, ybytes) ||
-                (acts && overlaps(acts[s].a_log, pb, y, ybytes)) ||
-                (acts && overlaps(acts[s].dt_bias, pb, y, ybytes)))
+                (decay && overlaps(acts[s].a_log, pb, y, ybytes)) ||
+                (decay && overlaps(acts[s].dt_bias, pb, y, ybytes)))
                 return NVFP4_ERR_INVALID_ARG;
         }
     }

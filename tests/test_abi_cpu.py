@@ -346,3 +346,19 @@ def test_fused_linear_host_rejects_bad_arguments_before_enqueuing(L):
     g_in_codes = scratch[:3] + (P(0x200010),) + scratch[4:]  # a_g inside a_codes
     assert f(H, 4, 64, FAKE, FAKE, segs, 2, H, *g_in_codes, NUL) == _lib.NVFP4_ERR_INVALID_ARG
     assert f(H, 0, 64, FAKE, FAKE, segs, 2, H, *scratch, NUL) == _lib.NVFP4_OK                     # M = 0
+
+
+def test_unused_gate_parameters_are_not_checked_for_aliasing(L):
+    # a sigmoid segment's a_log is documented as unused: whatever it points at,
+    # even inside y, does not refuse the call.  The decay segment has 300
+    # columns (over the 256 the kernels stage), so the call still stops on the
+    # host: NVFP4_ERR_CUDA here without a GPU, UNSUPPORTED_SHAPE on one --
+    # never the aliasing refusal, and never a launch.
+    P = ctypes.c_void_p
+    Y = 0x50000
+    segs = seg_array([(0, 64, 0x20000), (64, 300, 0x20010)])
+    acts = (_lib.SegmentAct * 2)()
+    acts[0].kind, acts[0].a_log, acts[0].dt_bias = _lib.ACT_SIGMOID, Y + 16, 0
+    acts[1].kind, acts[1].a_log, acts[1].dt_bias = _lib.ACT_DECAY_GATE, 0x30000, 0x34000
+    st = L.nvfp4_fused_gemm_act(FAKE, FAKE, FAKE, FAKE, FAKE, segs, acts, 2, P(Y), 368, 4, 64, NUL)
+    assert st in (_lib.NVFP4_ERR_CUDA, _lib.NVFP4_ERR_UNSUPPORTED_SHAPE), st
