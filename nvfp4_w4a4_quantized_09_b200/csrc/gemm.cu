@@ -14,7 +14,7 @@
 //                    swapped, K split over a cluster, persistent.
 //   128 < M <= 256   nvf4_gemm_kernel<128, 6, 2>: one CTA per 128 x 128 tile,
 //                    described below.
-//   M > 256          nvf4_gemm_pair_kernel<5, kSilu>: a CTA pair per 256 x 256
+//   M > 256          nvf4_gemm_pair_kernel<5, 128, kSilu>: a CTA pair per 256 x 256
 //                    tile (cta_group::2), described above its definition.
 // Epilogue variants: the gate functions of the Gated DeltaNet projection on
 // chosen segments (any kernel, `apply_gates`), and SiLU(gate) * up with the
@@ -58,8 +58,17 @@ constexpr int kAtom = 512;           // one scale atom: 128 rows x 4 scales
 constexpr int kAtomsPerStep = 4;     // 256 values = 16 scales = 4 atoms per row block
 constexpr int kEpiWarps = 8;         // two per TMEM lane quarter, each half the columns
 constexpr int kThreads = 64 + 32 * kEpiWarps;  // producer, MMA, epilogue warps
-constexpr int kPairThreads = kThreads + 32;      // + scale-copy warp
+constexpr int kPairThreads = kThreads;           // producer, MMA, epilogue warps
 constexpr uint64_t kTimeoutNs = 1000000000ull;  // 1 s per wait
+#ifndef NVFP4_PAIR_KB
+#define NVFP4_PAIR_KB 128
+#endif
+#ifndef NVFP4_PAIR_STAGES
+#define NVFP4_PAIR_STAGES 5
+#endif
+// CTA-pair kernel pipeline: bytes of every row per stage and stage count
+constexpr int kPairKB = NVFP4_PAIR_KB;
+constexpr int kPairStages = NVFP4_PAIR_STAGES;
 
 struct GemmArgs {
     const uint8_t* a_sf;
@@ -467,42 +476,50 @@ nvf4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
 // 256 x 256 output tile.  Each CTA loads its own 128 rows of A, its 128-row
 // half of the tile's B rows, its own A scale atoms and the B scale atoms of
 // the whole 256-row N tile; every load is a 2-D TMA whose bytes are counted on
-// the even CTA's full barrier.  A dedicated copy thread of the even CTA copies
-// each stage's scale atoms into that stage's own 48-column TMEM region of both
-// CTAs (each CTA's shared memory at the same offset into its own TMEM) and
-// signals sf_ready; the MMA thread, which then issues nothing but
-// tcgen05.mma.cta_group::2 (M = 256, N = 256, K = 64), overlaps with those
-// copies (issued from one thread, the copies and MMAs would run one after the
-// other; the copies alone cost more than the MMAs).  Accumulator rows 0..127
-// live in the even CTA's TMEM and 128..255 in the odd CTA's.  Commits are multicast to both CTAs'
-// barriers; both CTAs' epilogue warps release the accumulator on the even
-// CTA's barrier.  Per CTA and k-step this moves 38 KB from L2 for 128 x 256 x
-// 256 multiply-adds (the single-CTA 128 x 256 tile moves 54 KB).
+// the even CTA's full barrier.  A stage holds KB bytes of every row (2 KB
+// values of K): KB = 64 gives ten 19 KB stages (64-byte swizzle), KB = 128
+// five 38 KB stages (128-byte swizzle).  The MMA warp of the even CTA copies a
+// stage's scale atoms into that stage's own TMEM region of both CTAs
+// (tcgen05.cp, each CTA's shared memory into its own TMEM) and issues
+// tcgen05.mma.cta_group::2 (M = 256, N = 256, K = 64) right behind them from
+// the same thread, so the copies and the MMAs that read them execute in issue
+// order without any handshake.  Feeding the tensor cores is a latency
+// problem: a stage is refilled only after its MMAs complete, so the time from
+// that commit through the TMA reload to the next MMA on it must fit in the
+// MMA time of the other stages; every hop removed from that loop and every
+// finer stage raises the sustained rate.  Accumulator rows 0..127 live in the
+// even CTA's TMEM and 128..255 in the odd CTA's.  Commits are multicast to
+// both CTAs' barriers; both CTAs' epilogue warps release the accumulator on
+// the even CTA's barrier.  Per CTA and 256 values of K this moves 38 KB from
+// L2 for 128 x 256 x 256 multiply-adds (the single-CTA 128 x 256 tile moves
+// 54 KB).
 // ---------------------------------------------------------------------------
-template <int STAGES>
+template <int STAGES, int KB>
 struct PairCfg {
     static constexpr int BN = 256;
-    static constexpr int A_BYTES = kBM * kBKBytes;                 // own 128 rows of A
-    static constexpr int B_BYTES = 128 * kBKBytes;                 // own half of the N tile
-    static constexpr int SFA_BYTES = kAtomsPerStep * kAtom;        // own 128-row block
-    static constexpr int SFB_BYTES = 2 * kAtomsPerStep * kAtom;    // both 128-row blocks of N
+    static constexpr int ATOMS = KB / 32;                          // scale atoms per 128-row block
+    static constexpr int A_BYTES = kBM * KB;                       // own 128 rows of A
+    static constexpr int B_BYTES = 128 * KB;                       // own half of the N tile
+    static constexpr int SFA_BYTES = ATOMS * kAtom;                // own 128-row block
+    static constexpr int SFB_BYTES = 2 * ATOMS * kAtom;            // both 128-row blocks of N
     static constexpr int STAGE_TX = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
     static constexpr int OFF_A = 0;
     static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
     static constexpr int OFF_SFA = OFF_B + STAGES * B_BYTES;
     static constexpr int OFF_SFB = OFF_SFA + STAGES * SFA_BYTES;
     static constexpr int OFF_BAR = OFF_SFB + STAGES * SFB_BYTES;
-    static constexpr int NBAR = 3 * STAGES + 4;                  // full, empty, sf_ready, tmem_full, tmem_empty, drain x2
+    static constexpr int NBAR = 2 * STAGES + 3;                  // full, empty, tmem_full, tmem_empty, drain
     static constexpr int OFF_SEG = OFF_BAR + NBAR * 8;
     static constexpr int OFF_MISC = OFF_SEG + static_cast<int>((sizeof(SegTable) + 15) / 16 * 16);
     static constexpr int SMEM = OFF_MISC + 16 + 1024;
-    static constexpr int SFA_COL = BN;                           // one accumulator of 256 columns
-    static constexpr int SFB_COL = SFA_COL + kAtomsPerStep * 4;
-    static constexpr int SF_STRIDE = kAtomsPerStep * 12;         // 48 columns per stage region
+    static constexpr int SF_STRIDE = ATOMS * 12;                 // TMEM columns per stage region
+    static constexpr int SFB_COL = ATOMS * 4;                    // B scales after the A scales
     static constexpr int TMEM_COLS = 512;
+    static_assert(KB == 64 || KB == 128, "stage row bytes: 64 or 128");
     static_assert(BN + STAGES * SF_STRIDE <= TMEM_COLS, "tensor memory overflow");
     static_assert(SMEM <= 232448, "shared memory overflow");
     static_assert(SMEM > 228 * 1024 / 2, "two CTAs per SM would share TMEM");
+    static_assert(A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "swizzled tiles stay 1024-byte aligned");
 };
 
 // kind::mxf4nvf4 descriptor for the pair MMA: M = 256, N = 256.
@@ -511,25 +528,31 @@ __host__ __device__ constexpr uint32_t make_idesc_pair() {
            (static_cast<uint32_t>(256 >> 4) << 24);
 }
 
-template <int STAGES, bool kSilu>
+// K-major operand descriptor for rows of KB bytes in the matching swizzle.
+template <int KB>
+__device__ __forceinline__ uint64_t sdesc_kmajor(uint32_t saddr) {
+    if constexpr (KB == 128) return sdesc_kmajor_sw128(saddr);
+    else return sdesc_kmajor_sw64(saddr);
+}
+
+template <int STAGES, int KB, bool kSilu>
 __global__ void __launch_bounds__(kPairThreads, 1)
 nvf4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a,
                       const __grid_constant__ CUtensorMap tmap_b,
                       const __grid_constant__ CUtensorMap tmap_sfa,
                       const __grid_constant__ CUtensorMap tmap_sfb, const GemmArgs args) {
-    using C = PairCfg<STAGES>;
+    using C = PairCfg<STAGES, KB>;
     constexpr int BN = C::BN;
+    constexpr int ATOMS = C::ATOMS;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
     uint64_t* full = bars;
     uint64_t* empty = bars + STAGES;
-    uint64_t* sf_ready = bars + 2 * STAGES;
-    uint64_t* tmem_full = bars + 3 * STAGES;
-    uint64_t* tmem_empty = bars + 3 * STAGES + 1;
-    uint64_t* drain = bars + 3 * STAGES + 2;
-    uint64_t* drain2 = bars + 3 * STAGES + 3;
+    uint64_t* tmem_full = bars + 2 * STAGES;
+    uint64_t* tmem_empty = bars + 2 * STAGES + 1;
+    uint64_t* drain = bars + 2 * STAGES + 2;
     SegTable& seg_tab = *reinterpret_cast<SegTable*>(smem + C::OFF_SEG);
     const float* s_seg_alpha = seg_tab.alpha;
     const int* s_seg_end = seg_tab.end;
@@ -547,12 +570,10 @@ nvf4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a,
         for (int i = 0; i < STAGES; ++i) {
             mbar_init(&full[i], 1);
             mbar_init(&empty[i], 1);
-            mbar_init(&sf_ready[i], 1);
         }
         mbar_init(tmem_full, 1);
         mbar_init(tmem_empty, 2 * kEpiWarps);            // both CTAs' epilogue warps
         mbar_init(drain, 1);
-        mbar_init(drain2, 1);
         *s_abort = 0;
         fence_mbar_init();
         prefetch_tmap(&tmap_a);
@@ -577,9 +598,9 @@ nvf4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a,
 
     // The issuing roles run as whole warps with one elected lane issuing, so
     // ring counters, descriptors and addresses stay warp-uniform; only the
-    // last k-step of K can carry fewer than four scale atoms.
+    // last stage of K can carry fewer scale atoms than ATOMS.
     const int last_kb = args.k_steps - 1;
-    const int last_natoms = args.atoms_per_rb - last_kb * kAtomsPerStep;
+    const int last_natoms = args.atoms_per_rb - last_kb * ATOMS;
 
     if (warp == 0) {
         // ---------------- TMA producer (both CTAs) ----------------
@@ -592,7 +613,7 @@ nvf4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a,
             int mt, nt;
             tile_coords(t, args, mt, nt);
             for (int kb = 0; kb < args.k_steps; ++kb) {
-                if (!mbar_wait_warp(&empty[stage], phase ^ 1u, args.timeout_ns, s_abort, args.status)) {
+                if (!mbar_wait_warp_pipe(&empty[stage], phase ^ 1u, args.timeout_ns, s_abort, args.status)) {
                     ok = false;
                     break;
                 }
@@ -600,13 +621,13 @@ nvf4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a,
                 if (elect_one()) {
                     if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * C::STAGE_TX);
                     tma_load_2d_pair(smem + C::OFF_A + stage * C::A_BYTES, &tmap_a, fb,
-                                     kb * kBKBytes, mt * 256 + rank * 128, pol);
+                                     kb * KB, mt * 256 + rank * 128, pol);
                     tma_load_2d_pair(smem + C::OFF_B + stage * C::B_BYTES, &tmap_b, fb,
-                                     kb * kBKBytes, nt * BN + rank * 128, pol);
+                                     kb * KB, nt * BN + rank * 128, pol);
                     tma_load_2d_pair(smem + C::OFF_SFA + stage * C::SFA_BYTES, &tmap_sfa, fb,
-                                     kb * 256, mt * 2 + rank, pol);
+                                     kb * ATOMS * 64, mt * 2 + rank, pol);
                     tma_load_2d_pair(smem + C::OFF_SFB + stage * C::SFB_BYTES, &tmap_sfb, fb,
-                                     kb * 256, nt * 2, pol);
+                                     kb * ATOMS * 64, nt * 2, pol);
                 }
                 __syncwarp();
                 if (rank == 0) {
@@ -630,11 +651,13 @@ nvf4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a,
         __syncwarp();
     } else if (warp == 1) {
         if (rank == 0) {
-            // ---------------- MMA issuer (even CTA) ----------------
+            // ---------------- scale copies + MMA issuer (even CTA) ----------------
             constexpr uint32_t idesc = make_idesc_pair();
             // descriptor start-address fields advance by 2 per 32 bytes of K
-            const uint64_t da0 = sdesc_kmajor_sw128(smem_u32(smem + C::OFF_A));
-            const uint64_t db0 = sdesc_kmajor_sw128(smem_u32(smem + C::OFF_B));
+            const uint64_t da0 = sdesc_kmajor<KB>(smem_u32(smem + C::OFF_A));
+            const uint64_t db0 = sdesc_kmajor<KB>(smem_u32(smem + C::OFF_B));
+            const uint32_t ssfa0 = smem_u32(smem + C::OFF_SFA);
+            const uint32_t ssfb0 = smem_u32(smem + C::OFF_SFB);
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
@@ -646,25 +669,36 @@ nvf4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a,
                 }
                 tc_fence_after();
                 for (int kb = 0; kb < args.k_steps; ++kb) {
-                    if (!mbar_wait_warp(&sf_ready[stage], phase, args.timeout_ns, s_abort, args.status)) {
+                    if (!mbar_wait_warp_pipe(&full[stage], phase, args.timeout_ns, s_abort, args.status)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
                     const uint64_t da = da0 + static_cast<uint64_t>(stage * (C::A_BYTES / 16));
                     const uint64_t db = db0 + static_cast<uint64_t>(stage * (C::B_BYTES / 16));
-                    const uint32_t sfr = tmem_base + C::BN + stage * C::SF_STRIDE;
+                    const uint32_t ssfa = ssfa0 + stage * C::SFA_BYTES;
+                    const uint32_t ssfb = ssfb0 + stage * C::SFB_BYTES;
+                    const uint32_t sfr = tmem_base + BN + stage * C::SF_STRIDE;
                     const uint32_t first = kb != 0;
+                    const int natoms = kb == last_kb ? last_natoms : ATOMS;
                     if (elect_one()) {
-                        if (kb != last_kb) {
+                        // scale atoms of this stage into its TMEM region (both CTAs),
+                        // then the MMAs that read them: same thread, issue order
 #pragma unroll
-                            for (int j = 0; j < kAtomsPerStep; ++j)
+                        for (int j = 0; j < ATOMS; ++j) {
+                            if (j < natoms) {
+                                tc_copy_scales_pair(sfr + j * 4, sdesc_scales(ssfa + j * kAtom));
+                                tc_copy_scales_pair(sfr + C::SFB_COL + j * 8,
+                                                    sdesc_scales(ssfb + j * kAtom));
+                                tc_copy_scales_pair(sfr + C::SFB_COL + j * 8 + 4,
+                                                    sdesc_scales(ssfb + ATOMS * kAtom + j * kAtom));
+                            }
+                        }
+#pragma unroll
+                        for (int j = 0; j < ATOMS; ++j) {
+                            if (j < natoms)
                                 tc_mma_nvf4_pair(tmem_base, da + 2 * j, db + 2 * j, idesc, sfr + j * 4,
-                                                 sfr + 16 + j * 8, first | static_cast<uint32_t>(j));
-                        } else {
-                            for (int j = 0; j < last_natoms; ++j)
-                                tc_mma_nvf4_pair(tmem_base, da + 2 * j, db + 2 * j, idesc, sfr + j * 4,
-                                                 sfr + 16 + j * 8, first | static_cast<uint32_t>(j));
+                                                 sfr + C::SFB_COL + j * 8, first | static_cast<uint32_t>(j));
                         }
                         tc_commit_pair(&empty[stage], 0x3);
                     }
@@ -681,48 +715,6 @@ nvf4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a,
                 tc_commit_pair(drain, 0x1);
                 int local_abort = 0;
                 mbar_wait_bounded(drain, 0, args.timeout_ns, &local_abort, args.status);
-            }
-            __syncwarp();
-        }
-    } else if (warp == 2 + kEpiWarps) {
-        if (rank == 0) {
-            // ---------------- scale copies (even CTA) ----------------
-            const uint32_t ssfa0 = smem_u32(smem + C::OFF_SFA);
-            const uint32_t ssfb0 = smem_u32(smem + C::OFF_SFB);
-            int stage = 0;
-            uint32_t phase = 0;
-            bool ok = true;
-            for (int t = pair; t < total_tiles && ok; t += npairs) {
-                for (int kb = 0; kb < args.k_steps; ++kb) {
-                    if (!mbar_wait_warp(&full[stage], phase, args.timeout_ns, s_abort, args.status)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    const int natoms = kb == last_kb ? last_natoms : kAtomsPerStep;
-                    const uint32_t ssfa = ssfa0 + stage * C::SFA_BYTES;
-                    const uint32_t ssfb = ssfb0 + stage * C::SFB_BYTES;
-                    const uint32_t sfr = tmem_base + C::BN + stage * C::SF_STRIDE;
-                    if (elect_one()) {
-                        for (int j = 0; j < natoms; ++j) {
-                            tc_copy_scales_pair(sfr + j * 4, sdesc_scales(ssfa + j * kAtom));
-                            tc_copy_scales_pair(sfr + 16 + j * 8, sdesc_scales(ssfb + j * kAtom));
-                            tc_copy_scales_pair(sfr + 16 + j * 8 + 4,
-                                                sdesc_scales(ssfb + kAtomsPerStep * kAtom + j * kAtom));
-                        }
-                        tc_commit_pair(&sf_ready[stage], 0x1);
-                    }
-                    __syncwarp();
-                    if (++stage == STAGES) {
-                        stage = 0;
-                        phase ^= 1u;
-                    }
-                }
-            }
-            if (elect_one()) {
-                tc_commit_pair(drain2, 0x1);
-                int local_abort = 0;
-                mbar_wait_bounded(drain2, 0, args.timeout_ns, &local_abort, args.status);
             }
             __syncwarp();
         }
@@ -951,34 +943,36 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// [rows, row_bytes] byte matrix read in boxes of 128 bytes x box_rows rows,
-// 128-byte swizzle, zero fill out of bounds.
+// [rows, row_bytes] byte matrix read in boxes of box_bytes (128 or 64) x
+// box_rows rows, swizzled to the box width, zero fill out of bounds.
 bool make_code_map(CUtensorMap* m, const uint8_t* base, int64_t rows, int64_t row_bytes,
-                   int box_rows) {
+                   int box_rows, int box_bytes = kBKBytes) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[2] = {static_cast<cuuint64_t>(row_bytes), static_cast<cuuint64_t>(rows)};
     cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_bytes)};
-    cuuint32_t box[2] = {static_cast<cuuint32_t>(kBKBytes), static_cast<cuuint32_t>(box_rows)};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(box_bytes), static_cast<cuuint32_t>(box_rows)};
     cuuint32_t estr[2] = {1, 1};
+    const CUtensorMapSwizzle sw =
+        box_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
     CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(base), dims, strides,
-                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
 
 // Scale bytes in the tensor-core layout viewed as [row blocks, atoms * 64]
-// 8-byte units: one box of 256 units (2 KB) x box_rows row blocks is one
-// 256-element k-step of box_rows 128-row blocks.  Out-of-range row blocks and
-// k positions read as zero.
+// 8-byte units: one box of box_atoms * 64 units (box_atoms scale atoms of 512
+// bytes) x box_rows row blocks is one stage of K for box_rows 128-row blocks.
+// Out-of-range row blocks and k positions read as zero.
 bool make_sf_map(CUtensorMap* m, const uint8_t* base, int64_t rowblocks, int64_t atoms_per_rb,
-                 int box_rows) {
+                 int box_rows, int box_atoms = kAtomsPerStep) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[2] = {static_cast<cuuint64_t>(atoms_per_rb * 64),
                           static_cast<cuuint64_t>(rowblocks)};
     cuuint64_t strides[1] = {static_cast<cuuint64_t>(atoms_per_rb * kAtom)};
-    cuuint32_t box[2] = {256, static_cast<cuuint32_t>(box_rows)};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(box_atoms * 64), static_cast<cuuint32_t>(box_rows)};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT64, 2, const_cast<uint8_t*>(base), dims, strides,
                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
@@ -1029,11 +1023,11 @@ nvfp4_status launch_gemm(const uint8_t* a_codes, const uint8_t* w_codes, GemmArg
     return cuda_status(cudaGetLastError());
 }
 
-template <int STAGES, bool kSilu = false>
+template <int STAGES, int KB, bool kSilu = false>
 nvfp4_status launch_gemm_pair(const uint8_t* a_codes, const uint8_t* w_codes, GemmArgs& args,
                               const DeviceInfo& dev, cudaStream_t stream) {
-    using Cf = PairCfg<STAGES>;
-    auto kern = nvf4_gemm_pair_kernel<STAGES, kSilu>;
+    using Cf = PairCfg<STAGES, KB>;
+    auto kern = nvf4_gemm_pair_kernel<STAGES, KB, kSilu>;
     static PerDeviceOnce attr_once;
     int devid = 0;
     nvfp4_status st = current_device(&devid);
@@ -1045,10 +1039,11 @@ nvfp4_status launch_gemm_pair(const uint8_t* a_codes, const uint8_t* w_codes, Ge
     if (st != NVFP4_OK) return st;
     CUtensorMap ta, tb, tsa, tsb;
     const int64_t a_rb = (args.M + 127) / 128, w_rb = (args.N + 127) / 128;
-    if (!make_code_map(&ta, a_codes, args.M, args.K / 2, 128)) return NVFP4_ERR_CUDA;
-    if (!make_code_map(&tb, w_codes, args.N, args.K / 2, 128)) return NVFP4_ERR_CUDA;
-    if (!make_sf_map(&tsa, args.a_sf, a_rb, args.atoms_per_rb, 1)) return NVFP4_ERR_CUDA;
-    if (!make_sf_map(&tsb, args.w_sf, w_rb, args.atoms_per_rb, 2)) return NVFP4_ERR_CUDA;
+    if (!make_code_map(&ta, a_codes, args.M, args.K / 2, 128, KB)) return NVFP4_ERR_CUDA;
+    if (!make_code_map(&tb, w_codes, args.N, args.K / 2, 128, KB)) return NVFP4_ERR_CUDA;
+    if (!make_sf_map(&tsa, args.a_sf, a_rb, args.atoms_per_rb, 1, Cf::ATOMS)) return NVFP4_ERR_CUDA;
+    if (!make_sf_map(&tsb, args.w_sf, w_rb, args.atoms_per_rb, 2, Cf::ATOMS)) return NVFP4_ERR_CUDA;
+    args.k_steps = (args.K + 2 * KB - 1) / (2 * KB);
     args.m_tiles = (args.M + 255) / 256;
     args.n_tiles = (args.N + Cf::BN - 1) / Cf::BN;
     const int tiles = args.m_tiles * args.n_tiles;
@@ -1227,7 +1222,7 @@ nvfp4_status gemm_impl(const uint8_t* a_codes, const uint8_t* a_sf, const float*
     cudaStream_t cs = as_stream(stream);
     // The configuration depends on M only, so a fused GEMM and its per-module
     // GEMMs accumulate every output element identically.
-    if (M > 256) return launch_gemm_pair<5>(a_codes, w_codes, args, dev, cs);
+    if (M > 256) return launch_gemm_pair<kPairStages, kPairKB>(a_codes, w_codes, args, dev, cs);
     if (M <= kBM) return launch_gemm_decode(a_codes, w_codes, args, cs);
     return launch_gemm<128, 6, 2>(a_codes, w_codes, args, dev, cs);
 }
@@ -1285,7 +1280,7 @@ nvfp4_status gemm_silu_impl(const uint8_t* a_codes, const uint8_t* a_sf, const f
     args.h_ws = static_cast<unsigned int*>(workspace);
     args.h_g = h_g;
     args.h_amax = h_amax;
-    return launch_gemm_pair<5, true>(a_codes, w_codes, args, dev, as_stream(stream));
+    return launch_gemm_pair<kPairStages, kPairKB, true>(a_codes, w_codes, args, dev, as_stream(stream));
 }
 
 }  // namespace

@@ -135,6 +135,69 @@ __device__ __forceinline__ bool elect_one() {
     return pred != 0;
 }
 
+// Non-blocking test of a phase: never suspends the thread.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+
+// try_wait without a suspend-time hint (the system's own short limit).
+__device__ __forceinline__ bool mbar_try_wait_nohint(uint64_t* bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+
+#ifndef NVFP4_PIPE_WAIT
+#define NVFP4_PIPE_WAIT 0
+#endif
+
+// Bounded wait for the GEMM feed loop (TMA producer <-> MMA issuer), where the
+// wake-up latency of every hop adds to the time a stage stays out of use.
+__device__ __forceinline__ bool mbar_wait_pipe(uint64_t* bar, uint32_t parity, uint64_t limit_ns,
+                                               volatile int* abort, int* dev_status) {
+#if NVFP4_PIPE_WAIT == 0
+    return mbar_wait_bounded(bar, parity, limit_ns, abort, dev_status);
+#else
+    const uint64_t t0 = clock_cycles();
+    const uint64_t lim = limit_cycles(limit_ns);
+    while (true) {
+#if NVFP4_PIPE_WAIT == 1
+        if (mbar_try_wait_nohint(bar, parity)) return true;
+#else
+        if (mbar_test_wait(bar, parity)) return true;
+#endif
+        if (*abort) return false;
+        if (clock_cycles() - t0 > lim) {
+            *abort = 1;
+            atomicExch(dev_status, kDevTimeout);
+            return false;
+        }
+    }
+#endif
+}
+
+__device__ __forceinline__ bool mbar_wait_warp_pipe(uint64_t* bar, uint32_t parity,
+                                                    uint64_t limit_ns, volatile int* abort,
+                                                    int* dev_status) {
+    int ok = 1;
+    if ((threadIdx.x & 31) == 0) ok = mbar_wait_pipe(bar, parity, limit_ns, abort, dev_status);
+    return __shfl_sync(0xFFFFFFFFu, ok, 0) != 0;
+}
+
 // Bounded wait by the whole warp: lane 0 polls, the outcome is broadcast.
 __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, uint64_t limit_ns,
                                                volatile int* abort, int* dev_status) {
@@ -280,6 +343,18 @@ __device__ __forceinline__ uint64_t sdesc_kmajor_sw128(uint32_t saddr) {
     d |= static_cast<uint64_t>(1024 >> 4) << 32;             // stride between 8-row groups
     d |= static_cast<uint64_t>(1) << 46;                     // descriptor version
     d |= static_cast<uint64_t>(2) << 61;                     // 128-byte swizzle
+    return d;
+}
+
+// K-major operand tile, rows of exactly 64 bytes (128 packed FP4 values),
+// 64-byte swizzle, 8-row groups 512 bytes apart; the base must be 512-byte
+// aligned and K steps of 64 values add 32 bytes to the start address.
+__device__ __forceinline__ uint64_t sdesc_kmajor_sw64(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFF);      // start address
+    d |= static_cast<uint64_t>(512 >> 4) << 32;              // stride between 8-row groups
+    d |= static_cast<uint64_t>(1) << 46;                     // descriptor version
+    d |= static_cast<uint64_t>(4) << 61;                     // 64-byte swizzle
     return d;
 }
 
