@@ -507,7 +507,9 @@ struct PairCfg {
     static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
     static constexpr int OFF_SFA = OFF_B + STAGES * B_BYTES;
     static constexpr int OFF_SFB = OFF_SFA + STAGES * SFA_BYTES;
-    static constexpr int OFF_BAR = OFF_SFB + STAGES * SFB_BYTES;
+    static constexpr int OFF_EPI = OFF_SFB + STAGES * SFB_BYTES;  // epilogue staging, one per warp
+    static constexpr int EPI_BYTES = 32 * 64;                    // 32 rows x 32 BF16 columns
+    static constexpr int OFF_BAR = OFF_EPI + kEpiWarps * EPI_BYTES;
     static constexpr int NBAR = 2 * STAGES + 3;                  // full, empty, tmem_full, tmem_empty, drain
     static constexpr int OFF_SEG = OFF_BAR + NBAR * 8;
     static constexpr int OFF_MISC = OFF_SEG + static_cast<int>((sizeof(SegTable) + 15) / 16 * 16);
@@ -540,7 +542,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
 nvf4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a,
                       const __grid_constant__ CUtensorMap tmap_b,
                       const __grid_constant__ CUtensorMap tmap_sfa,
-                      const __grid_constant__ CUtensorMap tmap_sfb, const GemmArgs args) {
+                      const __grid_constant__ CUtensorMap tmap_sfb,
+                      const __grid_constant__ CUtensorMap tmap_y, const GemmArgs args) {
     using C = PairCfg<STAGES, KB>;
     constexpr int BN = C::BN;
     constexpr int ATOMS = C::ATOMS;
@@ -580,6 +583,7 @@ nvf4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a,
         prefetch_tmap(&tmap_b);
         prefetch_tmap(&tmap_sfa);
         prefetch_tmap(&tmap_sfb);
+        if constexpr (!kSilu) prefetch_tmap(&tmap_y);
     }
     if (warp == 1) {
         tmem_alloc_pair(s_tmem_base, C::TMEM_COLS);
@@ -809,12 +813,22 @@ nvf4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a,
             mag = __reduce_max_sync(0xFFFFFFFFu, mag);
             if (lane == 0 && mag) atomicMax(&args.h_ws[0], mag << 16);
         } else {
+        // Each warp owns TMEM lane quarter q (32 rows) and half of the 256
+        // columns.  Per 32-column chunk: alpha and gates in FP32, BF16 RNE,
+        // the 32 x 32 tile written into the warp's staging buffer in the
+        // 64-byte swizzle (conflict-free: lane i's row is 64 bytes at
+        // 64 i, its 16-byte pieces permuted by (i / 2) % 4), then one TMA store
+        // of the tile -- whole 32-byte sectors per row, rows and columns
+        // beyond M and N clipped by the tensor map.  A lane-per-row st.global
+        // would instead send 32 separate 16-byte pieces per instruction.
         constexpr int kHalf = BN / 2;
         constexpr int kChunks = kHalf / 32;
         const int q = warp & 3;
         const int half = (warp - 2) >> 2;
-        const int row = q * 32 + lane;
         const uint64_t pol_y = l2_policy_evict_first();
+        uint8_t* stage_y = smem + C::OFF_EPI + (warp - 2) * C::EPI_BYTES;
+        const uint32_t sy = smem_u32(stage_y);
+        const uint32_t swz = static_cast<uint32_t>((lane >> 1) & 3);
         int i = 0;
         for (int t = pair; t < total_tiles; t += npairs, ++i) {
             int mt, nt;
@@ -832,48 +846,59 @@ nvf4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a,
             tmem_ld_wait();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(tmem_empty_leader);
-            const int m = mt * 256 + static_cast<int>(rank) * 128 + row;
-            uint16_t* yrow = args.y + static_cast<int64_t>(m) * args.ldy;
+            // the values sit in registers: nothing of this thread is left to
+            // order before the release (the loads have completed)
+            if (lane == 0) mbar_arrive_cluster_relaxed(tmem_empty_leader);
+            const int m0 = mt * 256 + static_cast<int>(rank) * 128 + q * 32;   // row of lane 0
+            if (m0 >= args.M) continue;                                        // warp-uniform
 #pragma unroll
             for (int ch = 0; ch < kChunks; ++ch) {
                 const int n0 = nt * BN + half * kHalf + ch * 32;
+                if (n0 >= args.N) break;                                       // warp-uniform
                 int s0 = 0;
                 while (s0 < args.nseg - 1 && n0 >= s_seg_end[s0]) ++s0;
                 const bool one_seg = (s0 == args.nseg - 1) || (n0 + 31 < s_seg_end[s0]);
-                if (m < args.M && n0 < args.N) {
-                    float v[32];
-                    if (one_seg) {
-                        const float al = s_seg_alpha[s0];
+                float v[32];
+                if (one_seg) {
+                    const float al = s_seg_alpha[s0];
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) v[j] = __fmul_rn(__uint_as_float(r[ch][j]), al);
-                    } else {
-                        int s = s0;
+                    for (int j = 0; j < 32; ++j) v[j] = __fmul_rn(__uint_as_float(r[ch][j]), al);
+                } else {
+                    int s = s0;
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) {
-                            while (s < args.nseg - 1 && n0 + j >= s_seg_end[s]) ++s;
-                            v[j] = __fmul_rn(__uint_as_float(r[ch][j]), s_seg_alpha[s]);
-                        }
-                    }
-                    if (args.any_act && n0 < args.gate_hi && n0 + 32 > args.gate_lo)
-                        apply_gates<32>(v, n0, args.N, args.nseg, seg_tab);
-                    uint32_t o[16];
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) o[j] = pack_bf16x2(v[2 * j], v[2 * j + 1]);
-                    if (n0 + 32 <= args.N) {
-#pragma unroll
-                        for (int u = 0; u < 4; ++u)
-                            st_global_v4_hint(yrow + n0 + 8 * u, o[4 * u], o[4 * u + 1], o[4 * u + 2],
-                                              o[4 * u + 3], pol_y);
-                    } else {
-#pragma unroll
-                        for (int j = 0; j < 32; ++j)
-                            if (n0 + j < args.N)
-                                yrow[n0 + j] = static_cast<uint16_t>((o[j >> 1] >> (16 * (j & 1))) & 0xFFFFu);
+                    for (int j = 0; j < 32; ++j) {
+                        while (s < args.nseg - 1 && n0 + j >= s_seg_end[s]) ++s;
+                        v[j] = __fmul_rn(__uint_as_float(r[ch][j]), s_seg_alpha[s]);
                     }
                 }
+                if (args.any_act && n0 < args.gate_hi && n0 + 32 > args.gate_lo)
+                    apply_gates<32>(v, n0, args.N, args.nseg, seg_tab);
+                uint32_t o[16];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) o[j] = pack_bf16x2(v[2 * j], v[2 * j + 1]);
+                // the previous chunk's store has finished reading the buffer
+                if (ch > 0) {
+                    if (lane == 0) bulk_wait_read_all();
+                    __syncwarp();
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                    sts128(sy + lane * 64 + ((static_cast<uint32_t>(u) ^ swz) << 4), o[4 * u],
+                           o[4 * u + 1], o[4 * u + 2], o[4 * u + 3]);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    tma_store_2d(&tmap_y, stage_y, n0, m0, pol_y);
+                    bulk_commit_group();
+                }
             }
+            // the buffer is reused by the next tile's first chunk
+            if (lane == 0) bulk_wait_read_all();
+            __syncwarp();
         }
+        // every store of this warp has completed before the CTA exits
+        if (lane == 0) bulk_wait_all();
+        __syncwarp();
         }
     }
 
@@ -980,6 +1005,22 @@ bool make_sf_map(CUtensorMap* m, const uint8_t* base, int64_t rowblocks, int64_t
     return r == CUDA_SUCCESS;
 }
 
+// BF16 output [rows, cols] with row stride ld elements, written by TMA stores
+// of 32 x 32 tiles staged in the 64-byte swizzle; boxes reaching past rows or
+// cols are clipped.
+bool make_out_map(CUtensorMap* m, const uint16_t* base, int64_t rows, int64_t cols, int64_t ld) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld * 2)};
+    cuuint32_t box[2] = {32, 32};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(base), dims,
+                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                    CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 }  // namespace
 
 int* device_status_ptr() {
@@ -1037,12 +1078,14 @@ nvfp4_status launch_gemm_pair(const uint8_t* a_codes, const uint8_t* w_codes, Ge
             cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::SMEM));
     });
     if (st != NVFP4_OK) return st;
-    CUtensorMap ta, tb, tsa, tsb;
+    CUtensorMap ta, tb, tsa, tsb, ty;
     const int64_t a_rb = (args.M + 127) / 128, w_rb = (args.N + 127) / 128;
     if (!make_code_map(&ta, a_codes, args.M, args.K / 2, 128, KB)) return NVFP4_ERR_CUDA;
     if (!make_code_map(&tb, w_codes, args.N, args.K / 2, 128, KB)) return NVFP4_ERR_CUDA;
     if (!make_sf_map(&tsa, args.a_sf, a_rb, args.atoms_per_rb, 1, Cf::ATOMS)) return NVFP4_ERR_CUDA;
     if (!make_sf_map(&tsb, args.w_sf, w_rb, args.atoms_per_rb, 2, Cf::ATOMS)) return NVFP4_ERR_CUDA;
+    // the SiLU epilogue stores h directly and leaves this map unused
+    if (!make_out_map(&ty, args.y, args.M, kSilu ? args.N / 2 : args.N, args.ldy)) return NVFP4_ERR_CUDA;
     args.k_steps = (args.K + 2 * KB - 1) / (2 * KB);
     args.m_tiles = (args.M + 255) / 256;
     args.n_tiles = (args.N + Cf::BN - 1) / Cf::BN;
@@ -1061,7 +1104,7 @@ nvfp4_status launch_gemm_pair(const uint8_t* a_codes, const uint8_t* w_codes, Ge
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ta, tb, tsa, tsb, args);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ta, tb, tsa, tsb, ty, args);
     if (e != cudaSuccess) return NVFP4_ERR_CUDA;
     return cuda_status(cudaGetLastError());
 }
