@@ -98,24 +98,27 @@ global_scale_kernel(const uint8_t* __restrict__ x, int64_t rows, int64_t vec_per
 // flight), and warps walk (row, chunk) pairs with carries instead of
 // divisions.  The block max is a bf16x2 abs-max chain.
 //
-// No IEEE division on the fast path; every result still equals the binary32
-// step sequence exactly:
+// Every result equals the binary32 step sequence exactly, with no IEEE
+// division and no per-element branch on the fast path:
 //  * fl32(ab / 6): ab is BF16, i.e. (1 + m/128) * 2^e, and rounding commutes
 //    with scaling by 2^e, so it is a 128-entry table of RN((1 + m/128) / 6)
-//    with e added to the exponent (tiny ab, where that would underflow, take
-//    the IEEE division).
-//  * s8 = E4M3(fl32(u / g)): the products u*RN(1/g)*(1 -+ 2^-20) bracket the
-//    correctly rounded quotient and E4M3 rounding is monotone, so when both
-//    brackets encode to the same byte that byte is exact; otherwise the IEEE
-//    division decides.
-//  * code = E2M1(fl32(x / d)): likewise x*RN(1/d)*(1 -+ 2^-20) bracket
-//    fl32(x/d) and E2M1 rounding is monotone, so every element whose two
-//    bracket codes agree has its exact code.  The brackets disagree only for
-//    an x/d within ~2^-20 of a rounding threshold (0.25, 0.75, ..., 5); with
-//    g = amax / (21 * 2^7) such near-ties are structural rather than rare
-//    (d times a threshold often lands next to a BF16 number), so that single
-//    element -- not its block -- is recomputed with the IEEE division.
-//    Every lane runs the same instructions except for those few elements.
+//    with e added to the exponent (tiny ab take the IEEE division).
+//  * fl32(u / g) and fl32(x / d): with r = RN(1/v) and q0 = RN(a * r), the
+//    remainder a - q0 * v is exact in one FMA, and RN(q0 + (a - q0 * v) * r)
+//    is the correctly rounded quotient (Markstein's theorem: P. Markstein,
+//    "Computation of elementary functions on the IBM RISC System/6000
+//    processor", IBM J. Res. Dev. 34(1), 1990) provided no step over- or
+//    underflows.  The per-scale-byte table marks the d that keep every step in
+//    range; a block whose largest quotient could overflow, and every quotient
+//    outside those ranges, takes the IEEE division instead.
+//  * The element quotient is formed from -x (one integer operation on the
+//    BF16 bits) and -RN(1/d): q0 = (-x)(-r), e = q0 d + (-x), q = q0 + e (-r).
+//    Each step is the exact negation image of the textbook sequence, and the
+//    signed zeros come out as IEEE division gives them: x = -0 yields -0 (code
+//    0x8), x = +0 yields +0.
+// The conversions run on a narrow pipe, so each is used once per value: one
+// E2M1 pair conversion per two elements, one E4M3 pair conversion per two
+// blocks.
 //
 // Scales: four neighbouring threads' E4M3 bytes form one 32-bit word of the
 // tensor-core layout (block j of a 64-element group in byte j).
@@ -137,18 +140,10 @@ struct QuantParams {
 
 constexpr int kBlocksPerStep = 32;   // blocks per warp per load
 constexpr int kStepsPerChunk = 2;    // loads in flight per thread
-constexpr float kLo = 1.0f - 0x1p-20f;
-constexpr float kHi = 1.0f + 0x1p-20f;
 
-// UE4M3 encode (round to nearest even, saturate at 448) of a non-negative
-// float; the hardware conversion is exact RNE.
-__device__ __forceinline__ uint32_t e4m3_rne_satfinite(float s) {
-    uint16_t h;
-    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(h) : "f"(0.0f), "f"(s));
-    return h & 0xFFu;
-}
-
-// Two UE4M3 encodes at once: low byte from a, high byte from b.
+// Two UE4M3 encodes (round to nearest even, saturate at 448) of non-negative
+// floats at once: low byte from a, high byte from b.  The hardware conversion
+// is exact RNE.
 __device__ __forceinline__ uint32_t e4m3x2_rne_satfinite(float a, float b) {
     uint16_t h;
     asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(h) : "f"(b), "f"(a));
@@ -185,13 +180,21 @@ __device__ __forceinline__ uint32_t absmax_bf16x2(uint32_t a, uint32_t b) {
     return d;
 }
 
-// (a0, a1) * (r, r), each product rounded to nearest even.
-__device__ __forceinline__ void mul_f32x2(float a0, float a1, float r, float& o0, float& o1) {
-    uint64_t a, b, d;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(a) : "f"(a0), "f"(a1));
-    asm("mov.b64 %0, {%1, %1};" : "=l"(b) : "f"(r));
+// Packed pairs of binary32 values, each operation rounded to nearest even.
+__device__ __forceinline__ uint64_t f32x2(uint32_t lo, uint32_t hi) {
+    uint64_t v;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(v) : "r"(lo), "r"(hi));
+    return v;
+}
+__device__ __forceinline__ uint64_t mul_f32x2(uint64_t a, uint64_t b) {
+    uint64_t d;
     asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(o0), "=f"(o1) : "l"(d));
+    return d;
+}
+__device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
 }
 
 struct Block16 {
@@ -201,14 +204,15 @@ struct Block16 {
 // Per-CTA tables, built from g at kernel start.
 struct QuantTables {
     float div6[128];     // RN((1 + m/128) / 6)
-    float4 dq[128];      // per scale byte: d = fl32(E4M3 * g), RN(1/d)*(1 -+ 2^-20), usable
+    float4 dq[128];      // per scale byte: d = fl32(E4M3 * g), -RN(1/d), the largest block
+                         // max the fast path takes (0: never), unused
 };
 
 // Kernel-wide constants derived from g.
 struct ScaleConsts {
     float g;
-    float rg_lo, rg_hi;   // RN(1/g) * (1 -+ 2^-20)
-    bool fast;            // g and 1/g in the normal range: the bracket argument holds
+    float rg;             // RN(1/g)
+    bool fast;            // g and 1/g in the normal range
 };
 
 __device__ __forceinline__ bool normal_range(float v) {
@@ -216,71 +220,70 @@ __device__ __forceinline__ bool normal_range(float v) {
     return a >= 0x1p-125f && a <= 0x1p125f;
 }
 
-__device__ __forceinline__ uint32_t block_scale(float ab, const QuantTables& T,
+// fl32(fl32(ab / 6) / g), clamped to 1024 (any value from 464 up encodes to
+// 448, so the clamp changes no scale byte and keeps overflow away from the
+// encoder).  Fast path: ab >= 2^-97 (so fl32(ab/6) >= 2^-100 and the table
+// holds it) and g, 1/g normal; everything else divides.
+__device__ __forceinline__ float block_quotient(float ab, const QuantTables& T,
                                                 const ScaleConsts& K) {
     const uint32_t abits = __float_as_uint(ab);
-    if (abits == 0) return 0u;
-    if (K.fast && abits >= 0x04000000u) {                 // ab >= 2^-119: exact table path
+    float q;
+    if (K.fast && abits >= 0x0F000000u) {
         const uint32_t e = abits >> 23, m7 = (abits >> 16) & 127u;
         const float u = __uint_as_float(__float_as_uint(T.div6[m7]) + ((e - 127u) << 23));
-        const uint32_t both = e4m3x2_rne_satfinite(__fmul_rn(u, K.rg_lo), __fmul_rn(u, K.rg_hi));
-        if ((both & 0xFFu) == (both >> 8)) return both & 0xFFu;
-        return e4m3_rne_satfinite(__fdiv_rn(u, K.g));
+        const float q0 = __fmul_rn(u, K.rg);
+        const float r = __fmaf_rn(-q0, K.g, u);
+        q = __fmaf_rn(r, K.rg, q0);
+    } else {
+        if (abits == 0) return 0.0f;
+        const float u = abits >= 0x04000000u   // ab >= 2^-119: exact table path
+            ? __uint_as_float(__float_as_uint(T.div6[(abits >> 16) & 127u]) + (((abits >> 23) - 127u) << 23))
+            : __fdiv_rn(ab, 6.0f);
+        q = __fdiv_rn(u, K.g);
     }
-    return e4m3_rne_satfinite(__fdiv_rn(__fdiv_rn(ab, 6.0f), K.g));
+    return fminf(q, 1024.0f);
 }
 
-// One E2M1 code (low nibble) of fl32(x / d) by the IEEE division.
-__device__ __forceinline__ uint32_t e2m1_exact(float x, float d) {
-    uint16_t h;
-    asm("{\n\t.reg .b8 q;\n\tcvt.rn.satfinite.e2m1x2.f32 q, %1, %2;\n\tcvt.u16.u8 %0, q;\n\t}"
-        : "=h"(h)
-        : "f"(0.0f), "f"(__fdiv_rn(x, d)));
-    return h & 0xFu;
+// 16 E2M1 codes of fl32(x / d) for one block whose scale byte is s8.
+__device__ __forceinline__ void encode_block(const Block16& b, float ab, uint32_t s8,
+                                             const QuantTables& T, uint32_t (&c)[2]) {
+    const float4 q = T.dq[s8];
+    const float d = q.x;
+    float t[16];
+    if (ab < q.z) {
+        // d and 1/d in range and no quotient of the block can overflow
+        const uint64_t NR = f32x2(__float_as_uint(q.y), __float_as_uint(q.y));
+        const uint64_t D = f32x2(__float_as_uint(d), __float_as_uint(d));
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const uint32_t w = b.w[i];
+            // -x of both elements: the BF16 bits moved into place, sign flipped
+            const uint64_t nx = f32x2(w * 0x10000u + 0x80000000u, (w & 0xFFFF0000u) ^ 0x80000000u);
+            const uint64_t q0 = mul_f32x2(nx, NR);
+            const uint64_t e = fma_f32x2(q0, D, nx);
+            const uint64_t q1 = fma_f32x2(e, NR, q0);
+            t[2 * i] = __uint_as_float(static_cast<uint32_t>(q1));
+            t[2 * i + 1] = __uint_as_float(static_cast<uint32_t>(q1 >> 32));
+        }
+    } else if (d == 0.0f) {
+        c[0] = c[1] = 0;     // zero block or a scale that underflowed: every code 0
+        return;
+    } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            t[2 * i] = __fdiv_rn(__uint_as_float(b.w[i] << 16), d);
+            t[2 * i + 1] = __fdiv_rn(__uint_as_float(b.w[i] & 0xFFFF0000u), d);
+        }
+    }
+    c[0] = e2m1x8(t);
+    c[1] = e2m1x8(t + 8);
 }
 
-// Quantize one block: returns the E4M3 scale byte, writes 16 codes to c[2].
-__device__ __forceinline__ uint32_t quantize_block(const Block16& b, const QuantTables& T,
-                                                   const ScaleConsts& K, uint32_t (&c)[2]) {
+__device__ __forceinline__ float block_absmax(const Block16& b) {
     uint32_t m = absmax_bf16x2(b.w[0], b.w[1]);
 #pragma unroll
     for (int i = 2; i < 8; ++i) m = absmax_bf16x2(m, b.w[i]);
-    const float ab = __uint_as_float(max(m & 0x7FFFu, (m >> 16) & 0x7FFFu) << 16);
-    const uint32_t s8 = block_scale(ab, T, K);
-    const float4 q = T.dq[s8];
-    const float d = q.x;
-    c[0] = c[1] = 0;
-    if (d == 0.0f) return s8;
-    float x[16], t[16];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        x[2 * i] = __uint_as_float(b.w[i] << 16);
-        x[2 * i + 1] = __uint_as_float(b.w[i] & 0xFFFF0000u);
-    }
-    if (q.w != 0.0f) {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) mul_f32x2(x[2 * i], x[2 * i + 1], q.y, t[2 * i], t[2 * i + 1]);
-        c[0] = e2m1x8(t);
-        c[1] = e2m1x8(t + 8);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) mul_f32x2(x[2 * i], x[2 * i + 1], q.z, t[2 * i], t[2 * i + 1]);
-        const uint32_t diff0 = c[0] ^ e2m1x8(t), diff1 = c[1] ^ e2m1x8(t + 8);
-        if ((diff0 | diff1) == 0) return s8;
-        // near-tie elements only: the IEEE quotient decides
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const uint32_t sh = 4 * (i & 7);
-            uint32_t& ci = c[i >> 3];
-            if ((((i < 8) ? diff0 : diff1) >> sh) & 0xFu)
-                ci = (ci & ~(0xFu << sh)) | (e2m1_exact(x[i], d) << sh);
-        }
-        return s8;
-    }
-#pragma unroll
-    for (int i = 0; i < 16; ++i) t[i] = __fdiv_rn(x[i], d);
-    c[0] = e2m1x8(t);
-    c[1] = e2m1x8(t + 8);
-    return s8;
+    return __uint_as_float(max(m & 0x7FFFu, (m >> 16) & 0x7FFFu) << 16);
 }
 
 template <bool kWide>
@@ -297,84 +300,116 @@ __device__ __forceinline__ void load_block(const uint8_t* p, Block16& b) {
     }
 }
 
-template <bool kWide>
-__global__ void __launch_bounds__(kThreads, 4) quantize_kernel(QuantParams p) {
+#ifndef NVFP4_Q_MINB
+#define NVFP4_Q_MINB 3
+#endif
+// Resident CTAs of the quantizer per SM (one wave of the grid).
+constexpr int kQuantCtasPerSm = NVFP4_Q_MINB;
+
+// A warp quantizes chunks of 64 consecutive blocks of one row: lane l holds
+// blocks l and 32 + l (each load instruction reads 1 KB of contiguous bytes
+// and each code store writes 256).  Warps walk (row, chunk) pairs with the
+// grid's warp count as stride, carrying rows instead of dividing, and load
+// the next chunk while the current one is quantized.  The row is uniform over
+// the warp, so the checks for padding rows are uniform branches.  kFull: the
+// blocks per row are a multiple of 64, so no chunk is ragged.
+template <bool kWide, bool kFull>
+__device__ __forceinline__ void load_chunk(const QuantParams& p, uint32_t rl, uint32_t ch,
+                                           int lane, Block16 (&dst)[kStepsPerChunk]) {
+    const int64_t nblk = p.cols / 16;
+    const uint8_t* xrow = p.x + static_cast<int64_t>(rl) * p.ld_bytes;
+    const int64_t b0 = static_cast<int64_t>(ch) * (kBlocksPerStep * kStepsPerChunk) + lane;
+    if (kFull && rl < p.rows) {
+#pragma unroll
+        for (int u = 0; u < kStepsPerChunk; ++u) load_block<kWide>(xrow + (b0 + u * kBlocksPerStep) * 32, dst[u]);
+        return;
+    }
+#pragma unroll
+    for (int u = 0; u < kStepsPerChunk; ++u) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) dst[u].w[i] = 0;
+        const int64_t b = b0 + u * kBlocksPerStep;
+        if (rl < p.rows && b < nblk) load_block<kWide>(xrow + b * 32, dst[u]);
+    }
+}
+
+template <bool kWide, bool kFull>
+__global__ void __launch_bounds__(kThreads, kQuantCtasPerSm) quantize_kernel(QuantParams p) {
     const int lane = threadIdx.x & 31;
     const uint32_t warp = (blockIdx.x * kThreads + threadIdx.x) >> 5;
     const uint32_t nwarps = (gridDim.x * kThreads) >> 5;
     const int64_t code_row_bytes = p.cols / 2;
-    const int64_t sfcols = p.cols / 16;
     const int64_t nblk = p.cols / 16;
 
     __shared__ QuantTables T;
     ScaleConsts K;
     K.g = *p.g;
-    const float rg = __fdiv_rn(1.0f, K.g);
-    K.rg_lo = __fmul_rn(rg, kLo);
-    K.rg_hi = __fmul_rn(rg, kHi);
-    K.fast = normal_range(rg) && normal_range(K.g);
+    K.rg = __fdiv_rn(1.0f, K.g);
+    K.fast = normal_range(K.rg) && normal_range(K.g);
     for (int i = threadIdx.x; i < 128; i += kThreads) {
         T.div6[i] = __fdiv_rn(1.0f + static_cast<float>(i) * 0.0078125f, 6.0f);
-        // per scale byte: d, the two bracketing reciprocals, and whether they
-        // are usable (1/d in the normal range); otherwise the block divides
+        // per scale byte: d, -RN(1/d), and the block max below which the fast
+        // path is exact: d in [2^-96, 2^100] and ab * RN(1/d) < 2^126
         const float d = __fmul_rn(e4m3_decode(static_cast<uint32_t>(i)), K.g);
-        const bool usable = (i != 0) && (i != 127) && d >= 0x1p-120f && d <= 0x1p120f;
-        const float rd = usable ? __fdiv_rn(1.0f, d) : 0.0f;
-        T.dq[i] = make_float4(d, __fmul_rn(rd, kLo), __fmul_rn(rd, kHi), usable ? 1.0f : 0.0f);
+        const bool usable = (i != 0) && (i != 127) && d >= 0x1p-96f && d <= 0x1p100f;
+        T.dq[i] = make_float4(d, usable ? -__fdiv_rn(1.0f, d) : 0.0f,
+                              usable ? __fmul_rn(d, 0x1p125f) : 0.0f, 0.0f);
     }
     __syncthreads();
 
-    // Walk (row, chunk) pairs with a stride of nwarps chunks, carrying rows
-    // instead of dividing.  Software-pipelined: the next chunk's loads are in
-    // flight while the current chunk is quantized.
     const uint32_t cpr = p.chunks_per_row;
     const uint32_t step_r = nwarps / cpr, step_c = nwarps - step_r * cpr;
     uint32_t rl = warp / cpr, ch = warp - rl * cpr;
     Block16 cur[kStepsPerChunk], nxt[kStepsPerChunk];
-    auto load_chunk = [&](uint32_t lr, uint32_t lc, Block16 (&dst)[kStepsPerChunk]) {
-        const bool ok = lr < p.rows;
-        const uint8_t* xrow = p.x + static_cast<int64_t>(lr) * p.ld_bytes;
-        const int64_t b0 = static_cast<int64_t>(lc) * (kBlocksPerStep * kStepsPerChunk) + lane;
-#pragma unroll
-        for (int u = 0; u < kStepsPerChunk; ++u) {
-            const int64_t b = b0 + u * kBlocksPerStep;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) dst[u].w[i] = 0;
-            if (ok && b < nblk) load_block<kWide>(xrow + b * 32, dst[u]);
-        }
-    };
-    if (rl < p.rows_walk) load_chunk(rl, ch, cur);
+    if (rl < p.rows_walk) load_chunk<kWide, kFull>(p, rl, ch, lane, cur);
     while (rl < p.rows_walk) {
         uint32_t nr = rl + step_r, nc = ch + step_c;
         if (nc >= cpr) {
             nc -= cpr;
             ++nr;
         }
-        if (nr < p.rows_walk) load_chunk(nr, nc, nxt);
-        const bool row_ok = rl < p.rows;
+        if (nr < p.rows_walk) load_chunk<kWide, kFull>(p, nr, nc, lane, nxt);
+
+        static_assert(kStepsPerChunk == 2, "scale bytes are converted and gathered in pairs");
+        const float ab0 = block_absmax(cur[0]), ab1 = block_absmax(cur[1]);
+        // s8 of block l (low byte) and of block 32 + l (high byte)
+        const uint32_t s8pair = e4m3x2_rne_satfinite(block_quotient(ab0, T, K), block_quotient(ab1, T, K));
+        uint32_t c0[2], c1[2];
+        encode_block(cur[0], ab0, s8pair & 0xFFu, T, c0);
+        encode_block(cur[1], ab1, s8pair >> 8, T, c1);
+
         const int64_t r = p.row0 + rl;                               // row of the whole tensor
         const int64_t b0 = static_cast<int64_t>(ch) * (kBlocksPerStep * kStepsPerChunk) + lane;
-        uint8_t* crow = p.codes + r * code_row_bytes;
-        const uint64_t sf_row = (static_cast<uint64_t>(r >> 7) * p.sf_groups) * 512u +
-                                static_cast<uint64_t>(r & 31) * 16u +
-                                static_cast<uint64_t>((r >> 5) & 3) * 4u;
-#pragma unroll
-        for (int u = 0; u < kStepsPerChunk; ++u) {
-            const int64_t b = b0 + u * kBlocksPerStep;
-            uint32_t c[2];
-            const uint32_t s8 = quantize_block(cur[u], T, K, c);
-            if (row_ok && b < nblk)
-                *reinterpret_cast<uint2*>(crow + b * 8) = make_uint2(c[0], c[1]);
-            uint32_t w = s8 << (8 * (lane & 3));
-            w |= __shfl_xor_sync(0xFFFFFFFFu, w, 1);
-            w |= __shfl_xor_sync(0xFFFFFFFFu, w, 2);
-            if (p.layout == NVFP4_SF_TCGEN05) {
-                const int64_t unit = b >> 2;
-                if ((lane & 3) == 0 && unit < p.sf_groups)
-                    *reinterpret_cast<uint32_t*>(p.sf + sf_row + unit * 512u) = w;
-            } else if (row_ok && b < nblk) {
-                p.sf[r * sfcols + b] = static_cast<uint8_t>(s8);
+        if (rl < p.rows) {
+            uint8_t* crow = p.codes + r * code_row_bytes;
+            if (kFull || b0 < nblk) *reinterpret_cast<uint2*>(crow + b0 * 8) = make_uint2(c0[0], c0[1]);
+            if (kFull || b0 + kBlocksPerStep < nblk)
+                *reinterpret_cast<uint2*>(crow + (b0 + kBlocksPerStep) * 8) = make_uint2(c1[0], c1[1]);
+        }
+        if (p.layout == NVFP4_SF_TCGEN05) {
+            // One word of the tensor-core layout is the scale bytes of four
+            // consecutive blocks (lanes 4j..4j+3 of one step).  Both steps'
+            // words are gathered with two shuffles: lane 4j stores the step-0
+            // word of unit j, lane 4j+2 the step-1 word of unit 8 + j.
+            const uint32_t v = (s8pair & 0xFFu) | ((s8pair & 0xFF00u) << 8);   // bytes s0, 0, s1, 0
+            uint32_t x = v << (8 * (lane & 1));
+            x |= __shfl_xor_sync(0xFFFFFFFFu, x, 1);                       // s0 s0' s1 s1' of a lane pair
+            const uint32_t y = __shfl_xor_sync(0xFFFFFFFFu, x, 2);
+            const int64_t unit0 = static_cast<int64_t>(ch) * 16 + (lane >> 2);
+            const uint64_t sf_row = (static_cast<uint64_t>(r >> 7) * p.sf_groups) * 512u +
+                                    static_cast<uint64_t>(r & 31) * 16u +
+                                    static_cast<uint64_t>((r >> 5) & 3) * 4u;
+            if ((lane & 3) == 0) {
+                if (kFull || unit0 < p.sf_groups)
+                    *reinterpret_cast<uint32_t*>(p.sf + sf_row + unit0 * 512u) = __byte_perm(x, y, 0x5410);
+            } else if ((lane & 3) == 2) {
+                if (kFull || unit0 + 8 < p.sf_groups)
+                    *reinterpret_cast<uint32_t*>(p.sf + sf_row + (unit0 + 8) * 512u) = __byte_perm(y, x, 0x7632);
             }
+        } else if (rl < p.rows) {
+            if (kFull || b0 < nblk) p.sf[r * nblk + b0] = static_cast<uint8_t>(s8pair);
+            if (kFull || b0 + kBlocksPerStep < nblk)
+                p.sf[r * nblk + b0 + kBlocksPerStep] = static_cast<uint8_t>(s8pair >> 8);
         }
 #pragma unroll
         for (int u = 0; u < kStepsPerChunk; ++u) cur[u] = nxt[u];
@@ -540,9 +575,15 @@ nvfp4_status quantize_impl(const void* x, int64_t rows, int64_t cols, int64_t ld
     size_t sf_total = 0;
     const nvfp4_status sfst = nvfp4_sf_bytes(total_rows, cols, layout, &sf_total);
     if (sfst != NVFP4_OK) return sfst;
-    if (overlaps(g, 4, codes, static_cast<size_t>(total_rows) * static_cast<size_t>(cols / 2)) ||
-        overlaps(g, 4, sf, sf_total))
+    const size_t code_total = static_cast<size_t>(total_rows) * static_cast<size_t>(cols / 2);
+    if (overlaps(g, 4, codes, code_total) || overlaps(g, 4, sf, sf_total))
         return NVFP4_ERR_INVALID_ARG;
+    // CTAs read x while others write codes and scales: outputs may not alias it
+    {
+        const size_t xbytes = extent_bytes(rows, ld, cols, 2);
+        if (overlaps(x, xbytes, codes, code_total) || overlaps(x, xbytes, sf, sf_total))
+            return NVFP4_ERR_INVALID_ARG;
+    }
     QuantParams p;
     p.x = static_cast<const uint8_t*>(x);
     p.ld_bytes = ld * 2;
@@ -553,25 +594,28 @@ nvfp4_status quantize_impl(const void* x, int64_t rows, int64_t cols, int64_t ld
     p.sf = sf;
     p.layout = layout;
     p.row0 = row_offset;
-    const int64_t units = (cols + 63) / 64;
+    const int64_t units = (cols + 63) / 64;                 // = roundup(cols/16, 4) / 4
     const int64_t chunks_per_row = (cols / 16 + kBlocksPerStep * kStepsPerChunk - 1) /
                                    (kBlocksPerStep * kStepsPerChunk);
     if (rows_walk * chunks_per_row >= (int64_t(1) << 30)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
     p.rows_walk = static_cast<uint32_t>(rows_walk);
     p.chunks_per_row = static_cast<uint32_t>(chunks_per_row);
-    p.sf_groups = static_cast<uint32_t>(units);  // roundup(cols/16, 4) / 4
+    p.sf_groups = static_cast<uint32_t>(units);
     DeviceInfo dev;
     nvfp4_status st = current_device_info(&dev);
     if (st != NVFP4_OK) return st;
     const int64_t warps = rows_walk * chunks_per_row;
     int64_t blocks = (warps + kWarpsPerBlock - 1) / kWarpsPerBlock;
-    const int64_t max_blocks = static_cast<int64_t>(dev.sms) * 4;   // one resident wave
+    const int64_t max_blocks = static_cast<int64_t>(dev.sms) * kQuantCtasPerSm;   // one resident wave
     if (blocks > max_blocks) blocks = max_blocks;
     const bool wide = x && (reinterpret_cast<uintptr_t>(x) % 32 == 0) && (ld % 16 == 0);
-    if (wide)
-        quantize_kernel<true><<<static_cast<int>(blocks), kThreads, 0, as_stream(stream)>>>(p);
-    else
-        quantize_kernel<false><<<static_cast<int>(blocks), kThreads, 0, as_stream(stream)>>>(p);
+    const bool full = (cols / 16) % (kBlocksPerStep * kStepsPerChunk) == 0;
+    const dim3 grid(static_cast<unsigned>(blocks)), block(kThreads);
+    cudaStream_t cs = as_stream(stream);
+    if (wide && full) quantize_kernel<true, true><<<grid, block, 0, cs>>>(p);
+    else if (wide) quantize_kernel<true, false><<<grid, block, 0, cs>>>(p);
+    else if (full) quantize_kernel<false, true><<<grid, block, 0, cs>>>(p);
+    else quantize_kernel<false, false><<<grid, block, 0, cs>>>(p);
     return cuda_status(cudaGetLastError());
 }
 

@@ -34,6 +34,9 @@ def test_header_declares_the_path():
 
 UTILITIES = {"nvfp4_sf_bytes", "nvfp4_last_device_status", "nvfp4_debug_wait_timeout",
              "nvfp4_status_string", "nvfp4_version"}
+# entries that serve the library's callers rather than a step of the method:
+# their comment says the pages have no counterpart instead of citing one
+LIBRARY_ONLY = {"nvfp4_global_scale_noalloc"}
 
 
 def test_every_computational_entry_documents_its_source_and_errors():
@@ -47,7 +50,10 @@ def test_every_computational_entry_documents_its_source_and_errors():
         found.add(name)
         if name in UTILITIES:
             continue
-        assert "Source" in comment, f"{name}: no source passage"
+        if name in LIBRARY_ONLY:
+            assert "Source" not in comment and "No passage of the pages" in comment, name
+        else:
+            assert "Source" in comment, f"{name}: no source passage"
         assert "Errors" in comment or "errors" in comment, f"{name}: no error behaviour"
     assert set(declared_functions()) - found <= {"nvfp4_kv_quantize_e4m3"}   # shares the KV block
 
@@ -263,6 +269,11 @@ def test_extents_that_would_overflow_are_refused(L):
         _lib.NVFP4_ERR_UNSUPPORTED_SHAPE
     assert L.nvfp4_quantize(FAKE, big, 64, wide, FAKE, FAKE, FAKE, 1, NUL) == \
         _lib.NVFP4_ERR_UNSUPPORTED_SHAPE
+    # 2^30 work items (1024-element chunks, padding rows included): beyond the
+    # quantizer's walk bound, though the extents are fine
+    P = ctypes.c_void_p
+    assert L.nvfp4_quantize(FAKE, 1 << 26, 16384, 16384, P(1 << 44), P(1 << 42), P(1 << 43), 1, NUL) == \
+        _lib.NVFP4_ERR_UNSUPPORTED_SHAPE
     assert L.nvfp4_quantize_slice(FAKE, 4, 64, 64, FAKE, FAKE, FAKE, 1, 1 << 62, 1 << 62, NUL) == \
         _lib.NVFP4_ERR_INVALID_ARG                                              # offset + rows wraps
     assert L.nvfp4_kv_quantize_e4m3(FAKE, big, 64, wide, FAKE, FAKE, 64, NUL) == \
@@ -299,6 +310,9 @@ def test_scalars_aliasing_an_output_are_refused(L):
     # quantize: g inside the codes, or inside the scale bytes
     assert L.nvfp4_quantize(FAKE, 4, 64, 64, P(OUT + 16), P(OUT), P(OUT2), 1, NUL) == _lib.NVFP4_ERR_INVALID_ARG
     assert L.nvfp4_quantize(FAKE, 4, 64, 64, P(OUT2 + 256), P(OUT), P(OUT2), 1, NUL) == _lib.NVFP4_ERR_INVALID_ARG
+    # quantize: the codes, or the scale bytes, inside x (4 x 64 BF16 = 512 B)
+    assert L.nvfp4_quantize(P(OUT), 4, 64, 64, P(0x20000), P(OUT + 256), P(OUT2), 1, NUL) == _lib.NVFP4_ERR_INVALID_ARG
+    assert L.nvfp4_quantize(P(OUT), 4, 64, 64, P(0x20000), P(OUT2), P(OUT + 496), 1, NUL) == _lib.NVFP4_ERR_INVALID_ARG
     # global scale: g_out inside x
     assert L.nvfp4_global_scale(P(OUT), 4, 64, 64, P(OUT + 256), NUL, FAKE, NUL) == _lib.NVFP4_ERR_INVALID_ARG
     # GEMM: the activation's scale inside y (4 x 128 BF16 = 1 KB)
@@ -345,7 +359,20 @@ def test_fused_linear_host_rejects_bad_arguments_before_enqueuing(L):
     assert f(H, 4, 64, FAKE, FAKE, segs, 2, H, *same, NUL) == _lib.NVFP4_ERR_INVALID_ARG
     g_in_codes = scratch[:3] + (P(0x200010),) + scratch[4:]  # a_g inside a_codes
     assert f(H, 4, 64, FAKE, FAKE, segs, 2, H, *g_in_codes, NUL) == _lib.NVFP4_ERR_INVALID_ARG
+    codes_in_x = scratch[:1] + (P(0x100100),) + scratch[2:]  # a_codes inside x_dev (512 B)
+    assert f(H, 4, 64, FAKE, FAKE, segs, 2, H, *codes_in_x, NUL) == _lib.NVFP4_ERR_INVALID_ARG
+    sf_in_x = scratch[:2] + (P(0x1001F0),) + scratch[3:]     # a_sf reaching into x_dev
+    assert f(H, 4, 64, FAKE, FAKE, segs, 2, H, *sf_in_x, NUL) == _lib.NVFP4_ERR_INVALID_ARG
     assert f(H, 0, 64, FAKE, FAKE, segs, 2, H, *scratch, NUL) == _lib.NVFP4_OK                     # M = 0
+    # the overlapped form makes the same checks before enqueuing anything
+    o = L.nvfp4_fused_linear_host_overlap
+    assert o(H, 4, 48, FAKE, FAKE, segs, 2, H, *scratch, NUL, NUL) == _lib.NVFP4_ERR_UNSUPPORTED_SHAPE
+    assert o(H, 4, 64, FAKE, FAKE, odd, 2, H, *scratch, NUL, NUL) == _lib.NVFP4_ERR_ALIGNMENT
+    assert o(H, 4, 64, FAKE, FAKE, gap, 2, H, *scratch, NUL, NUL) == _lib.NVFP4_ERR_INVALID_ARG
+    assert o(NUL, 4, 64, FAKE, FAKE, segs, 2, H, *scratch, NUL, NUL) == _lib.NVFP4_ERR_INVALID_ARG
+    assert o(H, 4, 64, FAKE, FAKE, segs, 2, H, *same, NUL, NUL) == _lib.NVFP4_ERR_INVALID_ARG
+    assert o(H, 4, 64, FAKE, FAKE, segs, 2, H, *codes_in_x, NUL, NUL) == _lib.NVFP4_ERR_INVALID_ARG
+    assert o(H, 0, 64, FAKE, FAKE, segs, 2, H, *scratch, NUL, NUL) == _lib.NVFP4_OK
 
 
 def test_unused_gate_parameters_are_not_checked_for_aliasing(L):
