@@ -146,7 +146,8 @@ nvfp4_status nvfp4_global_scale(const void* x, int64_t rows, int64_t cols, int64
  * array, which keeps the last call's contents: calls that overlap on the GPU
  * (different streams, no ordering between them) race and may return a wrong
  * g; serialize them.  Arguments, results, requirements and errors as
- * nvfp4_global_scale, without `workspace`.  Source: as nvfp4_global_scale. */
+ * nvfp4_global_scale, without `workspace`.  No passage of the pages defines
+ * this entry point: it exists for callers of the library, not for the method. */
 nvfp4_status nvfp4_global_scale_noalloc(const void* x, int64_t rows, int64_t cols, int64_t ld,
                                         float* g_out, float* amax_out, void* stream);
 
@@ -360,7 +361,7 @@ nvfp4_status nvfp4_kv_quantize_e4m3(const void* x, int64_t rows, int64_t cols, i
  * Every check of the three composed calls is made before anything is
  * enqueued, so a refused call enqueues nothing.  Requirements: K % 32 == 0,
  * N % 8 == 0, device pointers 16-byte aligned, no scalar inside an output
- * and x_dev apart from y_dev.
+ * and x_dev apart from y_dev, a_codes and a_sf.
  * Errors: NVFP4_ERR_INVALID_ARG, NVFP4_ERR_ALIGNMENT,
  * NVFP4_ERR_UNSUPPORTED_SHAPE, NVFP4_ERR_DEVICE, as the composed calls;
  * NVFP4_ERR_CUDA when a copy or a launch fails.  M == 0 enqueues nothing.
@@ -372,6 +373,33 @@ nvfp4_status nvfp4_fused_linear_host(const void* x_host, int64_t M, int64_t K,
                                      const nvfp4_segment* segs, int nseg, void* y_host,
                                      void* x_dev, uint8_t* a_codes, uint8_t* a_sf, float* a_g,
                                      float* a_amax, void* workspace, void* y_dev, void* stream);
+
+/* nvfp4_fused_linear_host with its copy out on a second stream, so that the
+ * PCIe transfers overlap the kernels and each other.  On `stream`: the copy in,
+ * the global scale and the quantization; then the GEMM in row slices (about
+ * 2048 rows each, a multiple of 256; with M <= 3072 one slice), each slice's
+ * copy of y_dev to y_host issued on `copy_stream` as soon as that slice's
+ * GEMM is done, while the next slice computes.  Before the first slice
+ * rewrites y_dev, `stream` waits for everything already enqueued on
+ * copy_stream (the previous call's copy out of y_dev), so consecutive calls
+ * may reuse one set of device buffers: call i + 1's copy in and quantization
+ * run while call i's output is still being copied out (the link is full
+ * duplex).  Every slice runs the GEMM kernel that the whole M selects, so y
+ * equals nvfp4_fused_linear_host's output bit for bit.
+ *   Buffers, requirements and errors as nvfp4_fused_linear_host.  x_host must
+ *   stay unchanged until `stream` has passed the copy in; y_host holds the
+ *   output once `copy_stream` has passed this call's copies (synchronize it,
+ *   or record an event on it); a caller that rewrites or reads y_host between
+ *   calls orders that against copy_stream.  copy_stream may equal stream (the
+ *   call then runs in series).  The call creates one CUDA event and releases
+ *   it before returning; it allocates no device memory.
+ * Source: as nvfp4_fused_linear_host. */
+nvfp4_status nvfp4_fused_linear_host_overlap(const void* x_host, int64_t M, int64_t K,
+                                             const uint8_t* w_codes, const uint8_t* w_sf,
+                                             const nvfp4_segment* segs, int nseg, void* y_host,
+                                             void* x_dev, uint8_t* a_codes, uint8_t* a_sf,
+                                             float* a_g, float* a_amax, void* workspace,
+                                             void* y_dev, void* stream, void* copy_stream);
 
 /* MLP intermediate for the W4A4 down projection: h[r, c] = BF16_RNE(
  * fl32(SiLU(gate) * up)) with gate = gate_up[r, c], up = gate_up[r, f + c]

@@ -408,13 +408,18 @@ class HostLinearScratch:
 
 
 def linear_host(x_host: torch.Tensor, w, y_host: Optional[torch.Tensor] = None,
-                scratch: Optional[HostLinearScratch] = None, stream=None) -> torch.Tensor:
+                scratch: Optional[HostLinearScratch] = None, stream=None,
+                copy_stream=None) -> torch.Tensor:
     """The W4A4 linear layer from a host BF16 activation [M, K] to a host BF16
-    output [M, N] through one C-ABI call (nvfp4_fused_linear_host): copy in,
-    global scale, quantization, fused GEMM against the pre-quantized weight
-    (FusedWeight or QuantizedTensor), copy out.  The copies are asynchronous
-    when the host tensors are page-locked: synchronize `stream` before
-    reading y_host."""
+    output [M, N] through one C-ABI call: copy in, global scale, quantization,
+    fused GEMM against the pre-quantized weight (FusedWeight or
+    QuantizedTensor), copy out.  Without `copy_stream` everything runs on
+    `stream` (nvfp4_fused_linear_host): synchronize it before reading y_host.
+    With `copy_stream` (nvfp4_fused_linear_host_overlap) the output is copied
+    out on that stream in row slices while the GEMM proceeds, and consecutive
+    calls overlap one call's copy out with the next one's copy in: y_host is
+    ready once copy_stream has passed the call.  The copies are asynchronous
+    when the host tensors are page-locked."""
     if not isinstance(x_host, torch.Tensor) or x_host.dtype != torch.bfloat16 or x_host.dim() != 2 \
             or x_host.is_cuda or not x_host.is_contiguous():
         raise ValueError("x_host must be a contiguous 2-D bfloat16 host tensor")
@@ -444,10 +449,14 @@ def linear_host(x_host: torch.Tensor, w, y_host: Optional[torch.Tensor] = None,
     _check_devices(w_codes=w.codes, w_sf=w.sf, x=scratch.x, codes=scratch.codes, sf=scratch.sf,
                    g=scratch.g, workspace=scratch.workspace, y=scratch.y,
                    **{f"segments[{i}] g": g for i, (_, _, g) in enumerate(segments)})
-    _lib.check("nvfp4_fused_linear_host", _lib.lib().nvfp4_fused_linear_host(
-        _ptr(x_host), M, K, _ptr(w.codes), _ptr(w.sf), _segment_array(segments), len(segments),
-        _ptr(y_host), _ptr(scratch.x), _ptr(scratch.codes), _ptr(scratch.sf), _ptr(scratch.g),
-        _ptr(scratch.amax), _ptr(scratch.workspace), _ptr(scratch.y), _stream(stream)))
+    args = (_ptr(x_host), M, K, _ptr(w.codes), _ptr(w.sf), _segment_array(segments), len(segments),
+            _ptr(y_host), _ptr(scratch.x), _ptr(scratch.codes), _ptr(scratch.sf), _ptr(scratch.g),
+            _ptr(scratch.amax), _ptr(scratch.workspace), _ptr(scratch.y), _stream(stream))
+    if copy_stream is None:
+        _lib.check("nvfp4_fused_linear_host", _lib.lib().nvfp4_fused_linear_host(*args))
+    else:
+        _lib.check("nvfp4_fused_linear_host_overlap",
+                   _lib.lib().nvfp4_fused_linear_host_overlap(*args, _stream(copy_stream)))
     return y_host
 
 

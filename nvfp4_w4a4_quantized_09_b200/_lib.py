@@ -58,6 +58,8 @@ SIGNATURES = {
     "nvfp4_silu_mul": (ST, [P, I64, I64, I64, P, I64, P]),
     "nvfp4_fused_linear_host": (ST, [P, I64, I64, P, P, ctypes.POINTER(Segment), I32, P, P, P, P, P,
                                      P, P, P, P]),
+    "nvfp4_fused_linear_host_overlap": (ST, [P, I64, I64, P, P, ctypes.POINTER(Segment), I32, P, P, P,
+                                             P, P, P, P, P, P, P]),
     "nvfp4_gemm_silu_mul": (ST, [P, P, P, P, P, P, P, I64, I64, I64, I64, P, P, P, P]),
     "nvfp4_harmonize_scales": (ST, [P, I64, ctypes.POINTER(Segment), I32, I32, P, P]),
     "nvfp4_kv_scale_from_amax": (ST, [P, P, P]),
