@@ -735,6 +735,64 @@ def run_reference(args):
                     "d2h_bytes_per_step": 0}}
 
 
+# ---------------------------------------------------------------------------
+# profiler cases: one kernel of the path on a named workload, a few launches
+# ---------------------------------------------------------------------------
+PROFILE_CASES = {
+    "gemm_gdn": "fused GEMM, X [8192,5120] x W q/k/v/z/b/a [24704,5120]",
+    "gemm_gateup": "GEMM, X [8192,5120] x W [34816,5120]",
+    "gemm_decode": "fused GEMM, X [32,5120] x W [24640,5120]",
+    "gemm_decode_m1": "fused GEMM, X [1,5120] x W [24640,5120]",
+    "quantize_act": "quantizer on the activation [32768,5120]",
+    "global_scale_act": "global scale of the activation [32768,5120]",
+}
+
+
+def run_profile_case(case: str, launches: int) -> None:
+    """Build the inputs of `case` (their kernels run first), launch the case's
+    kernel `launches` times and synchronize; for ncu captures (-k/-s/-c)."""
+    import nvfp4_w4a4_quantized_09_b200 as nv
+    from nvfp4_w4a4_quantized_09_b200 import synth
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    if case in ("gemm_gdn", "gemm_decode", "gemm_decode_m1"):
+        M = {"gemm_gdn": 8192, "gemm_decode": 32, "gemm_decode_m1": 1}[case]
+        mods = synth.GDN_MODULES if case == "gemm_gdn" else synth.GDN_MODULES_DECODE
+        x = synth.student_t_activations(M, K_HID, seed=3, device=dev)
+        fw = nv.FusedWeight.from_modules([w for _, w in synth.gdn_weights(mods, device=dev)])
+        a = nv.quantize_tensor(x)
+        segs = fw.segments()
+        y = torch.empty(M, fw.rows, dtype=torch.bfloat16, device=dev)
+        torch.cuda.synchronize()
+        for _ in range(launches):
+            nv.fused_gemm(a, fw.codes, fw.sf, segs, y)
+    elif case == "gemm_gateup":
+        x = synth.student_t_activations(8192, K_HID, seed=1, device=dev)
+        w = synth.gaussian_weights(34816, K_HID, 0.015, seed=20, device=dev)
+        a, wq = nv.quantize_tensor(x), nv.quantize_tensor(w)
+        y = torch.empty(8192, 34816, dtype=torch.bfloat16, device=dev)
+        torch.cuda.synchronize()
+        for _ in range(launches):
+            nv.gemm(a, wq, y)
+    elif case in ("quantize_act", "global_scale_act"):
+        x = synth.student_t_activations(32768, K_HID, seed=1, device=dev)
+        g, amax = nv.global_scale(x)
+        codes = torch.empty(32768, K_HID // 2, dtype=torch.uint8, device=dev)
+        sf = torch.empty(nv.sf_bytes(32768, K_HID), dtype=torch.uint8, device=dev)
+        torch.cuda.synchronize()
+        for _ in range(launches):
+            if case == "quantize_act":
+                nv.quantize(x, g, nv.SF_TCGEN05, codes, sf)
+            else:
+                nv.global_scale(x, g, amax)
+    else:
+        raise SystemExit(f"unknown profile case {case!r}; cases: {', '.join(PROFILE_CASES)}")
+    torch.cuda.synchronize()
+    status = nv.last_device_status()
+    if status != 0:
+        raise SystemExit(f"device status {status}")
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -747,7 +805,13 @@ def main():
     ap.add_argument("--no-harmonize", action="store_true")
     ap.add_argument("--no-kv", action="store_true")
     ap.add_argument("--no-gates", action="store_true")
+    ap.add_argument("--profile-case", choices=sorted(PROFILE_CASES),
+                    help="run one kernel on a named workload for a profiler, then exit")
+    ap.add_argument("--launches", type=int, default=3, help="launches of --profile-case")
     args = ap.parse_args()
+    if args.profile_case:
+        run_profile_case(args.profile_case, args.launches)
+        return
     args.warmup = max(args.warmup, 3)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
