@@ -39,11 +39,11 @@ WORKLOAD = "fused GDN input projection prefill: X bf16 [8192,5120] -> W q/k/v/z/
 L2_FLUSH_BYTES = 256 << 20
 
 
-def gemm_traffic():
-    """DRAM bytes per launch of the fused GEMM from the committed ncu record,
-    or None when the kernel source changed since the counters were taken."""
+def _traffic_record(name):
+    """DRAM bytes per launch from a committed ncu record under profiles/, or
+    None when a source it names changed since the counters were taken."""
     import hashlib
-    path = os.path.join(ROOT, "profiles", "traffic_gemm_pair_fused_gdn_8192x24704x5120.json")
+    path = os.path.join(ROOT, "profiles", name)
     try:
         with open(path) as f:
             rec = json.load(f)
@@ -56,6 +56,16 @@ def gemm_traffic():
         return int(rec["dram_bytes_read"] + rec["dram_bytes_write"])
     except (OSError, KeyError, ValueError):
         return None
+
+
+def gemm_traffic():
+    """DRAM bytes per launch of the fused GEMM (ncu record), or None."""
+    return _traffic_record("traffic_gemm_pair_fused_gdn_8192x24704x5120.json")
+
+
+def quantizer_traffic():
+    """DRAM bytes per launch of the quantizer on [32768, 5120] (ncu record), or None."""
+    return _traffic_record("traffic_quantize_activation_32768x5120.json")
 
 
 def load_peaks():
@@ -74,7 +84,7 @@ class ClockSampler:
     REASONS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
                "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80}
 
-    def __init__(self, device_index: int, period_s: float = 0.01):
+    def __init__(self, device_index: int, period_s: float = 0.001):
         self.samples, self.reasons = [], set()
         self.max_mhz = None
         self.period = period_s
@@ -162,56 +172,6 @@ def build_workload(dev):
     fw = nv.FusedWeight.from_modules(ws)
     del ws
     return x, fw
-
-
-def e2e_overlapped(nv, x_host, x, fw, y, stream, steps, flops, world):
-    """The end-to-end step with consecutive steps' copies overlapped: step
-    i + 1's X goes in on one stream while step i's Y comes out on another (the
-    link is full duplex), the kernels on the launching stream.  Every step
-    still copies its own X in and its own Y out inside the timed region; two
-    device buffers of each keep a step from overwriting one still in use, and
-    every wait is on an event recorded earlier in host order (no cycle)."""
-    s_in, s_out = torch.cuda.Stream(x.device), torch.cuda.Stream(x.device)
-    xd = [torch.empty_like(x) for _ in range(2)]
-    yd = [torch.empty_like(y) for _ in range(2)]
-    yh = [torch.empty(tuple(y.shape), dtype=y.dtype).pin_memory() for _ in range(2)]
-    ev_in = [torch.cuda.Event() for _ in range(2)]
-    ev_done = [torch.cuda.Event() for _ in range(2)]
-    ev_out = [torch.cuda.Event() for _ in range(2)]
-
-    def run(n):
-        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        torch.cuda.synchronize()
-        t0.record(stream)
-        s_in.wait_event(t0)
-        s_out.wait_event(t0)
-        for i in range(n):
-            b = i & 1
-            if i >= 2:
-                s_in.wait_event(ev_done[b])        # step i - 2 has read xd[b]
-            with torch.cuda.stream(s_in):
-                xd[b].copy_(x_host, non_blocking=True)
-            ev_in[b].record(s_in)
-            stream.wait_event(ev_in[b])
-            if i >= 2:
-                stream.wait_event(ev_out[b])       # step i - 2's yd[b] is out
-            nv.linear(xd[b], fw, yd[b], stream=stream)
-            ev_done[b].record(stream)
-            s_out.wait_event(ev_done[b])
-            with torch.cuda.stream(s_out):
-                yh[b].copy_(yd[b], non_blocking=True)
-            ev_out[b].record(s_out)
-        stream.wait_stream(s_in)
-        stream.wait_stream(s_out)
-        t1.record(stream)
-        torch.cuda.synchronize()
-        return t0.elapsed_time(t1) / n
-
-    run(2)
-    ms = run(steps)
-    return {"value": round(world * flops / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
-            "h2d_bytes_per_step": int(x.numel() * 2), "d2h_bytes_per_step": int(y.numel() * 2),
-            "ms_per_step": round(ms, 3), "steps": steps}
 
 
 def act_stats(x):
@@ -315,6 +275,16 @@ def run_ours(args, dev, world, rank):
         "both_GBps": round((q_bytes + n_el * 2) / ((qz_ms + gs_ms) * 1e-3) / 1e9, 1),
         "quantize_us": round(qz_ms * 1e3, 2), "global_scale_us": round(gs_ms * 1e3, 2),
         "hbm_peak_GBps": hbm, "peak_source": peak_src}
+    # the quantizer's roofline beside the GEMM's (bound: HBM)
+    roofline["quantizer"] = {
+        "bound": "hbm", "kernel": "quantize_kernel (activation [32768,5120] bf16)",
+        "achieved": quantizer["quantize_GBps"], "peak": hbm, "unit": "GB/s",
+        "frac": quantizer["quantize_frac_hbm"], "us": quantizer["quantize_us"],
+        "algorithmic_bytes_per_launch": int(q_bytes),
+        "global_scale": {"achieved": quantizer["global_scale_GBps"], "frac": quantizer["global_scale_frac_hbm"],
+                         "us": quantizer["global_scale_us"], "algorithmic_bytes_per_launch": int(n_el * 2)},
+        "traffic": quantizer_traffic(),
+        "peak_source": f"{peak_src} HBM copy bandwidth"}
     del xq, cq, sq
 
     # decode-shaped sweep (weight-bandwidth bound): K = 5120, M tokens, rotating
@@ -457,52 +427,58 @@ def run_ours(args, dev, world, rank):
         del xm, wq_gu, wq_gui, wq_dn, am, hm, ym, hcodes, hsf
         torch.cuda.empty_cache()
 
-    # end to end with host buffers: pinned X in, Y out, every step.  Measured
-    # through the C-ABI call that takes host buffers (nvfp4_fused_linear_host);
-    # should that path raise, through the Python API with torch's copies.
+    # end to end with host buffers, through the C ABI: every step copies its
+    # pinned X in and its Y out inside the timed region.  Headline: the
+    # overlapped entry (nvfp4_fused_linear_host_overlap: copy out on a second
+    # stream in row slices; the next step's copy in runs during it).  Beside
+    # it: the one-stream entry, and the link's own copy rates for context.
     x_host = x.cpu().pin_memory()
     y_host = torch.empty(M, N, dtype=torch.bfloat16).pin_memory()
     e2e_steps = max(3, min(args.steps, 20))
+    copy_stream = torch.cuda.Stream(dev)
+    scratch = nv.HostLinearScratch(M, K, N, dev)
 
-    def timed_e2e(one_step):
-        for i in range(2 + e2e_steps):
-            if i == 2:
-                torch.cuda.synchronize()
-                s0 = torch.cuda.Event(enable_timing=True)
-                s0.record(stream)
+    def timed_host_steps(one_step, n):
+        one_step()
+        one_step()
+        torch.cuda.synchronize()
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        copy_stream.wait_event(s0)
+        for _ in range(n):
             one_step()
-        s1 = torch.cuda.Event(enable_timing=True)
+        stream.wait_stream(copy_stream)
         s1.record(stream)
         torch.cuda.synchronize()
-        return s0.elapsed_time(s1) / e2e_steps
+        return s0.elapsed_time(s1) / n
 
-    e2e_path, e2e_error = "C ABI: nvfp4_fused_linear_host, pinned host X in and Y out", None
-    try:
-        scratch = nv.HostLinearScratch(M, K, N, dev)
-        e2e_ms = timed_e2e(lambda: nv.linear_host(x_host, fw, y_host, scratch=scratch, stream=stream))
-        del scratch
-    except Exception as exc:  # noqa: BLE001 - fall back to the Python API's form
-        e2e_error = repr(exc)[:300]
-        e2e_path = "Python API: torch copies of pinned X in and Y out around nv.linear"
-        x_dev = torch.empty_like(x)
-
-        def torch_step():
-            x_dev.copy_(x_host, non_blocking=True)
-            nv.linear(x_dev, fw, y)
-            y_host.copy_(y, non_blocking=True)
-        e2e_ms = timed_e2e(torch_step)
-        del x_dev
+    e2e_ms = timed_host_steps(
+        lambda: nv.linear_host(x_host, fw, y_host, scratch=scratch, stream=stream,
+                               copy_stream=copy_stream), e2e_steps)
+    serial_ms = timed_host_steps(
+        lambda: nv.linear_host(x_host, fw, y_host, scratch=scratch, stream=stream), e2e_steps)
+    # raw pinned copies of the same bytes (one direction at a time)
+    xd_tmp = torch.empty_like(x)
+    c0, c1, c2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+    torch.cuda.synchronize()
+    c0.record(stream)
+    xd_tmp.copy_(x_host, non_blocking=True)
+    c1.record(stream)
+    y_host.copy_(y, non_blocking=True)
+    c2.record(stream)
+    torch.cuda.synchronize()
+    h2d_gbs = x.numel() * 2 / (c0.elapsed_time(c1) * 1e-3) / 1e9
+    d2h_gbs = y.numel() * 2 / (c1.elapsed_time(c2) * 1e-3) / 1e9
+    del xd_tmp, scratch
     e2e = {"value": round(world * flops / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
            "h2d_bytes_per_step": int(x.numel() * 2), "d2h_bytes_per_step": int(y.numel() * 2),
-           "ms_per_step": round(e2e_ms, 3), "path": e2e_path}
-    if e2e_error:
-        e2e["c_abi_error"] = e2e_error
-    # the same with the two copy directions of consecutive steps overlapped;
-    # an extra leg, so a failure in it is recorded and never stops the line
-    try:
-        e2e_ovl = e2e_overlapped(nv, x_host, x, fw, y, stream, e2e_steps, flops, world)
-    except Exception as exc:  # noqa: BLE001
-        e2e_ovl = {"error": repr(exc)[:300]}
+           "ms_per_step": round(e2e_ms, 3), "steps": e2e_steps,
+           "path": "C ABI nvfp4_fused_linear_host_overlap: pinned X in, Y out on a second stream in row slices",
+           "link_h2d_GBps": round(h2d_gbs, 1), "link_d2h_GBps": round(d2h_gbs, 1),
+           "d2h_alone_ms": round(y.numel() * 2 / (d2h_gbs * 1e9) * 1e3, 3),
+           "serial": {"value": round(world * flops / (serial_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+                      "ms_per_step": round(serial_ms, 3),
+                      "path": "C ABI nvfp4_fused_linear_host: one stream, copies in series"}}
     torch.cuda.empty_cache()
 
     # sanity (reported, not a target): quantized vs BF16 GEMM on sampled rows
@@ -632,7 +608,7 @@ def run_ours(args, dev, world, rank):
                    "l2": "flushed between timed steps (256 MB write)"},
         "components_us": {"global_scale+quantize": round(float(np.mean(quant_ms)) * 1e3, 2),
                           "fused_gemm": round(gemm_avg_ms * 1e3, 2)},
-        "roofline": roofline, "quantizer": quantizer, "e2e": e2e, "e2e_overlapped": e2e_ovl,
+        "roofline": roofline, "quantizer": quantizer, "e2e": e2e,
         "decode_sweep": decode, "mlp_32k": mlp_line,
         "harmonize": harm, "kv_cache_fp8": kv, "gate_epilogue": gates,
         "gpu_launches": 3 * args.steps,
