@@ -81,6 +81,7 @@ struct GemmArgs {
     int atoms_per_rb;     // ceil(K/64): scale atoms per 128-row block
     int w_rowblocks;      // ceil(N/128)
     int group_m;          // raster: tiles visit group_m m-tiles per n sweep
+    int nt_first;         // raster: the n sweep starts at this n-tile (the gated columns')
     int nseg;
     int seg_end[NVFP4_MAX_SEGMENTS];
     const float* seg_g[NVFP4_MAX_SEGMENTS];
@@ -107,7 +108,7 @@ struct SegTable {
     int end[NVFP4_MAX_SEGMENTS];              // one past the segment's last column
     int kind[NVFP4_MAX_SEGMENTS];             // nvfp4_act_kind
     int goff[NVFP4_MAX_SEGMENTS];             // decay gate: first index in gp0/gp1
-    float gp0[kMaxGateCols];                  // decay gate: A_log per column
+    float gp0[kMaxGateCols];                  // decay gate: -exp(A_log) per column
     float gp1[kMaxGateCols];                  // decay gate: dt_bias per column
 };
 
@@ -156,7 +157,8 @@ __device__ __forceinline__ void tile_coords(int t, const GemmArgs& a, int& mt, i
     const int gsize = min(group_m, a.m_tiles - first_m);
     const int local = t - grp * per_group;
     mt = first_m + local % gsize;
-    nt = local / gsize;
+    nt = local / gsize + a.nt_first;           // rotated sweep: gated tiles early, not in the tail
+    if (nt >= a.n_tiles) nt -= a.n_tiles;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -174,7 +176,9 @@ __device__ __forceinline__ void fill_seg_table(SegTable& T, const GemmArgs& a, i
     T.goff[t] = in ? a.seg_goff[t] : 0;
 }
 
-// Stage the decay-gate parameters (all threads of the CTA; before a barrier).
+// Stage the decay-gate parameters (all threads of the CTA; before a barrier):
+// per column -exp(A_log) (the same binary32 value the gate would compute per
+// element) and dt_bias.
 __device__ __forceinline__ void stage_gate_params(SegTable& T, const GemmArgs& a) {
     if (!a.any_act) return;
     for (int s = 0; s < a.nseg; ++s) {
@@ -182,32 +186,76 @@ __device__ __forceinline__ void stage_gate_params(SegTable& T, const GemmArgs& a
         const int start = s == 0 ? 0 : a.seg_end[s - 1];
         const int n = a.seg_end[s] - start;
         for (int c = threadIdx.x; c < n; c += blockDim.x) {
-            T.gp0[a.seg_goff[s] + c] = a.seg_p0[s][c];
+            T.gp0[a.seg_goff[s] + c] = -expf(a.seg_p0[s][c]);
             T.gp1[a.seg_goff[s] + c] = a.seg_p1[s][c];
         }
     }
 }
 
 // Gated DeltaNet gate functions in FP32: the log-space decay gate
-// -exp(A_log) * softplus(v + dt_bias), softplus(z) = max(z, 0) + log(1 +
-// e^-|z|) (no branch, no overflow), and the sigmoid 1 / (1 + e^-v).
-__device__ __forceinline__ float gate_fn(float v, int kind, float a_log, float dt_bias) {
+// -exp(A_log) * softplus(v + dt_bias) with -exp(A_log) staged per column, and
+// the sigmoid.  Both are written so that every intermediate stays in (0, 1]
+// and no special value reaches a library routine, whatever the size of v:
+//   softplus(z) = max(z, 0) + log1p(t), t = e^-|z|, with log1p(t) taken as t
+//   once t < 2^-24 (|z| > 17: the two agree to a relative 2^-25);
+//   sigmoid(v) = 1 / (1 + t) for v >= 0 and t / (1 + t) below, t = e^-|v|.
+__device__ __forceinline__ float gate_fn(float v, int kind, float neg_exp_alog, float dt_bias) {
     if (kind == NVFP4_ACT_DECAY_GATE) {
         const float z = __fadd_rn(v, dt_bias);
-        const float sp = __fadd_rn(fmaxf(z, 0.0f), log1pf(expf(-fabsf(z))));
-        return __fmul_rn(-expf(a_log), sp);
+        const float a = fabsf(z);
+        const float t = expf(-a);
+        const float l = a > 17.0f ? t : log1pf(t);
+        return __fmul_rn(neg_exp_alog, __fadd_rn(fmaxf(z, 0.0f), l));
     }
-    if (kind == NVFP4_ACT_SIGMOID) return __frcp_rn(__fadd_rn(1.0f, expf(-v)));
+    if (kind == NVFP4_ACT_SIGMOID) {
+        const float t = expf(-fabsf(v));
+        const float s = __frcp_rn(__fadd_rn(1.0f, t));
+        return v >= 0.0f ? s : __fmul_rn(t, s);
+    }
     return v;
 }
 
 // Apply the segments' gate functions to CNT consecutive scaled outputs
-// starting at column n0 (columns at or beyond N are left alone).
-template <int CNT>
-__device__ __forceinline__ void apply_gates(float (&v)[CNT], int n0, int N, int nseg,
-                                            const SegTable& T) {
-    int s = 0;
+// starting at column n0 (columns at or beyond N are left alone).  Out of line:
+// the math functions inlined once per element would bloat every epilogue
+// that contains this call (only chunks that meet the gated columns reach it,
+// and their values take a trip through local memory).  A chunk inside one
+// segment, the usual case, is evaluated eight elements at a time so that the
+// exp / log1p chains of different elements overlap.
+template <int KIND>
+__device__ __forceinline__ void gate_run(float* v, int n0, int N, int cnt, int g0, const SegTable& T) {
+#pragma unroll 1
+    for (int j0 = 0; j0 < cnt; j0 += 8) {
+        float x[8];
 #pragma unroll
+        for (int jj = 0; jj < 8; ++jj) x[jj] = v[j0 + jj];
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) {
+            if (n0 + j0 + jj < N) {
+                const int g = g0 + j0 + jj;
+                x[jj] = KIND == NVFP4_ACT_DECAY_GATE ? gate_fn(x[jj], KIND, T.gp0[g], T.gp1[g])
+                                                     : gate_fn(x[jj], KIND, 0.0f, 0.0f);
+            }
+        }
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) v[j0 + jj] = x[jj];
+    }
+}
+
+template <int CNT>
+__device__ __noinline__ void apply_gates(float* v, int n0, int N, int nseg, const SegTable& T) {
+    static_assert(CNT % 8 == 0 || CNT < 8, "chunks of eight");
+    int s = 0;
+    while (s < nseg - 1 && n0 >= T.end[s]) ++s;
+    if (CNT % 8 == 0 && (s == nseg - 1 || n0 + CNT <= T.end[s])) {
+        const int kind = T.kind[s];
+        const int g0 = T.goff[s] + n0 - (s == 0 ? 0 : T.end[s - 1]);
+        if (kind == NVFP4_ACT_DECAY_GATE) gate_run<NVFP4_ACT_DECAY_GATE>(v, n0, N, CNT, g0, T);
+        else if (kind == NVFP4_ACT_SIGMOID) gate_run<NVFP4_ACT_SIGMOID>(v, n0, N, CNT, 0, T);
+        return;
+    }
+    // a chunk that meets two or more segments: one element at a time
+#pragma unroll 1
     for (int j = 0; j < CNT; ++j) {
         const int n = n0 + j;
         while (s < nseg - 1 && n >= T.end[s]) ++s;
@@ -218,6 +266,19 @@ __device__ __forceinline__ void apply_gates(float (&v)[CNT], int n0, int N, int 
             v[j] = gate_fn(v[j], kind, decay ? T.gp0[g] : 0.0f, decay ? T.gp1[g] : 0.0f);
         }
     }
+}
+
+// The gated chunk's values go through a local copy, so the caller's array
+// never has its address taken and stays in registers on every other chunk.
+template <int CNT>
+__device__ __forceinline__ void apply_gates_copy(float (&v)[CNT], int n0, int N, int nseg,
+                                                 const SegTable& T) {
+    float tmp[CNT];
+#pragma unroll
+    for (int j = 0; j < CNT; ++j) tmp[j] = v[j];
+    apply_gates<CNT>(tmp, n0, N, nseg, T);
+#pragma unroll
+    for (int j = 0; j < CNT; ++j) v[j] = tmp[j];
 }
 
 template <int BN, int STAGES, int ACC>
@@ -437,7 +498,7 @@ nvf4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                         }
                     }
                     if (args.any_act && n0 < args.gate_hi && n0 + 32 > args.gate_lo)
-                        apply_gates<32>(v, n0, args.N, args.nseg, seg_tab);
+                        apply_gates_copy<32>(v, n0, args.N, args.nseg, seg_tab);
                     uint32_t o[16];
 #pragma unroll
                     for (int j = 0; j < 16; ++j) o[j] = pack_bf16x2(v[2 * j], v[2 * j + 1]);
@@ -583,7 +644,7 @@ nvf4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a,
         prefetch_tmap(&tmap_b);
         prefetch_tmap(&tmap_sfa);
         prefetch_tmap(&tmap_sfb);
-        if constexpr (!kSilu) prefetch_tmap(&tmap_y);
+        prefetch_tmap(&tmap_y);
     }
     if (warp == 1) {
         tmem_alloc_pair(s_tmem_base, C::TMEM_COLS);
@@ -733,9 +794,11 @@ nvf4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a,
             // magnitude bits) for the requantization's global scale.
             const int q = warp & 3;
             const int half = (warp - 2) >> 2;
-            const int row = q * 32 + lane;
             const uint64_t pol_y = l2_policy_evict_first();
             const float al = s_seg_alpha[0];
+            uint8_t* stage_y = smem + C::OFF_EPI + (warp - 2) * C::EPI_BYTES;
+            const uint32_t sy = smem_u32(stage_y);
+            const uint32_t swz = static_cast<uint32_t>((lane >> 1) & 3);
             uint32_t mag = 0;
             int i = 0;
             for (int t = pair; t < total_tiles; t += npairs, ++i) {
@@ -756,60 +819,77 @@ nvf4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a,
                 tmem_ld_wait();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive_cluster(tmem_empty_leader);
+                if (lane == 0) mbar_arrive_cluster_relaxed(tmem_empty_leader);
                 // every lane computes (the votes below need the whole warp);
-                // only rows inside M store and count toward the max
-                const int m = mt * 256 + static_cast<int>(rank) * 128 + row;
-                const bool row_ok = m < args.M;
-                {
-                    uint16_t* hrow = args.y + static_cast<int64_t>(row_ok ? m : 0) * args.ldy;
+                // only rows inside M count toward the max, and the TMA store
+                // clips rows beyond M
+                const int m0 = mt * 256 + static_cast<int>(rank) * 128 + q * 32;   // row of lane 0
+                const bool row_ok = m0 + lane < args.M;
 #pragma unroll
-                    for (int ch = 0; ch < 2; ++ch) {
-                        const int j0 = nt * (BN / 2) + half * 64 + ch * 32;
-                        // branch-free FP32 for every element (fast division: within
-                        // 2 ulp, far inside the BF16 result's rounding); the rare
-                        // g < -80, where e^-g overflows, is redone in FP64 after a
-                        // vote.  Eight outputs per 16-byte store keep few values live.
+                for (int ch = 0; ch < 2; ++ch) {
+                    const int j0 = nt * (BN / 2) + half * 64 + ch * 32;
+                    // branch-free FP32 for every element (fast division: within
+                    // 2 ulp, far inside the BF16 result's rounding); the rare
+                    // g < -80, where e^-g overflows, is redone by the scaled
+                    // form of silu_mul_tail after a vote.
+                    uint32_t o[16];
 #pragma unroll
-                        for (int q8 = 0; q8 < 4; ++q8) {
-                            uint32_t o[4];
-                            bool rare = false;
+                    for (int q8 = 0; q8 < 4; ++q8) {
+                        bool rare = false;
+#pragma unroll
+                        for (int jj = 0; jj < 4; ++jj) {
+                            const int j = 4 * q8 + jj;
+                            const float g0 = __fmul_rn(__uint_as_float(r[ch][2 * j]), al);
+                            const float g1 = __fmul_rn(__uint_as_float(r[ch][2 * j + 1]), al);
+                            const float u0 = __fmul_rn(__uint_as_float(r[2 + ch][2 * j]), al);
+                            const float u1 = __fmul_rn(__uint_as_float(r[2 + ch][2 * j + 1]), al);
+                            rare |= (g0 < -80.0f) | (g1 < -80.0f);
+                            const float s0 = __fdividef(g0, __fadd_rn(1.0f, expf(-g0)));
+                            const float s1 = __fdividef(g1, __fadd_rn(1.0f, expf(-g1)));
+                            o[j] = pack_bf16x2(__fmul_rn(s0, u0), __fmul_rn(s1, u1));
+                        }
+                        if (__any_sync(0xFFFFFFFFu, rare)) {
 #pragma unroll
                             for (int jj = 0; jj < 4; ++jj) {
                                 const int j = 4 * q8 + jj;
                                 const float g0 = __fmul_rn(__uint_as_float(r[ch][2 * j]), al);
                                 const float g1 = __fmul_rn(__uint_as_float(r[ch][2 * j + 1]), al);
-                                const float u0 = __fmul_rn(__uint_as_float(r[2 + ch][2 * j]), al);
-                                const float u1 = __fmul_rn(__uint_as_float(r[2 + ch][2 * j + 1]), al);
-                                rare |= (g0 < -80.0f) | (g1 < -80.0f);
-                                const float s0 = __fdividef(g0, __fadd_rn(1.0f, expf(-g0)));
-                                const float s1 = __fdividef(g1, __fadd_rn(1.0f, expf(-g1)));
-                                o[jj] = pack_bf16x2(__fmul_rn(s0, u0), __fmul_rn(s1, u1));
-                            }
-                            if (__any_sync(0xFFFFFFFFu, rare)) {
-#pragma unroll
-                                for (int jj = 0; jj < 4; ++jj) {
-                                    const int j = 4 * q8 + jj;
-                                    const float g0 = __fmul_rn(__uint_as_float(r[ch][2 * j]), al);
-                                    const float g1 = __fmul_rn(__uint_as_float(r[ch][2 * j + 1]), al);
-                                    if (g0 < -80.0f)
-                                        o[jj] = (o[jj] & 0xFFFF0000u) |
-                                                silu_mul1(g0, __fmul_rn(__uint_as_float(r[2 + ch][2 * j]), al));
-                                    if (g1 < -80.0f)
-                                        o[jj] = (o[jj] & 0xFFFFu) |
-                                                (silu_mul1(g1, __fmul_rn(__uint_as_float(r[2 + ch][2 * j + 1]), al)) << 16);
-                                }
-                            }
-                            if (row_ok) {
-#pragma unroll
-                                for (int jj = 0; jj < 4; ++jj)
-                                    mag = max(mag, max(o[jj] & 0x7FFFu, (o[jj] >> 16) & 0x7FFFu));
-                                st_global_v4_hint(hrow + j0 + 8 * q8, o[0], o[1], o[2], o[3], pol_y);
+                                if (g0 < -80.0f)
+                                    o[j] = (o[j] & 0xFFFF0000u) |
+                                           silu_mul1(g0, __fmul_rn(__uint_as_float(r[2 + ch][2 * j]), al));
+                                if (g1 < -80.0f)
+                                    o[j] = (o[j] & 0xFFFFu) |
+                                           (silu_mul1(g1, __fmul_rn(__uint_as_float(r[2 + ch][2 * j + 1]), al)) << 16);
                             }
                         }
                     }
+                    if (row_ok) {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) mag = max(mag, max(o[j] & 0x7FFFu, (o[j] >> 16) & 0x7FFFu));
+                    }
+                    if (m0 < args.M) {                                  // warp-uniform
+                        // 32 x 32 tile through the staging buffer, one TMA store
+                        if (ch > 0) {
+                            if (lane == 0) bulk_wait_read_all();
+                            __syncwarp();
+                        }
+#pragma unroll
+                        for (int u = 0; u < 4; ++u)
+                            sts128(sy + lane * 64 + ((static_cast<uint32_t>(u) ^ swz) << 4), o[4 * u],
+                                   o[4 * u + 1], o[4 * u + 2], o[4 * u + 3]);
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {
+                            tma_store_2d(&tmap_y, stage_y, j0, m0, pol_y);
+                            bulk_commit_group();
+                        }
+                    }
                 }
+                if (lane == 0) bulk_wait_read_all();
+                __syncwarp();
             }
+            if (lane == 0) bulk_wait_all();
+            __syncwarp();
             mag = __reduce_max_sync(0xFFFFFFFFu, mag);
             if (lane == 0 && mag) atomicMax(&args.h_ws[0], mag << 16);
         } else {
@@ -872,7 +952,7 @@ nvf4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a,
                     }
                 }
                 if (args.any_act && n0 < args.gate_hi && n0 + 32 > args.gate_lo)
-                    apply_gates<32>(v, n0, args.N, args.nseg, seg_tab);
+                    apply_gates_copy<32>(v, n0, args.N, args.nseg, seg_tab);
                 uint32_t o[16];
 #pragma unroll
                 for (int j = 0; j < 16; ++j) o[j] = pack_bf16x2(v[2 * j], v[2 * j + 1]);
@@ -1058,6 +1138,7 @@ nvfp4_status launch_gemm(const uint8_t* a_codes, const uint8_t* w_codes, GemmArg
     if (!make_code_map(&tb, w_codes, args.N, args.K / 2, BN)) return NVFP4_ERR_CUDA;
     args.m_tiles = (args.M + kBM - 1) / kBM;
     args.n_tiles = (args.N + BN - 1) / BN;
+    args.nt_first /= BN;
     const int tiles = args.m_tiles * args.n_tiles;
     const int grid = tiles < dev.sms ? tiles : dev.sms;
     kern<<<grid, kThreads, Cf::SMEM, stream>>>(ta, tb, args);
@@ -1084,11 +1165,12 @@ nvfp4_status launch_gemm_pair(const uint8_t* a_codes, const uint8_t* w_codes, Ge
     if (!make_code_map(&tb, w_codes, args.N, args.K / 2, 128, KB)) return NVFP4_ERR_CUDA;
     if (!make_sf_map(&tsa, args.a_sf, a_rb, args.atoms_per_rb, 1, Cf::ATOMS)) return NVFP4_ERR_CUDA;
     if (!make_sf_map(&tsb, args.w_sf, w_rb, args.atoms_per_rb, 2, Cf::ATOMS)) return NVFP4_ERR_CUDA;
-    // the SiLU epilogue stores h directly and leaves this map unused
+    // the output: y [M, N], or h [M, N / 2] for the SiLU epilogue
     if (!make_out_map(&ty, args.y, args.M, kSilu ? args.N / 2 : args.N, args.ldy)) return NVFP4_ERR_CUDA;
     args.k_steps = (args.K + 2 * KB - 1) / (2 * KB);
     args.m_tiles = (args.M + 255) / 256;
     args.n_tiles = (args.N + Cf::BN - 1) / Cf::BN;
+    args.nt_first /= Cf::BN;
     const int tiles = args.m_tiles * args.n_tiles;
     const int max_pairs = dev.sms / 2;
     const int pairs = tiles < max_pairs ? tiles : max_pairs;
@@ -1260,6 +1342,9 @@ nvfp4_status gemm_impl(const uint8_t* a_codes, const uint8_t* a_sf, const float*
         }
     }
     if (gate_cols > kMaxGateCols) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    // the n-tile width is the kernel's: the launchers turn this column into
+    // the first n-tile of the sweep (0 without gates)
+    args.nt_first = args.any_act ? args.gate_lo : 0;
     args.timeout_ns = kTimeoutNs;
     args.status = status;
     cudaStream_t cs = as_stream(stream);

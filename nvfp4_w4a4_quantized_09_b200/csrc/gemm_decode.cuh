@@ -465,7 +465,7 @@ nvf4_gemm_decode_kernel(const __grid_constant__ CUtensorMap tmap_w,
                 float o4[4] = {__fmul_rn(sum.x, al[0]), __fmul_rn(sum.y, al[1]),
                                __fmul_rn(sum.z, al[2]), __fmul_rn(sum.w, al[3])};
                 if (args.any_act && n0 < args.gate_hi && n0 + 4 > args.gate_lo)
-                    apply_gates<4>(o4, n0, args.N, args.nseg, seg_tab);
+                    apply_gates_copy<4>(o4, n0, args.N, args.nseg, seg_tab);
                 return make_uint2(pack_bf16x2(o4[0], o4[1]), pack_bf16x2(o4[2], o4[3]));
             };
             auto store_one = [&](int t, uint2 o) {

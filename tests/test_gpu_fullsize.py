@@ -162,3 +162,45 @@ def test_mlp_32k_prefill_sampled():
     cd, sd = oracle.quantize(wdb, gd)
     assert_gemm_matches(host_bits(y[rid]), dequant(ch, sh), dequant(cd, sd),
                         oracle.segment_alpha(gh, [(0, H, gd)]), label="down 32K")
+
+
+def test_mlp_32k_fused_silu_sampled():
+    # the fused MLP intermediate at the 32K prefill size the benchmark times:
+    # gate_up [34816, 5120] (rows interleaved gate/up in 128-row blocks) with
+    # h = SiLU(gate) * up and its global scale in the epilogue.  h on 64 seeded
+    # rows against SiLU(gate) * up of the exact GEMM; the returned scale equals
+    # the standalone global scale of the whole h and the oracle's; the
+    # requantization with it equals the unfused quantizer's bytes.
+    from parity_helpers import assert_silu_matches
+    M, H, F = 32768, 5120, 17408
+    x = synth.student_t_activations(M, H, seed=1, device=DEV)
+    w_gu = synth.gaussian_weights(2 * F, H, 0.015, seed=20, device=DEV)
+    a = nv.quantize_tensor(x)
+    wi = nv.quantize_tensor(nv.interleave_gate_up(w_gu))
+    h, g_h, amax_h = nv.gemm_silu_mul(a, wi)
+    g_chk, amax_chk = nv.global_scale(h)
+    c1, s1 = nv.quantize(h, g_h)
+    q2 = nv.quantize_tensor(h)
+    torch.cuda.synchronize()
+    assert nv.last_device_status() == 0
+    assert np_f32(g_h)[0] == np_f32(g_chk)[0] and np_f32(amax_h)[0] == np_f32(amax_chk)[0]
+    assert torch.equal(c1, q2.codes) and torch.equal(s1, q2.sf)
+    del c1, s1, q2
+    g_or, amax_or = oracle.global_scale(host_bits(h))
+    assert np_f32(g_h)[0] == g_or and np_f32(amax_h)[0] == amax_or
+    rows = sample_rows(M, 62, 11)
+    rid = torch.from_numpy(rows).to(DEV)
+    xb = host_bits(x)
+    ga, _ = oracle.global_scale(xb)
+    ca, sa = oracle.quantize(xb[rows], ga)
+    wgb = host_bits(w_gu)
+    gw, _ = oracle.global_scale(wgb)
+    cw, sw = oracle.quantize(wgb, gw)
+    A, W = dequant(ca, sa), dequant(cw, sw)
+    del cw, sw
+    alpha = oracle.segment_alpha(ga, [(0, 2 * F, gw)])
+    y64 = oracle.gemm_f64(A, W, alpha)
+    S = (np.abs(A) @ np.abs(W).T) * np.abs(alpha)[None, :]
+    exact = assert_silu_matches(host_bits(h[rid]), y64[:, :F], y64[:, F:], S[:, :F], S[:, F:], H,
+                                label="fused SiLU 32K")
+    assert exact > 0.9

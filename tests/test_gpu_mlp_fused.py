@@ -63,3 +63,20 @@ def test_gemm_silu_mul_then_requantize_is_the_unfused_quantizer():
     q2 = nv.quantize_tensor(h)
     torch.cuda.synchronize()
     assert torch.equal(c1, q2.codes) and torch.equal(s1, q2.sf)
+
+
+def test_mlp_interleaved_is_the_fused_three_launch_path():
+    # nv.mlp(interleaved=True): fused gate_up + SiLU epilogue, requantization of
+    # h with the returned scale, down GEMM -- bit for bit the composed calls
+    M, H, F = 300, 512, 256
+    x = synth.student_t_activations(M, H, seed=41, device=DEV)
+    w_gu = synth.gaussian_weights(2 * F, H, 0.015, seed=42, device=DEV)
+    w_dn = synth.gaussian_weights(H, F, 0.01, seed=43, device=DEV)
+    wi = nv.quantize_tensor(nv.interleave_gate_up(w_gu))
+    wd = nv.quantize_tensor(w_dn)
+    y = nv.mlp(x, wi, wd, interleaved=True)
+    h, g_h, _ = nv.gemm_silu_mul(nv.quantize_tensor(x), wi)
+    codes, sf = nv.quantize(h, g_h)
+    y_ref = nv.gemm(nv.QuantizedTensor(codes, sf, g_h, M, F), wd)
+    torch.cuda.synchronize()
+    assert torch.equal(y.view(torch.int16), y_ref.view(torch.int16))
