@@ -179,13 +179,13 @@ __device__ __forceinline__ void fill_seg_table(SegTable& T, const GemmArgs& a, i
 // Stage the decay-gate parameters (all threads of the CTA; before a barrier):
 // per column -exp(A_log) (the same binary32 value the gate would compute per
 // element) and dt_bias.
-__device__ __forceinline__ void stage_gate_params(SegTable& T, const GemmArgs& a) {
+__device__ __forceinline__ void stage_gate_params(SegTable& T, const GemmArgs& a, int tid, int nthreads) {
     if (!a.any_act) return;
     for (int s = 0; s < a.nseg; ++s) {
         if (a.seg_kind[s] != NVFP4_ACT_DECAY_GATE) continue;
         const int start = s == 0 ? 0 : a.seg_end[s - 1];
         const int n = a.seg_end[s] - start;
-        for (int c = threadIdx.x; c < n; c += blockDim.x) {
+        for (int c = tid; c < n; c += nthreads) {
             T.gp0[a.seg_goff[s] + c] = -expf(a.seg_p0[s][c]);
             T.gp1[a.seg_goff[s] + c] = a.seg_p1[s][c];
         }
@@ -326,7 +326,7 @@ nvf4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
     }
     if (threadIdx.x >= 64 && threadIdx.x < 64 + NVFP4_MAX_SEGMENTS)
         fill_seg_table(seg_tab, args, threadIdx.x - 64);
-    stage_gate_params(seg_tab, args);
+    stage_gate_params(seg_tab, args, threadIdx.x, blockDim.x);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -652,7 +652,7 @@ nvf4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a,
     }
     if (threadIdx.x >= 64 && threadIdx.x < 64 + NVFP4_MAX_SEGMENTS)
         fill_seg_table(seg_tab, args, threadIdx.x - 64);
-    stage_gate_params(seg_tab, args);
+    stage_gate_params(seg_tab, args, threadIdx.x, blockDim.x);
     tc_fence_before();
     __syncthreads();
     cluster_sync();                                      // barriers of both CTAs initialised

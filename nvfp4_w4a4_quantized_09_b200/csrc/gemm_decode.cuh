@@ -192,15 +192,16 @@ nvf4_gemm_decode_kernel(const __grid_constant__ CUtensorMap tmap_w,
         tmem_alloc(s_tmem_base, kDecTmemCols);
         tmem_relinquish();
     }
-    if (threadIdx.x >= 64 && threadIdx.x < 64 + NVFP4_MAX_SEGMENTS)
-        fill_seg_table(seg_tab, args, threadIdx.x - 64);
-    stage_gate_params(seg_tab, args);
     tc_fence_before();
     __syncthreads();
-    // the peers' barriers are initialised before anyone arrives on them remotely
-    cluster_sync();
     tc_fence_after();
     const uint32_t tmem_base = *s_tmem_base;
+    // Cross-CTA set-up without holding up the weight stream: every thread
+    // arrives on the cluster barrier now; the roles that touch a peer's
+    // shared memory or barriers (pushers, reducers) wait on it before their
+    // first remote access, the others only at the end.  The producer and the
+    // MMA warp use local barriers only, so the first weight loads leave at once.
+    cluster_arrive();
 
     // Loop-invariant step data.  Every role walks the same (tile, k-step)
     // sequence with incremental ring counters -- no division in the loops;
@@ -383,6 +384,7 @@ nvf4_gemm_decode_kernel(const __grid_constant__ CUtensorMap tmap_w,
         const int rr = row - owner * R;
         const uint32_t part_owner = mapa_shared(smem_u32(part), static_cast<uint32_t>(owner));
         const uint32_t full_owner0 = mapa_shared(smem_u32(part_full), static_cast<uint32_t>(owner));
+        cluster_wait();                     // the owners' barriers are initialised
         int i = 0;
         for (int nt = cluster_id; nt < args.n_tiles; nt += num_clusters, ++i) {
             const int acc = i % NACC;
@@ -421,6 +423,11 @@ nvf4_gemm_decode_kernel(const __grid_constant__ CUtensorMap tmap_w,
         // The results stay in registers until this warp has released the
         // partial buffer, so that release never waits on the global stores.
         const int red_tid = threadIdx.x - 10 * 32;
+        // the segment table and gate parameters are the reducers' alone
+        if (red_tid < NVFP4_MAX_SEGMENTS) fill_seg_table(seg_tab, args, red_tid);
+        stage_gate_params(seg_tab, args, red_tid, 128);
+        named_barrier_sync(1, 128);
+        cluster_wait();                     // the peers' barriers are initialised
         const int ngroups = R / 4;
         const int rg = red_tid % ngroups;
         const int tstep = 128 / ngroups;
@@ -505,6 +512,7 @@ nvf4_gemm_decode_kernel(const __grid_constant__ CUtensorMap tmap_w,
     // arrive on its barriers
     tc_fence_before();
     __syncwarp();
+    if (warp < 6) cluster_wait();           // the roles that did not wait above
     cluster_sync();
     tc_fence_after();
     if (warp == 1) tmem_dealloc(tmem_base, kDecTmemCols);

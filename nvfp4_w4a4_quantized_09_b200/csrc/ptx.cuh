@@ -439,6 +439,22 @@ __device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t cluster_sad
                  : "memory");
 }
 
+// The two halves of cluster_sync, for roles that can start before their
+// peers: arrive (release: this thread's earlier writes, barrier set-up
+// included, become visible to the cluster) and, later, wait (acquire).
+__device__ __forceinline__ void cluster_arrive() {
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void cluster_wait() {
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Barrier among `count` threads of the CTA on named barrier `id` (1..15).
+__device__ __forceinline__ void named_barrier_sync(int id, int count) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 __device__ __forceinline__ void cluster_sync() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
                      : "memory");
