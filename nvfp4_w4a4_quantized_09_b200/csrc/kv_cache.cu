@@ -5,15 +5,22 @@
 // KV-cache scales, throughput-free).  The formula is the plain reading of a
 // per-tensor FP8 scale; the pages give none.
 //
-// Bandwidth-bound (2 bytes in, 1 byte out per element); each thread keeps four
-// 16-byte loads in flight.  Exactness without a
-// division per element: with r = RN(1/s), the reals r(1 - 2^-20) and
-// r(1 + 2^-20), rounded, bracket 1/s (r is within 2^-24 of 1/s), so x*rlo and
-// x*rhi bracket the exact quotient x/s; fl32 rounding and the E4M3 RNE encode
-// are both monotone, so when the two bracket codes agree they equal the code
-// of fl32(x/s).  Elements whose bracket codes differ (a quotient within 2^-20
-// of a rounding boundary) take the IEEE division.  If 1/s is not a normal
-// float every element divides.
+// Bandwidth-bound (2 bytes in, 1 byte out per element); each thread keeps
+// several 16-byte loads in flight.  The quotient fl32(x / s) is exact without
+// a division per element: with r = RN(1/s) and q0 = RN(x r), the remainder
+// x - q0 s is exact in one FMA and RN(q0 + (x - q0 s) r) is the correctly
+// rounded quotient (Markstein's theorem: P. Markstein, "Computation of
+// elementary functions on the IBM RISC System/6000 processor", IBM J. Res.
+// Dev. 34(1), 1990), provided no step over- or underflows.
+//  * s in [2^-92, 2^100] keeps r normal and the remainder exact for every
+//    quotient of 2^-11 or more; below that (x subnormal or tiny) the result
+//    stays under 2^-11 with the sign of x/s, and every such value encodes to a
+//    signed zero, as the exact quotient does.  Other s divide.
+//  * The quotient is formed from -x and -r, each step the exact negation image
+//    of the textbook one, so that x = -0 gives -0 (byte 0x80) as division does.
+//  * A quotient that overflows (x/s >= 2^128, or x infinite) comes out NaN;
+//    the NaN byte marks its group of eight, which divides instead.
+// One E4M3 pair conversion per two elements (the conversion pipe is narrow).
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -24,7 +31,14 @@ namespace nvfp4 {
 namespace {
 
 constexpr int kKvThreads = 256;
-constexpr int kKvUnroll = 4;      // vectors in flight per thread
+#ifndef NVFP4_KV_UNROLL
+#define NVFP4_KV_UNROLL 4
+#endif
+#ifndef NVFP4_KV_MINB
+#define NVFP4_KV_MINB 4
+#endif
+constexpr int kKvUnroll = NVFP4_KV_UNROLL;      // vectors in flight per thread
+constexpr int kKvCtasPerSm = NVFP4_KV_MINB;     // resident CTAs per SM the grid is sized for
 
 struct KvArgs {
     const uint8_t* x;
@@ -43,6 +57,23 @@ __device__ __forceinline__ uint32_t e4m3x2(float a, float b) {
     return h;
 }
 
+// Packed pairs of binary32 values, each operation rounded to nearest even.
+__device__ __forceinline__ uint64_t f32x2(uint32_t lo, uint32_t hi) {
+    uint64_t v;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(v) : "r"(lo), "r"(hi));
+    return v;
+}
+__device__ __forceinline__ uint64_t mul_f32x2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+
 // 16-byte streaming load that does not allocate in L1.
 __device__ __forceinline__ uint4 ld_stream16(const void* p) {
     uint4 v;
@@ -52,51 +83,53 @@ __device__ __forceinline__ uint4 ld_stream16(const void* p) {
     return v;
 }
 
+struct KvConsts {
+    float s;
+    uint64_t S;      // s in both halves
+    uint64_t NR;     // -RN(1/s) in both halves
+    bool fast;       // s in [2^-92, 2^100]
+};
+
 // Eight BF16 values -> eight signed E4M3 bytes of fl32(x / s).
-__device__ __forceinline__ uint2 quantize8(const uint4 w, float s, float rlo, float rhi, bool fast) {
-    float x[8];
+__device__ __forceinline__ uint2 quantize8(const uint4 w, const KvConsts& K) {
     const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+    if (K.fast) {
+        uint32_t h[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            // -x of both elements: the BF16 bits moved into place, sign flipped
+            const uint64_t nx = f32x2(ww[i] * 0x10000u + 0x80000000u, (ww[i] & 0xFFFF0000u) ^ 0x80000000u);
+            const uint64_t q0 = mul_f32x2(nx, K.NR);
+            const uint64_t e = fma_f32x2(q0, K.S, nx);
+            const uint64_t q1 = fma_f32x2(e, K.NR, q0);
+            h[i] = e4m3x2(__uint_as_float(static_cast<uint32_t>(q1)),
+                          __uint_as_float(static_cast<uint32_t>(q1 >> 32)));
+        }
+        const uint32_t b0 = h[0] | (h[1] << 16), b1 = h[2] | (h[3] << 16);
+        // a byte whose low seven bits are all set is the NaN code (no finite
+        // quotient converts to it under saturation)
+        const uint32_t nan = (((b0 & 0x7F7F7F7Fu) + 0x01010101u) | ((b1 & 0x7F7F7F7Fu) + 0x01010101u)) &
+                             0x80808080u;
+        if (nan == 0) return make_uint2(b0, b1);
+    }
+    // out of the fast range, an overflowed quotient or a NaN input: divide
+    uint32_t b[2] = {0, 0};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        x[2 * i] = __uint_as_float(ww[i] << 16);
-        x[2 * i + 1] = __uint_as_float(ww[i] & 0xFFFF0000u);
+        const uint32_t h = e4m3x2(__fdiv_rn(__uint_as_float(ww[i] << 16), K.s),
+                                  __fdiv_rn(__uint_as_float(ww[i] & 0xFFFF0000u), K.s));
+        b[i >> 1] |= h << (16 * (i & 1));
     }
-    uint32_t lo[2], hi[2];
-    if (fast) {
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            lo[h] = e4m3x2(__fmul_rn(x[4 * h], rlo), __fmul_rn(x[4 * h + 1], rlo)) |
-                    (e4m3x2(__fmul_rn(x[4 * h + 2], rlo), __fmul_rn(x[4 * h + 3], rlo)) << 16);
-            hi[h] = e4m3x2(__fmul_rn(x[4 * h], rhi), __fmul_rn(x[4 * h + 1], rhi)) |
-                    (e4m3x2(__fmul_rn(x[4 * h + 2], rhi), __fmul_rn(x[4 * h + 3], rhi)) << 16);
-        }
-    }
-    if (!fast || ((lo[0] ^ hi[0]) | (lo[1] ^ hi[1])) != 0) {
-        // near a rounding boundary (or no usable reciprocal): divide
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            uint32_t word = 0;
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int sh = 8 * j;
-                if (!fast || (((lo[h] ^ hi[h]) >> sh) & 0xFFu))
-                    word |= (e4m3x2(__fdiv_rn(x[4 * h + j], s), 0.0f) & 0xFFu) << sh;
-                else
-                    word |= lo[h] & (0xFFu << sh);
-            }
-            lo[h] = word;
-        }
-    }
-    return make_uint2(lo[0], lo[1]);
+    return make_uint2(b[0], b[1]);
 }
 
-__global__ void __launch_bounds__(kKvThreads) kv_quantize_kernel(const KvArgs a) {
-    const float s = *a.scale;
-    const float rs = __fdiv_rn(1.0f, s);
-    const float ars = fabsf(rs);
-    const bool fast = ars >= 0x1p-125f && ars <= 0x1p125f;
-    const float rlo = __fmul_rn(rs, 1.0f - 0x1p-20f);
-    const float rhi = __fmul_rn(rs, 1.0f + 0x1p-20f);
+__global__ void __launch_bounds__(kKvThreads, kKvCtasPerSm) kv_quantize_kernel(const KvArgs a) {
+    KvConsts K;
+    K.s = *a.scale;
+    K.fast = K.s >= 0x1p-92f && K.s <= 0x1p100f;
+    const float nr = K.fast ? -__fdiv_rn(1.0f, K.s) : 0.0f;
+    K.S = f32x2(__float_as_uint(K.s), __float_as_uint(K.s));
+    K.NR = f32x2(__float_as_uint(nr), __float_as_uint(nr));
     // Walk (row, vector) pairs with carries instead of dividing; each thread
     // keeps kKvUnroll vectors in flight (loads issued before any math).
     const uint32_t vpr = a.vec_per_row;
@@ -122,7 +155,7 @@ __global__ void __launch_bounds__(kKvThreads) kv_quantize_kernel(const KvArgs a)
 #pragma unroll
         for (int u = 0; u < kKvUnroll; ++u) {
             if (r[u] < a.rows) {
-                const uint2 o = quantize8(w[u], s, rlo, rhi, fast);
+                const uint2 o = quantize8(w[u], K);
                 *reinterpret_cast<uint2*>(a.out + r[u] * a.ldo + 8 * static_cast<int64_t>(v[u])) = o;
             }
             r[u] += step_r;
@@ -180,7 +213,7 @@ extern "C" nvfp4_status nvfp4_kv_quantize_e4m3(const void* x, int64_t rows, int6
     a.scale = scale;
     const int64_t vecs = rows * (cols / 8);
     int64_t grid = (vecs + kKvThreads - 1) / kKvThreads;
-    const int64_t cap = static_cast<int64_t>(dev.sms) * 8;
+    const int64_t cap = static_cast<int64_t>(dev.sms) * kKvCtasPerSm;
     if (grid > cap) grid = cap;
     kv_quantize_kernel<<<static_cast<unsigned>(grid), kKvThreads, 0, as_stream(stream)>>>(a);
     return cuda_status(cudaGetLastError());

@@ -25,9 +25,11 @@ def all_finite_bf16(cols=512):
     return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(DEV)
 
 
-@pytest.mark.parametrize("s", [1.0, 0.37, 3.1e-3, 41.0, 2.0 ** -126, 2.0 ** 126])
+@pytest.mark.parametrize("s", [1.0, 0.37, 3.1e-3, 41.0, 2.0 ** -126, 2.0 ** 126,
+                               2.0 ** -92, 1.37 * 2.0 ** -90, 2.0 ** 100, 1.5 * 2.0 ** 100])
 def test_kv_every_bf16_value_bitexact(s):
-    # includes scales whose reciprocal leaves the normal range (division path)
+    # includes scales outside [2^-92, 2^100] (division path) and the edges of
+    # that range, where large x overflow the quotient (the group divides)
     x = all_finite_bf16()
     scale = torch.tensor([s], dtype=torch.float32, device=DEV)
     out = nv.kv_quantize(x, scale)
