@@ -1191,8 +1191,11 @@ nvfp4_status launch_gemm_pair(const uint8_t* a_codes, const uint8_t* w_codes, Ge
     return cuda_status(cudaGetLastError());
 }
 
-// Few tokens (M <= 128): operands swapped, K split over a cluster.  NT, the
-// ring depth and the split depend on M and K only.
+// Few tokens (M <= 128): operands swapped, K split over a cluster.  NT and
+// the ring depth depend on M alone, the split on K alone (the largest of 1, 2,
+// 4, 8 that leaves each CTA at least 8 k-steps), so a row's result never
+// depends on N.  Launched as a programmatic dependent of the previous grid on
+// the stream (the kernel waits for it before reading any global memory).
 nvfp4_status launch_gemm_decode(const uint8_t* a_codes, const uint8_t* w_codes,
                                 GemmArgs& args, cudaStream_t stream) {
     auto kern = nvf4_gemm_decode_kernel;
@@ -1216,7 +1219,7 @@ nvfp4_status launch_gemm_decode(const uint8_t* a_codes, const uint8_t* w_codes,
     d.nt_tok = ((args.M + 15) / 16) * 16;
     dec_config(d.nt_tok, &d.stages, &d.nparts, &d.nacc);
     d.split = 1;
-    while (d.split < kDecMaxSplit && args.k_steps / (2 * d.split) >= 4) d.split *= 2;
+    while (d.split < kDecMaxSplit && args.k_steps / (2 * d.split) >= 8) d.split *= 2;
     d.g.m_tiles = 1;
     d.g.n_tiles = (args.N + kBM - 1) / kBM;
     const uint32_t smem = dec_layout(d.nt_tok, d.stages, d.nparts).bytes;
@@ -1225,13 +1228,15 @@ nvfp4_status launch_gemm_decode(const uint8_t* a_codes, const uint8_t* w_codes,
     cfg.blockDim = dim3(kDecThreads, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = static_cast<unsigned>(d.split);
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 1;            // the occupancy query takes the cluster shape only
     // persistent: as many clusters as can be resident at once
     // (racing threads may both measure; they store the same value)
     std::atomic<int>& cached = max_clusters[devid][d.split][d.nt_tok / 16];
@@ -1244,6 +1249,7 @@ nvfp4_status launch_gemm_decode(const uint8_t* a_codes, const uint8_t* w_codes,
     }
     const int clusters = d.g.n_tiles < slots ? d.g.n_tiles : slots;
     cfg.gridDim = dim3(static_cast<unsigned>(clusters * d.split), 1, 1);
+    cfg.numAttrs = 2;
     CUtensorMap tw, tx;
     if (!make_code_map(&tw, w_codes, args.N, args.K / 2, kBM)) return NVFP4_ERR_CUDA;
     if (!make_code_map(&tx, a_codes, args.M, args.K / 2, d.nt_tok)) return NVFP4_ERR_CUDA;

@@ -9,7 +9,9 @@
 //     padded to NT = 16..128, on its N side, so a tile is 128 outputs wide in n
 //     whatever the token count.
 //   * K is split over a cluster of S CTAs (S = 1, 2, 4 or 8, chosen from K
-//     alone); each CTA accumulates its fixed K slice of a tile in TMEM.
+//     alone: the largest that leaves every CTA at least 8 k-steps, since
+//     each further split costs a partial-sum exchange per tile); each CTA
+//     accumulates its fixed K slice of a tile in TMEM.
 //   * Persistent: one cluster per scheduling slot; cluster c takes weight
 //     tiles c, c + C, c + 2C, ...  The shared-memory ring runs across tiles, so
 //     weight loads stay in flight while earlier tiles drain.
@@ -23,6 +25,17 @@
 //     warps (one per TMEM lane quarter) instead of tcgen05.cp, writing the same
 //     replicated layout the copy would: lane l of every quarter holds bytes
 //     [16 l, 16 l + 16) of each 512-byte scale atom in four columns.
+//
+//   * Start-up: warp 0 sets up the barriers (one lane per ring stage) and
+//     starts the weight stream without waiting for the TMEM allocation; the
+//     feed-loop waits of the producer and the MMA warp spin on the phase
+//     instead of suspending, so the two handshakes of every stage add no
+//     wake-up latency.
+//   * Launched as a programmatic dependent: each CTA lets the next grid on
+//     the stream launch at once, so that grid's CTAs set up on the SMs this
+//     one leaves while its last tiles drain; every role that reads global
+//     memory first waits for the previous grid (griddepcontrol.wait), so
+//     stream order holds for all data.
 //
 // Roles (14 warps): 0 TMA producer; 1 TMEM owner and MMA issuer; 2..5 scale
 // writers; 6..9 pushers (accumulator -> owners' shared memory); 10..13
@@ -161,6 +174,7 @@ nvf4_gemm_decode_kernel(const __grid_constant__ CUtensorMap tmap_w,
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    grid_launch_dependents();
     const int rank = static_cast<int>(cluster_ctarank());
     const int cluster_id = blockIdx.x / S;
     const int num_clusters = gridDim.x / S;
@@ -168,34 +182,43 @@ nvf4_gemm_decode_kernel(const __grid_constant__ CUtensorMap tmap_w,
     const int k_end = ((rank + 1) * args.k_steps) / S;
     const int R = kBM / S;                  // rows of a tile owned by each CTA
 
-    if (threadIdx.x == 0) {
-        for (int i = 0; i < STAGES; ++i) {
-            mbar_init(&full[i], 1);
-            mbar_init(&empty[i], 1);
-            mbar_init(&sf_ready[i], 4);
+    if (warp == 0) {
+        // lane i sets up the barriers of ring stage i, accumulator i and
+        // partial buffer i; the warp then goes straight to the weight stream
+        // (named barrier 2: arrive only), the others wait for the set-up and
+        // the TMEM allocation
+        if (lane < STAGES) {
+            mbar_init(&full[lane], 1);
+            mbar_init(&empty[lane], 1);
+            mbar_init(&sf_ready[lane], 4);
         }
-        for (int i = 0; i < kDecMaxAcc; ++i) {
-            mbar_init(&tmem_full[i], 1);
-            mbar_init(&tmem_empty[i], 4);         // the four pusher warps
+        if (lane < kDecMaxAcc) {
+            mbar_init(&tmem_full[lane], 1);
+            mbar_init(&tmem_empty[lane], 4);      // the four pusher warps
         }
-        for (int i = 0; i < NPART; ++i) {
-            mbar_init(&part_full[i], kBM);        // R rows from each of the S CTAs
-            mbar_init(&part_free[i], 4 * S);      // the 4 reducer warps of each of the S CTAs
+        if (lane < NPART) {
+            mbar_init(&part_full[lane], kBM);     // R rows from each of the S CTAs
+            mbar_init(&part_free[lane], 4 * S);   // the 4 reducer warps of each of the S CTAs
         }
-        mbar_init(drain, 1);
-        *s_abort = 0;
+        if (lane == 0) {
+            mbar_init(drain, 1);
+            *s_abort = 0;
+            prefetch_tmap(&tmap_w);
+            prefetch_tmap(&tmap_x);
+        }
         fence_mbar_init();
-        prefetch_tmap(&tmap_w);
-        prefetch_tmap(&tmap_x);
+        __syncwarp();
+        named_barrier_arrive(2, kDecThreads);
+    } else {
+        if (warp == 1) {
+            tmem_alloc(s_tmem_base, kDecTmemCols);
+            tmem_relinquish();
+        }
+        tc_fence_before();
+        named_barrier_sync(2, kDecThreads);
+        tc_fence_after();
     }
-    if (warp == 1) {
-        tmem_alloc(s_tmem_base, kDecTmemCols);
-        tmem_relinquish();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem_base = *s_tmem_base;
+    const uint32_t tmem_base = warp == 0 ? 0u : *s_tmem_base;   // the producer needs none
     // Cross-CTA set-up without holding up the weight stream: every thread
     // arrives on the cluster barrier now; the roles that touch a peer's
     // shared memory or barriers (pushers, reducers) wait on it before their
@@ -216,6 +239,7 @@ nvf4_gemm_decode_kernel(const __grid_constant__ CUtensorMap tmap_w,
 
     if (warp == 0) {
         // ---------------- TMA producer (whole warp; one elected lane issues) ----------------
+        grid_dependency_wait();     // weights, tokens and scales may come from the previous grid
         const uint64_t pol_w = l2_policy_evict_first();   // each weight byte is read once
         const uint64_t pol_x = l2_policy_evict_last();    // tokens are read by every tile
         const uint32_t full_bytes = kBM * kBKBytes + NT * kBKBytes + 2 * kAtomsPerStep * kAtom;
@@ -229,7 +253,7 @@ nvf4_gemm_decode_kernel(const __grid_constant__ CUtensorMap tmap_w,
                                               static_cast<size_t>(k_begin) * kAtomsPerStep) * kAtom;
             const uint8_t* xsf = args.a_sf + static_cast<size_t>(k_begin) * kAtomsPerStep * kAtom;
             for (int kb = k_begin; kb < k_end; ++kb) {
-                if (!mbar_wait_warp(&empty[stage], phase ^ 1u, args.timeout_ns, s_abort, args.status)) {
+                if (!mbar_spin_warp(&empty[stage], phase ^ 1u, args.timeout_ns, s_abort, args.status)) {
                     ok = false;
                     break;
                 }
@@ -275,7 +299,7 @@ nvf4_gemm_decode_kernel(const __grid_constant__ CUtensorMap tmap_w,
         int stage = 0, acc = 0;
         uint32_t phase = 0, acc_phase = 0;
         for (int nt = cluster_id; nt < args.n_tiles && ok; nt += num_clusters) {
-            if (!mbar_wait_warp(&tmem_empty[acc], acc_phase ^ 1u, args.timeout_ns, s_abort,
+            if (!mbar_spin_warp(&tmem_empty[acc], acc_phase ^ 1u, args.timeout_ns, s_abort,
                                 args.status)) {
                 ok = false;
                 break;
@@ -283,7 +307,7 @@ nvf4_gemm_decode_kernel(const __grid_constant__ CUtensorMap tmap_w,
             tc_fence_after();
             const uint32_t d_tmem = tmem_base + acc * ACC_STRIDE;
             for (int kb = k_begin; kb < k_end; ++kb) {
-                if (!mbar_wait_warp(&sf_ready[stage], phase, args.timeout_ns, s_abort, args.status)) {
+                if (!mbar_spin_warp(&sf_ready[stage], phase, args.timeout_ns, s_abort, args.status)) {
                     ok = false;
                     break;
                 }
@@ -402,14 +426,15 @@ nvf4_gemm_decode_kernel(const __grid_constant__ CUtensorMap tmap_w,
             tc_fence_after();
             const uint32_t dst = part_owner + static_cast<uint32_t>(
                 pb * dec_part_bytes(NT) + ((rank * NT) * R + rr) * 4);
-            for (int c = 0; c < NT; c += 16) {
+            for (int c = 0; c < args.M; c += 16) {      // the columns of real tokens only
                 uint32_t r[16];
                 tmem_ld_16cols(tmem_base + lane_base + acc * ACC_STRIDE + c, r);
                 tmem_ld_wait();
 #pragma unroll
                 for (int j = 0; j < 16; ++j)
-                    st_shared_cluster_f32(dst + static_cast<uint32_t>((c + j) * R * 4),
-                                          __uint_as_float(r[j]));
+                    if (c + j < args.M)
+                        st_shared_cluster_f32(dst + static_cast<uint32_t>((c + j) * R * 4),
+                                              __uint_as_float(r[j]));
             }
             tc_fence_before();
             __syncwarp();
@@ -423,6 +448,7 @@ nvf4_gemm_decode_kernel(const __grid_constant__ CUtensorMap tmap_w,
         // The results stay in registers until this warp has released the
         // partial buffer, so that release never waits on the global stores.
         const int red_tid = threadIdx.x - 10 * 32;
+        grid_dependency_wait();     // the activation scale may come from the previous grid
         // the segment table and gate parameters are the reducers' alone
         if (red_tid < NVFP4_MAX_SEGMENTS) fill_seg_table(seg_tab, args, red_tid);
         stage_gate_params(seg_tab, args, red_tid, 128);

@@ -198,6 +198,32 @@ __device__ __forceinline__ bool mbar_wait_warp_pipe(uint64_t* bar, uint32_t pari
     return __shfl_sync(0xFFFFFFFFu, ok, 0) != 0;
 }
 
+// Whole-warp bounded wait that never suspends: every lane tests the phase
+// (one broadcast read) until it completes.  For the feed loop of the
+// few-token GEMM, where each stage crosses two handshakes and the wake-up
+// latency of a suspended try_wait would add to every one of them.  Same
+// limits as mbar_wait_bounded; all 32 lanes must call it.
+__device__ __forceinline__ bool mbar_spin_warp(uint64_t* bar, uint32_t parity, uint64_t limit_ns,
+                                               volatile int* abort, int* dev_status) {
+    if (__shfl_sync(0xFFFFFFFFu, mbar_test_wait(bar, parity) ? 1 : 0, 0)) return true;
+    const uint64_t t0 = clock_cycles();
+    const uint64_t lim = limit_cycles(limit_ns);
+    while (true) {
+        if (__shfl_sync(0xFFFFFFFFu, mbar_test_wait(bar, parity) ? 1 : 0, 0)) return true;
+        int stop = 0;
+        if ((threadIdx.x & 31) == 0) {
+            if (*abort) {
+                stop = 1;
+            } else if (clock_cycles() - t0 > lim) {
+                *abort = 1;
+                atomicExch(dev_status, kDevTimeout);
+                stop = 1;
+            }
+        }
+        if (__shfl_sync(0xFFFFFFFFu, stop, 0)) return false;
+    }
+}
+
 // Bounded wait by the whole warp: lane 0 polls, the outcome is broadcast.
 __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, uint64_t limit_ns,
                                                volatile int* abort, int* dev_status) {
@@ -448,6 +474,24 @@ __device__ __forceinline__ void cluster_arrive() {
 
 __device__ __forceinline__ void cluster_wait() {
     asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Arrive on named barrier `id` without waiting; the calling thread's earlier
+// writes are visible to the threads that wait on the barrier.
+__device__ __forceinline__ void named_barrier_arrive(int id, int count) {
+    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// Programmatic dependent launch.  launch_dependents lets the next grid on the
+// stream (when it was launched as a programmatic dependent) be scheduled now,
+// so its CTAs start on SMs as this grid's CTAs leave them; dependency_wait
+// returns once the previous grid has completed and its memory writes are
+// visible (at once when this grid was launched the ordinary way).
+__device__ __forceinline__ void grid_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void grid_dependency_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 // Barrier among `count` threads of the CTA on named barrier `id` (1..15).

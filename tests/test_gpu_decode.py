@@ -20,21 +20,23 @@ DEV = "cuda"
 
 
 def k_split(K):
-    """Cluster size the library picks for K (a function of K alone)."""
+    """Cluster size the library picks for K (a function of K alone: the largest
+    of 1, 2, 4, 8 that leaves every CTA at least 8 k-steps of 256)."""
     ks, s = (K + 255) // 256, 1
-    while s < 8 and ks // (2 * s) >= 4:
+    while s < 8 and ks // (2 * s) >= 8:
         s *= 2
     return s
 
 
 @pytest.mark.parametrize("M,N,K", [
     (64, 130, 96),       # one k-step, K % 64 == 32, split 1
-    (3, 200, 2048),      # split 2, one full ring
-    (17, 264, 4160),     # split 4, 4..5 steps in a ring of 4, last step one atom
-    (128, 384, 2304),    # token width 128, ring of 3 wraps, split 2
-    (100, 520, 5120),    # token width 112, split 4
+    (3, 200, 2048),      # split 1, one full ring
+    (17, 264, 4160),     # split 2, 8..9 steps in a ring of 4, last step one atom
+    (9, 392, 8224),      # split 4, K % 64 == 32, 8..9 steps per CTA
+    (128, 384, 2304),    # token width 128, ring of 3 wraps, split 1
+    (100, 520, 5120),    # token width 112, split 2
     (45, 136, 17440),    # split 8, K % 64 == 32, ring wraps twice
-    (1, 5, 7168),        # one token, five outputs
+    (1, 5, 7168),        # one token, five outputs, split 2
 ])
 def test_decode_shapes(M, N, K):
     assert k_split(K) in (1, 2, 4, 8)
@@ -56,7 +58,7 @@ def test_decode_shapes(M, N, K):
 
 
 def test_decode_splits_cover_1_2_4_8():
-    assert sorted({k_split(K) for K in (96, 2048, 4160, 17440)}) == [1, 2, 4, 8]
+    assert sorted({k_split(K) for K in (96, 4160, 8224, 17440)}) == [1, 2, 4, 8]
 
 
 @pytest.mark.parametrize("M", [1, 24, 128])
