@@ -458,6 +458,7 @@ nvf4_gemm_decode_kernel(const __grid_constant__ CUtensorMap tmap_w,
         const int rg = red_tid % ngroups;
         const int tstep = 128 / ngroups;
         const int t_first = red_tid / ngroups;
+        int sg_first = 0;           // segment of this thread's first row: rows only grow from tile to tile
         int i = 0;
         for (int nt = cluster_id; nt < args.n_tiles; nt += num_clusters, ++i) {
             const int pb = i % NPART;
@@ -467,10 +468,11 @@ nvf4_gemm_decode_kernel(const __grid_constant__ CUtensorMap tmap_w,
             if (!__all_sync(0xFFFFFFFFu, got)) break;
             const float* pbuf = part + pb * (dec_part_bytes(NT) / 4);
             const int n0 = nt * kBM + rank * R + 4 * rg;
+            while (sg_first < args.nseg - 1 && n0 >= s_seg_end[sg_first]) ++sg_first;
             float al[4];
+            int sgi = sg_first;
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
-                int sgi = 0;
                 while (sgi < args.nseg - 1 && n0 + u >= s_seg_end[sgi]) ++sgi;
                 al[u] = s_seg_alpha[sgi];
             }

@@ -37,6 +37,8 @@ def k_split(K):
     (100, 520, 5120),    # token width 112, split 2
     (45, 136, 17440),    # split 8, K % 64 == 32, ring wraps twice
     (1, 5, 7168),        # one token, five outputs, split 2
+    (2, 300, 5120),      # split 2, two tokens
+    (8, 136, 17440),     # split 8, eight tokens, ragged N
 ])
 def test_decode_shapes(M, N, K):
     assert k_split(K) in (1, 2, 4, 8)

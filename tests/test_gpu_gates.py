@@ -1,7 +1,8 @@
 """GPU parity of the gate epilogue of the fused Gated DeltaNet input
 projection (evolve.pub, Key claims under review, second bullet: log-space
 softplus/exponential decay gate and sigmoid write strength), in all three
-GEMM kernels (M = 7: few-token kernel; 200: one-CTA kernel; 300: CTA pairs).
+GEMM kernels (M = 1 and 7: few-token kernel; 200: one-CTA kernel; 300: CTA
+pairs).
 
 Tolerance, derived from the arithmetic.  Before the gate function the kernel
 holds v = fl32(acc * alpha) with |v - y64| <= e_v = 2^-23 |y64| + K 2^-22 S
@@ -52,7 +53,7 @@ def build(layout, K, seed0):
     return ws, fw, acts, params
 
 
-@pytest.mark.parametrize("M", [7, 200, 300])
+@pytest.mark.parametrize("M", [1, 7, 200, 300])
 @pytest.mark.parametrize("layout", ["gdn", "ragged"])
 def test_gate_epilogue_matches_oracle(M, layout):
     K = 512
