@@ -9,9 +9,12 @@
 // largest module scale as the common one is the reading taken here (it never
 // saturates a scale); the pages give no formula.
 //
-// Memory-bound and tiny (N*K/16 bytes, read and written once): a grid-stride
-// loop over 16-byte chunks; each thread finds the row of each byte (linear
-// or tensor-core scale layout), that row's module, and rescales the byte.
+// Memory-bound and small (N*K/16 bytes, read and written once): a grid-stride
+// loop over 16-byte chunks.  A chunk's rows come from one division per chunk:
+// in the tensor-core layout its bytes are four scales of each of four rows
+// (32 rows apart), in the linear layout one run of consecutive rows; the
+// module of each row is found by walking the segment table forward from the
+// previous row's.  Bytes are decoded, rescaled and encoded in pairs.
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -23,6 +26,7 @@ namespace nvfp4 {
 namespace {
 
 constexpr int kHarmThreads = 256;
+static_assert(kHarmThreads >= NVFP4_MAX_SEGMENTS, "one thread per module scale");
 
 struct HarmArgs {
     uint8_t* sf;
@@ -36,69 +40,100 @@ struct HarmArgs {
     float* g_common;
 };
 
-// E4M3 byte -> float, exact (every E4M3 value is an FP16 value).  The byte
-// fills both halves of the pair, so either half of the result holds it.
-__device__ __forceinline__ float e4m3_value_f32(uint32_t byte) {
+// Two E4M3 bytes (low byte first) -> two floats, exact (every E4M3 value is
+// an FP16 value).
+__device__ __forceinline__ float2 e4m3x2_values(uint32_t pair) {
     uint32_t h2;
-    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(static_cast<uint16_t>(byte | (byte << 8))));
-    return __half2float(__ushort_as_half(static_cast<unsigned short>(h2 & 0xFFFFu)));
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(static_cast<uint16_t>(pair)));
+    return make_float2(__half2float(__ushort_as_half(static_cast<unsigned short>(h2 & 0xFFFFu))),
+                       __half2float(__ushort_as_half(static_cast<unsigned short>(h2 >> 16))));
 }
 
-// Non-negative float -> UE4M3 byte, round to nearest even, saturating at 448.
-__device__ __forceinline__ uint32_t e4m3_encode_rne(float s) {
+// Two non-negative floats -> two UE4M3 bytes (lo in the low byte), round to
+// nearest even, saturating at 448.
+__device__ __forceinline__ uint32_t e4m3x2_encode_rne(float lo, float hi) {
     uint16_t h;
-    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(h) : "f"(0.0f), "f"(s));
-    return h & 0xFFu;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(h) : "f"(hi), "f"(lo));
+    return h;
 }
 
-// Row of the scale byte at offset o of the layout.
-__device__ __forceinline__ int64_t row_of(int64_t o, const HarmArgs& a) {
-    if (a.layout == NVFP4_SF_TCGEN05) {
-        // 512-byte atoms of 128 rows x 4 scales: inner offset
-        // (r % 32) * 16 + ((r / 32) % 4) * 4 + c % 4
-        const int64_t blk = o / a.block_bytes;
-        const int inner = static_cast<int>(o & 511);
-        return blk * 128 + ((inner & 15) >> 2) * 32 + (inner >> 4);
-    }
-    return o / a.sfcols;
+// Module of row r, walking forward from segment s (rows only grow).
+__device__ __forceinline__ int seg_from(int s, int64_t r, int nseg, const int* end) {
+    while (s < nseg - 1 && r >= end[s]) ++s;
+    return s;
 }
 
 __global__ void __launch_bounds__(kHarmThreads) harmonize_kernel(const HarmArgs a) {
+    __shared__ float s_g[NVFP4_MAX_SEGMENTS];
     __shared__ float s_ratio[NVFP4_MAX_SEGMENTS];
     __shared__ int s_end[NVFP4_MAX_SEGMENTS];
-    if (threadIdx.x == 0) {
-        float gc = *a.seg_g[0];
-        for (int i = 1; i < a.nseg; ++i) gc = fmaxf(gc, *a.seg_g[i]);
-        for (int i = 0; i < NVFP4_MAX_SEGMENTS; ++i) {
-            s_ratio[i] = (i < a.nseg) ? __fdiv_rn(*a.seg_g[i], gc) : 1.0f;
-            s_end[i] = (i < a.nseg) ? a.seg_end[i] : 0x7FFFFFFF;
-        }
-        if (blockIdx.x == 0) *a.g_common = gc;
+    // the module scales are read in parallel (one dependent load per CTA, not nseg)
+    if (threadIdx.x < a.nseg) s_g[threadIdx.x] = *a.seg_g[threadIdx.x];
+    __syncthreads();
+    if (threadIdx.x < NVFP4_MAX_SEGMENTS) {
+        float gc = s_g[0];
+        for (int i = 1; i < a.nseg; ++i) gc = fmaxf(gc, s_g[i]);
+        const int i = threadIdx.x;
+        s_ratio[i] = (i < a.nseg) ? __fdiv_rn(s_g[i], gc) : 1.0f;
+        s_end[i] = (i < a.nseg) ? a.seg_end[i] : 0x7FFFFFFF;
+        if (blockIdx.x == 0 && i == 0) *a.g_common = gc;
     }
     __syncthreads();
     const int64_t stride = static_cast<int64_t>(gridDim.x) * kHarmThreads * 16;
     for (int64_t o = (static_cast<int64_t>(blockIdx.x) * kHarmThreads + threadIdx.x) * 16;
          o < a.nbytes; o += stride) {
-        uint8_t v[16];
+        uint32_t w[4];
         const bool whole = o + 16 <= a.nbytes;
         if (whole) {
-            *reinterpret_cast<uint4*>(v) = *reinterpret_cast<const uint4*>(a.sf + o);
+            const uint4 q = *reinterpret_cast<const uint4*>(a.sf + o);
+            w[0] = q.x, w[1] = q.y, w[2] = q.z, w[3] = q.w;
         } else {
-            for (int k = 0; k < 16; ++k) v[k] = (o + k < a.nbytes) ? a.sf[o + k] : 0;
+            for (int j = 0; j < 4; ++j) {
+                w[j] = 0;
+                for (int b = 0; b < 4; ++b)
+                    if (o + 4 * j + b < a.nbytes) w[j] |= static_cast<uint32_t>(a.sf[o + 4 * j + b]) << (8 * b);
+            }
+        }
+        // module ratio of every byte of the chunk
+        float ratio[16];
+        if (a.layout == NVFP4_SF_TCGEN05) {
+            // 512-byte atoms of 128 rows x 4 scales, inner offset
+            // (r % 32) * 16 + ((r / 32) % 4) * 4 + c % 4: word j of the chunk
+            // holds the four scales of row 32 j + (inner / 16) of the block
+            const int64_t r0 = (o / a.block_bytes) * 128 + ((o & 511) >> 4);
+            int s = 0;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                s = seg_from(s, r0 + 32 * j, a.nseg, s_end);   // padding rows hold 0 and stay 0
+#pragma unroll
+                for (int b = 0; b < 4; ++b) ratio[4 * j + b] = s_ratio[s];
+            }
+        } else {
+            // consecutive bytes of consecutive rows, sfcols per row
+            int64_t r = o / a.sfcols;
+            int64_t left = (r + 1) * a.sfcols - o;       // bytes of row r from o on
+            int s = seg_from(0, r, a.nseg, s_end);
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+                while (k >= left) {
+                    ++r;
+                    left += a.sfcols;
+                    s = seg_from(s, r, a.nseg, s_end);
+                }
+                ratio[k] = s_ratio[s];
+            }
         }
 #pragma unroll
-        for (int k = 0; k < 16; ++k) {
-            const int64_t r = row_of(o + k, a);
-            int s = 0;
-            while (s < a.nseg - 1 && r >= s_end[s]) ++s;
-            // padding rows of the tensor-core layout hold 0 and stay 0
-            v[k] = static_cast<uint8_t>(e4m3_encode_rne(__fmul_rn(e4m3_value_f32(v[k]), s_ratio[s])));
+        for (int j = 0; j < 4; ++j) {
+            const float2 lo = e4m3x2_values(w[j] & 0xFFFFu), hi = e4m3x2_values(w[j] >> 16);
+            w[j] = e4m3x2_encode_rne(__fmul_rn(lo.x, ratio[4 * j]), __fmul_rn(lo.y, ratio[4 * j + 1])) |
+                   (e4m3x2_encode_rne(__fmul_rn(hi.x, ratio[4 * j + 2]), __fmul_rn(hi.y, ratio[4 * j + 3])) << 16);
         }
         if (whole) {
-            *reinterpret_cast<uint4*>(a.sf + o) = *reinterpret_cast<const uint4*>(v);
+            *reinterpret_cast<uint4*>(a.sf + o) = make_uint4(w[0], w[1], w[2], w[3]);
         } else {
             for (int k = 0; k < 16; ++k)
-                if (o + k < a.nbytes) a.sf[o + k] = v[k];
+                if (o + k < a.nbytes) a.sf[o + k] = static_cast<uint8_t>(w[k >> 2] >> (8 * (k & 3)));
         }
     }
 }

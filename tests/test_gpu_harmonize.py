@@ -54,8 +54,9 @@ def test_harmonize_tcgen05_layout_bitexact(K):
     assert max(float(np_f32(g)[0]) for g in fw.g_list) == gc
 
 
-def test_harmonize_linear_layout_bitexact():
-    K = 160                                        # 10 scales per row: 16-byte chunks span rows
+@pytest.mark.parametrize("K", [160, 32])
+def test_harmonize_linear_layout_bitexact(K):
+    # 10 scales per row: 16-byte chunks span two rows; 2 per row: a chunk spans eight
     ws = modules(K, seed0=70)
     N = sum(ROWS)
     codes = torch.empty(N, K // 2, dtype=torch.uint8, device=DEV)
