@@ -16,7 +16,8 @@
 //     tiles c, c + C, c + 2C, ...  The shared-memory ring runs across tiles, so
 //     weight loads stay in flight while earlier tiles drain.
 //   * Split-K reduction through distributed shared memory: every CTA pushes its
-//     FP32 partial of each row to the CTA owning that row (128/S rows each);
+//     FP32 partial of each row (the real tokens' columns only) to the CTA
+//     owning that row (128/S rows each);
 //     the owner adds the S partials in rank order 0..S-1 (a fixed order: the
 //     result depends on neither N nor the segment table nor timing), applies
 //     alpha and writes BF16.  Handshakes are mbarriers arrived on across the
@@ -25,7 +26,6 @@
 //     warps (one per TMEM lane quarter) instead of tcgen05.cp, writing the same
 //     replicated layout the copy would: lane l of every quarter holds bytes
 //     [16 l, 16 l + 16) of each 512-byte scale atom in four columns.
-//
 //   * Start-up: warp 0 sets up the barriers (one lane per ring stage) and
 //     starts the weight stream without waiting for the TMEM allocation; the
 //     feed-loop waits of the producer and the MMA warp spin on the phase
