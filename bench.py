@@ -625,7 +625,12 @@ def run_ours(args, dev, world, rank):
         "components_us": {"global_scale+quantize": round(float(np.mean(quant_ms)) * 1e3, 2),
                           "fused_gemm": round(gemm_avg_ms * 1e3, 2)},
         "roofline": roofline, "quantizer": quantizer, "e2e": e2e,
-        "decode_sweep": decode, "mlp_32k": mlp_line,
+        "decode_sweep": decode,
+        "decode_sweep_method": ("us: CUDA-graph replay of back-to-back launches over rotating weight "
+                                "copies (together > 2 x L2); each launch is a programmatic dependent "
+                                "of the one before (its set-up overlaps that launch's end, every read "
+                                "waits for it); us_eager: one Python call at a time"),
+        "mlp_32k": mlp_line,
         "harmonize": harm, "kv_cache_fp8": kv, "gate_epilogue": gates,
         "gpu_launches": 3 * args.steps,
         "clocks": clk.summary(),
