@@ -102,7 +102,9 @@ __host__ __device__ constexpr DecLayout dec_layout(int nt_tok, int stages, int n
 
 // Accumulators, partial buffers and ring depth for a token width.
 __host__ __device__ constexpr void dec_config(int nt_tok, int* stages, int* nparts, int* nacc) {
-    const int np = nt_tok <= 32 ? 4 : (nt_tok <= 64 ? 2 : 1);
+    // four partial buffers only where they still leave the ring its eight
+    // stages (width 16); from width 32 two, so the ring keeps seven stages
+    const int np = nt_tok <= 16 ? 4 : (nt_tok <= 64 ? 2 : 1);
     int st = static_cast<int>((kDecStageBudget - np * dec_part_bytes(nt_tok)) / dec_stage_bytes(nt_tok));
     st = st > kDecMaxStages ? kDecMaxStages : st;
     *stages = st < 2 ? 2 : st;
