@@ -742,6 +742,8 @@ PROFILE_CASES = {
     "gemm_decode_m1": "fused GEMM, X [1,5120] x W [24640,5120]",
     "quantize_act": "quantizer on the activation [32768,5120]",
     "global_scale_act": "global scale of the activation [32768,5120]",
+    "kv_quantize": "FP8 E4M3 KV cache: BF16 [65536,2048] -> bytes, calibrated per-tensor scale",
+    "harmonize_gdn": "harmonisation of the fused GDN weight's scales [24704,5120], in place",
 }
 
 
@@ -782,6 +784,18 @@ def run_profile_case(case: str, launches: int) -> None:
                 nv.quantize(x, g, nv.SF_TCGEN05, codes, sf)
             else:
                 nv.global_scale(x, g, amax)
+    elif case == "kv_quantize":
+        x = synth.student_t_activations(65536, 2048, seed=30, device=dev)
+        s = nv.kv_scale(x[:4096])
+        out = torch.empty(65536, 2048, dtype=torch.uint8, device=dev)
+        torch.cuda.synchronize()
+        for _ in range(launches):
+            nv.kv_quantize(x, s, out)
+    elif case == "harmonize_gdn":
+        fw = nv.FusedWeight.from_modules([w for _, w in synth.gdn_weights(synth.GDN_MODULES, device=dev)])
+        torch.cuda.synchronize()
+        for _ in range(launches):
+            nv.harmonize(fw)
     else:
         raise SystemExit(f"unknown profile case {case!r}; cases: {', '.join(PROFILE_CASES)}")
     torch.cuda.synchronize()
