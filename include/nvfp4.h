@@ -204,6 +204,11 @@ nvfp4_status nvfp4_quantize_slice(const void* x, int64_t rows, int64_t cols, int
  * nvfp4_quantize like activations.  No bias.
  * Requirements: K % 32 == 0, K >= 32; ldy >= N, ldy % 8 == 0; all pointers
  * 16-byte aligned.  M == 0 or N == 0 enqueues nothing.
+ * Few tokens (M <= 128): the kernel is launched as a programmatic dependent
+ * of the previous kernel on the stream.  Its CTAs may start before that
+ * kernel has finished, but they read no memory until it has completed, so
+ * stream order holds for every operand and for y.  Its FP32 summation order
+ * depends on K alone, so a row's result does not depend on N.
  * Errors: NVFP4_ERR_INVALID_ARG (null pointer, negative size, a scale inside
  * y), NVFP4_ERR_ALIGNMENT (ldy or a pointer), NVFP4_ERR_UNSUPPORTED_SHAPE (K,
  * the size bounds), NVFP4_ERR_DEVICE (not sm_100), CUDA errors.  A bounded
