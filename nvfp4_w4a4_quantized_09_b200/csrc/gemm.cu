@@ -894,7 +894,10 @@ nvf4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a,
             if (lane == 0 && mag) atomicMax(&args.h_ws[0], mag << 16);
         } else {
         // Each warp owns TMEM lane quarter q (32 rows) and half of the 256
-        // columns.  Per 32-column chunk: alpha and gates in FP32, BF16 RNE,
+        // columns -- or, in a tile whose columns end within its first half
+        // (the last tile when N % 256 <= 128), every other 32-column chunk of
+        // that half, so both warps of a quarter share its work (there the
+        // gate segments of the fused GDN projection sit).  Per 32-column chunk: alpha and gates in FP32, BF16 RNE,
         // the 32 x 32 tile written into the warp's staging buffer in the
         // 64-byte swizzle (conflict-free: lane i's row is 64 bytes at
         // 64 i, its 16-byte pieces permuted by (i / 2) % 4), then one TMA store
@@ -913,6 +916,10 @@ nvf4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a,
         for (int t = pair; t < total_tiles; t += npairs, ++i) {
             int mt, nt;
             tile_coords(t, args, mt, nt);
+            // chunk ch of this warp is column chunk chunk_of(ch) of the tile
+            const bool narrow = nt * BN + kHalf >= args.N;
+            auto chunk_of = [&](int ch) { return narrow ? half + 2 * ch : half * kChunks + ch; };
+            const int nch = narrow ? kChunks / 2 : kChunks;
             int ok = 1;
             if (lane == 0)
                 ok = mbar_wait_bounded(tmem_full, i & 1, args.timeout_ns, s_abort, args.status);
@@ -920,9 +927,10 @@ nvf4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a,
             if (!ok) break;
             tc_fence_after();
             uint32_t r[kChunks][32];
-            const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + half * kHalf;
+            const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
 #pragma unroll
-            for (int ch = 0; ch < kChunks; ++ch) tmem_ld_32cols(taddr + ch * 32, r[ch]);
+            for (int ch = 0; ch < kChunks; ++ch)
+                if (ch < nch) tmem_ld_32cols(taddr + chunk_of(ch) * 32, r[ch]);
             tmem_ld_wait();
             tc_fence_before();
             __syncwarp();
@@ -933,7 +941,8 @@ nvf4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a,
             if (m0 >= args.M) continue;                                        // warp-uniform
 #pragma unroll
             for (int ch = 0; ch < kChunks; ++ch) {
-                const int n0 = nt * BN + half * kHalf + ch * 32;
+                if (ch >= nch) break;                                          // warp-uniform
+                const int n0 = nt * BN + chunk_of(ch) * 32;
                 if (n0 >= args.N) break;                                       // warp-uniform
                 int s0 = 0;
                 while (s0 < args.nseg - 1 && n0 >= s_seg_end[s0]) ++s0;
